@@ -1,0 +1,143 @@
+"""Seeded synthetic inputs for the attention forward.
+
+This module only draws numbers and rounds them to bf16; it holds none of the
+attention arithmetic.  Both the CUDA path (through the binding) and the CPU
+oracle consume what it produces, so neither has to import the other.
+
+Recipe (the same for every workload):
+  * ``numpy.random.default_rng(seed)`` (PCG64) draws fp32 ``standard_normal``
+    in the order Q, K, V, each of shape ``[B, H, N, d]`` (K and V use the KV
+    head count);
+  * K is multiplied by ``k_scale`` before rounding (2.0 for the GQA workload,
+    an exact power-of-two scaling);
+  * every tensor is rounded to bf16 with round-to-nearest-even; the fp32 copy
+    that the oracle reads holds exactly those bf16 values;
+  * key-padded workloads then draw ``seqlens = rng.integers(lo, hi + 1, B)``
+    from the same generator;
+  * sampled-row checks draw their query rows from ``default_rng(seed + 100)``
+    without replacement, independently per (batch, head).
+"""
+from __future__ import annotations
+
+import dataclasses
+import math
+
+import numpy as np
+
+
+@dataclasses.dataclass(frozen=True)
+class Workload:
+    name: str
+    B: int
+    Hq: int
+    Hkv: int
+    N: int
+    d: int
+    causal: bool
+    seed: int
+    k_scale: float = 1.0
+    seqlen_range: tuple[int, int] | None = None  # inclusive [lo, hi] key lengths
+    sample_rows: int | None = None  # oracle rows per head for large cases
+
+    @property
+    def scale(self) -> float:
+        return 1.0 / math.sqrt(self.d)
+
+
+# The five workloads the pages' problem statement is measured on (shapes of
+# GPT-2 small, BERT-large with padding, a Llama-style GQA layer and a long
+# context), plus the tiny exact case.
+TINY = Workload("tiny_b1_h2_n256_d64", 1, 2, 2, 256, 64, False, seed=1)
+GPT2 = Workload("gpt2_causal_b8_h12_n1024_d64", 8, 12, 12, 1024, 64, True, seed=2)
+BERT = Workload("bert_padded_b16_h16_n512_d64", 16, 16, 16, 512, 64, False, seed=3,
+                seqlen_range=(64, 512))
+LLAMA_GQA = Workload("llama_gqa_causal_b2_hq32_hkv8_n8192_d128", 2, 32, 8, 8192, 128, True,
+                     seed=4, k_scale=2.0, sample_rows=256)
+LONG = Workload("long_causal_b1_h16_n32768_d128", 1, 16, 16, 32768, 128, True, seed=5,
+                sample_rows=256)
+
+ALL = (TINY, GPT2, BERT, LLAMA_GQA, LONG)
+BY_NAME = {w.name: w for w in ALL}
+
+
+def round_to_bf16_bits(x: np.ndarray) -> np.ndarray:
+    """fp32 -> bf16 bit patterns (uint16), round to nearest, ties to even.
+
+    Inputs here are finite normal draws, so no NaN handling is needed; a NaN
+    or an infinity is rejected rather than silently re-encoded."""
+    x = np.ascontiguousarray(x, dtype=np.float32)
+    if not np.all(np.isfinite(x)):
+        raise ValueError("round_to_bf16_bits: non-finite input")
+    u = x.view(np.uint32).astype(np.uint64)
+    lsb = (u >> 16) & 1
+    r = (u + 0x7FFF + lsb) >> 16
+    return r.astype(np.uint16)
+
+
+def bf16_bits_to_f32(b: np.ndarray) -> np.ndarray:
+    """bf16 bit patterns -> the fp32 values they encode (exact)."""
+    b = np.ascontiguousarray(b, dtype=np.uint16)
+    return (b.astype(np.uint32) << 16).view(np.float32)
+
+
+@dataclasses.dataclass
+class Inputs:
+    """One seeded draw.  ``*_bits`` are the bf16 tensors the kernels read;
+    ``*_f32`` hold exactly the same values in fp32 for the oracle and for the
+    fp32 check mode."""
+    q_bits: np.ndarray
+    k_bits: np.ndarray
+    v_bits: np.ndarray
+    seqlens: np.ndarray | None  # int32 [B] or None
+
+    @property
+    def q_f32(self) -> np.ndarray:
+        return bf16_bits_to_f32(self.q_bits)
+
+    @property
+    def k_f32(self) -> np.ndarray:
+        return bf16_bits_to_f32(self.k_bits)
+
+    @property
+    def v_f32(self) -> np.ndarray:
+        return bf16_bits_to_f32(self.v_bits)
+
+
+def draw(B: int, Hq: int, Hkv: int, N: int, d: int, seed: int, *, k_scale: float = 1.0,
+         seqlen_range: tuple[int, int] | None = None) -> Inputs:
+    rng = np.random.default_rng(seed)
+    q = rng.standard_normal((B, Hq, N, d), dtype=np.float32)
+    k = rng.standard_normal((B, Hkv, N, d), dtype=np.float32)
+    v = rng.standard_normal((B, Hkv, N, d), dtype=np.float32)
+    if k_scale != 1.0:
+        k *= np.float32(k_scale)
+    seqlens = None
+    if seqlen_range is not None:
+        lo, hi = seqlen_range
+        seqlens = rng.integers(lo, hi + 1, B).astype(np.int32)
+    return Inputs(round_to_bf16_bits(q), round_to_bf16_bits(k), round_to_bf16_bits(v), seqlens)
+
+
+def draw_workload(w: Workload) -> Inputs:
+    return draw(w.B, w.Hq, w.Hkv, w.N, w.d, w.seed, k_scale=w.k_scale,
+                seqlen_range=w.seqlen_range)
+
+
+def sample_rows(w: Workload, rows_per_head: int | None = None) -> np.ndarray:
+    """Query rows to check for a large workload: int64 [B*Hq, R], sorted per
+    (batch, head), drawn without replacement from ``default_rng(seed + 100)``."""
+    r = rows_per_head or w.sample_rows or w.N
+    rng = np.random.default_rng(w.seed + 100)
+    out = np.empty((w.B * w.Hq, r), dtype=np.int64)
+    for bh in range(w.B * w.Hq):
+        out[bh] = np.sort(rng.choice(w.N, size=r, replace=False))
+    return out
+
+
+def flops(w: Workload, seqlens: np.ndarray | None = None) -> float:
+    """Attention forward FLOPs as the metric counts them: 4*B*Hq*N^2*d,
+    halved for causal; with key padding 4*Hq*d*N*sum(len_b)."""
+    if seqlens is not None:
+        return 4.0 * w.Hq * w.d * w.N * float(np.sum(seqlens))
+    f = 4.0 * w.B * w.Hq * w.N * w.N * w.d
+    return f / 2 if w.causal else f

@@ -1,0 +1,102 @@
+"""fp64 CPU oracle for the exact attention forward.  TEST INFRASTRUCTURE.
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
+``bench.py`` may import this package.  The CUDA library never calls it, and it
+imports nothing from the CUDA package: the two meet only through the seeded
+inputs that the tests pass to both.
+
+The arithmetic lives in ``attention_ref.c`` (plain C, fp64, POSIX threads over
+(batch, head, block of query rows)); this file only marshals arrays.  See
+that file's header for the definition it follows and the readings taken
+where the pages are silent.  Parity pins: ``tests/test_oracle.py``.
+"""
+from __future__ import annotations
+
+import ctypes
+
+import numpy as np
+
+from . import build as _build
+
+_IN_KIND = {np.dtype(np.float64): 0, np.dtype(np.float32): 1, np.dtype(np.uint16): 2}
+_lib = None
+
+
+def open_library(path: str):
+    """Bind a compiled copy of attention_ref.c (the default one, or a test's
+    deliberately mutated copy)."""
+    lib = ctypes.CDLL(path)
+    lib.oracle_attention_fwd.restype = ctypes.c_int
+    lib.oracle_attention_fwd.argtypes = [
+        ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int,
+        ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+        ctypes.c_double, ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int,
+        ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int,
+    ]
+    return lib
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        _lib = open_library(_build.build())
+    return _lib
+
+
+def num_threads() -> int:
+    """Threads the oracle uses: the cores this process may run on."""
+    import os
+    return max(1, len(os.sched_getaffinity(0)))
+
+
+def attention_forward(q, k, v, *, causal: bool, scale: float, seqlens=None, rows=None,
+                      return_probs: bool = False, threads: int | None = None,
+                      _lib_override=None):
+    """Exact softmax attention in fp64.
+
+    q: [B, Hq, N, d]; k, v: [B, Hkv, N, d]; dtype float64, float32 or uint16
+    (bf16 bit patterns).  seqlens: int [B] key lengths or None.  rows: int
+    [B*Hq, R] query rows per (batch, head) or None for all rows.
+
+    Returns (o [B, Hq, R, d], lse [B, Hq, R]) in fp64, plus P [B, Hq, R, N]
+    when return_probs is set (small cases only).
+    """
+    q = np.ascontiguousarray(q)
+    k = np.ascontiguousarray(k)
+    v = np.ascontiguousarray(v)
+    if not (q.dtype == k.dtype == v.dtype) or q.dtype not in _IN_KIND:
+        raise TypeError("q, k, v must share one dtype among float64, float32, uint16(bf16)")
+    B, Hq, N, d = q.shape
+    Bk, Hkv, Nk, dk = k.shape
+    if (Bk, Nk, dk) != (B, N, d) or v.shape != k.shape:
+        raise ValueError("shape mismatch between q and k/v")
+    if Hq % Hkv:
+        raise ValueError("Hq must be a multiple of Hkv")
+    sl = None
+    if seqlens is not None:
+        sl = np.ascontiguousarray(seqlens, dtype=np.int32)
+        if sl.shape != (B,) or np.any(sl < 0) or np.any(sl > N):
+            raise ValueError("seqlens must be int[B] within [0, N]")
+    if rows is None:
+        R = N
+        rw = None
+    else:
+        rw = np.ascontiguousarray(rows, dtype=np.int64)
+        if rw.ndim != 2 or rw.shape[0] != B * Hq or np.any(rw < 0) or np.any(rw >= N):
+            raise ValueError("rows must be int[B*Hq, R] within [0, N)")
+        R = rw.shape[1]
+    o = np.empty((B, Hq, R, d), dtype=np.float64)
+    lse = np.empty((B, Hq, R), dtype=np.float64)
+    p = np.empty((B, Hq, R, N), dtype=np.float64) if return_probs else None
+
+    def ptr(a):
+        return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+    lib = _lib_override if _lib_override is not None else _load()
+    rc = lib.oracle_attention_fwd(
+        ptr(q), ptr(k), ptr(v), _IN_KIND[q.dtype], B, Hq, Hkv, N, d, float(scale),
+        int(bool(causal)), ptr(sl), ptr(rw), R, ptr(o), ptr(lse), ptr(p),
+        int(threads or num_threads()))
+    if rc != 0:
+        raise RuntimeError(f"oracle_attention_fwd failed ({rc})")
+    return (o, lse, p) if return_probs else (o, lse)

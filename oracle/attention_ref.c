@@ -1,0 +1,189 @@
+/*
+ * Exact attention forward, fp64, on the CPU.  TEST INFRASTRUCTURE ONLY.
+ *
+ * This is the oracle the CUDA path is checked against.  Only the tests, the
+ * smoke check and the benchmark's CPU-baseline leg may call it; the product
+ * path never does.  It shares no code, header or constant with the GPU
+ * library.
+ *
+ * What it computes (the plain definition, no tiling, no online softmax):
+ *   for each batch b and query head h, with kv head g = h / (Hq / Hkv):
+ *     S[i][j] = scale * sum_c Q[b,h,i,c] * K[b,g,j,c]         (fp64)
+ *     S[i][j] = -inf  if j >= len_b, or (causal and j > i)
+ *     M_i     = max_j S[i][j]
+ *     P[i][j] = exp(S[i][j] - M_i) / sum_j' exp(S[i][j'] - M_i)
+ *     O[i]    = sum_j P[i][j] * V[b,g,j,:]
+ *     LSE_i   = M_i + log(sum_j exp(S[i][j] - M_i))
+ *   A row with no visible key gets O = 0 and LSE = -inf.
+ *
+ * Sources (page title, section):
+ *   - "FlashAttention" wiki note (llm-wiki-maxwellmou), section "what it is":
+ *     O = softmax(Q K^T / sqrt(d)) V; for one head S = Q K^T, P = softmax(S),
+ *     output P V, with S and P both T x T.
+ *   - "FlashAttention" explainer (liu-gong-zi), pseudo-code of standard
+ *     attention: scores, softmax over each row, weighted sum of V.
+ *   - "Why is FlashAttention faster" interview notes (arfxm), section on what
+ *     standard attention stores: mask applied to the scores before softmax.
+ *   - wiki note, same section: causal and padding masks and multiple heads
+ *     are handled per tile; enable_gqa in the SDPA call (GQA head sharing).
+ * Readings where the pages are silent: the mask is additive 0/-inf, causal is
+ * top-left aligned (key j visible to query i iff j <= i), key padding masks
+ * keys j >= len_b only (every query row is still computed), GQA groups are
+ * contiguous (query heads [g*G, (g+1)*G) share kv head g), LSE is the
+ * natural log.
+ *
+ * S and P are materialised per block of query rows, exactly as defined.
+ * Blocks are independent and run on a pool of POSIX threads.
+ */
+#include <math.h>
+#include <pthread.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+enum { ORACLE_IN_F64 = 0, ORACLE_IN_F32 = 1, ORACLE_IN_BF16 = 2 };
+
+#define ORACLE_ROW_BLOCK 16
+
+/* Decode one input element to fp64.  bf16 and fp32 values widen exactly. */
+static double in_at(const void *base, int kind, int64_t idx) {
+  if (kind == ORACLE_IN_F64) return ((const double *)base)[idx];
+  if (kind == ORACLE_IN_F32) return (double)((const float *)base)[idx];
+  uint32_t u = (uint32_t)((const uint16_t *)base)[idx] << 16;
+  float f;
+  memcpy(&f, &u, sizeof f);
+  return (double)f;
+}
+
+typedef struct {
+  const void *q, *k, *v;
+  int in_kind, B, Hq, Hkv, N, d, causal, R, nblk;
+  double scale;
+  const int32_t *seqlens;
+  const int64_t *rows;
+  double *o, *lse, *p_out;
+  int64_t total;
+  int64_t next; /* shared task counter */
+  int bad;
+} job_t;
+
+/* One task: one block of up to ORACLE_ROW_BLOCK query rows of one (b, h). */
+static void run_block(const job_t *J, int64_t t, double *S, double *qrow) {
+  const int N = J->N, d = J->d, R = J->R;
+  const int64_t bh = t / J->nblk;
+  const int blk = (int)(t % J->nblk);
+  const int b = (int)(bh / J->Hq);
+  const int h = (int)(bh % J->Hq);
+  const int g = h / (J->Hq / J->Hkv);
+  int len = J->seqlens ? J->seqlens[b] : N;
+  if (len < 0) len = 0;
+  if (len > N) len = N;
+  const int64_t qbase = ((int64_t)b * J->Hq + h) * N * d;
+  const int64_t kvbase = ((int64_t)b * J->Hkv + g) * N * d;
+  const int r0 = blk * ORACLE_ROW_BLOCK;
+  const int r1 = (r0 + ORACLE_ROW_BLOCK < R) ? r0 + ORACLE_ROW_BLOCK : R;
+
+  /* 1. S for this block of query rows, masked entries set to -inf. */
+  for (int r = r0; r < r1; ++r) {
+    const int64_t i = J->rows ? J->rows[bh * R + r] : r;
+    double *Srow = S + (size_t)(r - r0) * N;
+    for (int c = 0; c < d; ++c) qrow[c] = in_at(J->q, J->in_kind, qbase + i * d + c);
+    for (int j = 0; j < N; ++j) {
+      const int visible = (j < len) && (!J->causal || j <= i);
+      if (!visible) {
+        Srow[j] = -INFINITY;
+        continue;
+      }
+      double acc = 0.0;
+      for (int c = 0; c < d; ++c) acc += qrow[c] * in_at(J->k, J->in_kind, kvbase + (int64_t)j * d + c);
+      Srow[j] = J->scale * acc;
+    }
+  }
+
+  /* 2. P = softmax(S) row by row (in place over S), LSE from the same sum. */
+  for (int r = r0; r < r1; ++r) {
+    double *Srow = S + (size_t)(r - r0) * N;
+    double m = -INFINITY;
+    for (int j = 0; j < N; ++j)
+      if (Srow[j] > m) m = Srow[j];
+    double *orow = J->o + (bh * R + r) * (int64_t)d;
+    if (m == -INFINITY) {
+      for (int j = 0; j < N; ++j) Srow[j] = 0.0;
+      J->lse[bh * R + r] = -INFINITY;
+    } else {
+      double denom = 0.0;
+      for (int j = 0; j < N; ++j) denom += exp(Srow[j] - m);
+      for (int j = 0; j < N; ++j) Srow[j] = exp(Srow[j] - m) / denom;
+      J->lse[bh * R + r] = m + log(denom);
+    }
+    if (J->p_out) memcpy(J->p_out + (bh * R + r) * (int64_t)N, Srow, sizeof(double) * (size_t)N);
+
+    /* 3. O = P V. */
+    for (int c = 0; c < d; ++c) orow[c] = 0.0;
+    for (int j = 0; j < N; ++j) {
+      const double p = Srow[j];
+      if (p == 0.0) continue;
+      for (int c = 0; c < d; ++c) orow[c] += p * in_at(J->v, J->in_kind, kvbase + (int64_t)j * d + c);
+    }
+  }
+}
+
+static void *worker(void *arg) {
+  job_t *J = (job_t *)arg;
+  double *S = (double *)malloc(sizeof(double) * (size_t)ORACLE_ROW_BLOCK * (size_t)J->N);
+  double *qrow = (double *)malloc(sizeof(double) * (size_t)J->d);
+  if (!S || !qrow) {
+    __atomic_store_n(&J->bad, 1, __ATOMIC_RELAXED);
+  } else {
+    for (;;) {
+      const int64_t t = __atomic_fetch_add(&J->next, 1, __ATOMIC_RELAXED);
+      if (t >= J->total) break;
+      run_block(J, t, S, qrow);
+    }
+  }
+  free(S);
+  free(qrow);
+  return NULL;
+}
+
+/*
+ * q: [B, Hq, N, d]; k, v: [B, Hkv, N, d]; element type given by in_kind.
+ * seqlens: int32 [B] key lengths (0 <= len_b <= N) or NULL for N.
+ * rows: int64 [B*Hq, R] query rows to compute per (b, h), or NULL for all N
+ *       (then R must equal N).
+ * o: fp64 [B*Hq, R, d]; lse: fp64 [B*Hq, R].
+ * p_out: optional fp64 [B*Hq, R, N], the probability rows P[i][:].
+ * nthreads: worker threads (>= 1); tasks are independent blocks of rows, so
+ *           the result does not depend on it.
+ * Returns 0, or -1 on a bad argument or an allocation failure.
+ */
+int oracle_attention_fwd(const void *q, const void *k, const void *v, int in_kind, int B, int Hq,
+                         int Hkv, int N, int d, double scale, int causal,
+                         const int32_t *seqlens, const int64_t *rows, int R, double *o,
+                         double *lse, double *p_out, int nthreads) {
+  if (!q || !k || !v || !o || !lse) return -1;
+  if (B <= 0 || Hq <= 0 || Hkv <= 0 || N <= 0 || d <= 0 || R <= 0) return -1;
+  if (Hq % Hkv != 0) return -1;
+  if (!rows && R != N) return -1;
+  if (in_kind < ORACLE_IN_F64 || in_kind > ORACLE_IN_BF16) return -1;
+  job_t J;
+  memset(&J, 0, sizeof J);
+  J.q = q; J.k = k; J.v = v; J.in_kind = in_kind;
+  J.B = B; J.Hq = Hq; J.Hkv = Hkv; J.N = N; J.d = d; J.causal = causal; J.R = R;
+  J.scale = scale; J.seqlens = seqlens; J.rows = rows; J.o = o; J.lse = lse; J.p_out = p_out;
+  J.nblk = (R + ORACLE_ROW_BLOCK - 1) / ORACLE_ROW_BLOCK;
+  J.total = (int64_t)B * Hq * J.nblk;
+  if (nthreads < 1) nthreads = 1;
+  if ((int64_t)nthreads > J.total) nthreads = (int)J.total;
+  pthread_t *th = (pthread_t *)malloc(sizeof(pthread_t) * (size_t)nthreads);
+  if (!th) return -1;
+  int started = 0;
+  for (int t = 1; t < nthreads; ++t) {
+    if (pthread_create(&th[t], NULL, worker, &J) != 0) break;
+    ++started;
+  }
+  worker(&J);
+  for (int t = 1; t <= started; ++t) pthread_join(th[t], NULL);
+  free(th);
+  return J.bad ? -1 : 0;
+}
