@@ -1,0 +1,334 @@
+"""Benchmark: exact attention forward TFLOP/s on B200 (bf16, causal counts half
+the FLOPs), as a fraction of the measured dense-bf16 tensor-core peak.
+
+One step = one forward of the whole workload (one kernel launch) on inputs
+already resident in device memory.  Default workload: the Llama-style GQA
+causal layer, B=2, Hq=32, Hkv=8, N=8192, d=128, K scaled by 2.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl mine|reference]
+
+With N > 1 (launched by torch.distributed.run) every rank runs its own
+replica of the workload on its own GPU; there is no data exchange between
+ranks (the work units are independent), so scaling is weak.  Rank 0 prints
+one JSON line.  `--impl reference` times the CPU oracle instead (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from exact_io_aware_92_b200 import workloads as wl  # noqa: E402
+
+L2_BYTES = 126 * 1024 * 1024
+FALLBACK_PEAKS = {"bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "hbm_gbs": 6650.0}
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    except (OSError, ValueError):
+        return FALLBACK_PEAKS, "fallback"
+
+
+def dist_env():
+    return (int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")),
+            int(os.environ.get("LOCAL_RANK", "0")))
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons, sampled every 200 ms while the
+    timed region runs."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.out = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=self.out, stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.out.flush()
+        self.out.seek(0)
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.out.read().splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax.append(float(parts[2]))
+            except ValueError:
+                continue
+            for name, flag in zip(names, parts[5:9]):
+                if flag.lower().startswith("active"):
+                    reasons.add(name)
+        os.unlink(self.out.name)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        loaded = [s for s in sm if s > 0.5 * max(sm)] or sm
+        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": max(smax),
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def oracle_sample_rows(w: wl.Workload, rows_per_head: int, seed: int = 1234) -> np.ndarray:
+    rng = np.random.default_rng(seed)
+    return np.stack([np.sort(rng.choice(w.N, rows_per_head, replace=False))
+                     for _ in range(w.B * w.Hq)])
+
+
+def sample_flops(w: wl.Workload, rows: np.ndarray, seqlens) -> float:
+    """Metric FLOPs of the sampled query rows: 4*d per visible key, with the
+    causal count halved as the metric defines it (whole rows otherwise)."""
+    total = 0.0
+    for bh in range(rows.shape[0]):
+        L = w.N if seqlens is None else int(seqlens[bh // w.Hq])
+        total += 4.0 * w.d * L * rows.shape[1]
+    return total / 2 if w.causal else total
+
+
+def time_oracle(w: wl.Workload, inp: wl.Inputs, budget_s: float):
+    """The CPU oracle on a bounded sample of query rows of the same workload."""
+    import oracle
+    threads = oracle.num_threads()
+    rows_per_head = 4
+    scale = float(np.float32(w.scale))
+    while True:
+        rows = oracle_sample_rows(w, rows_per_head)
+        t0 = time.perf_counter()
+        oracle.attention_forward(inp.q_bits, inp.k_bits, inp.v_bits, causal=w.causal, scale=scale,
+                                 seqlens=inp.seqlens, rows=rows, threads=threads)
+        dt = time.perf_counter() - t0
+        if dt > budget_s / 4 or rows_per_head >= w.N:
+            break
+        rows_per_head = min(w.N, rows_per_head * max(2, int(budget_s / 4 / max(dt, 1e-3))))
+    f = sample_flops(w, rows, inp.seqlens)
+    return {"value": f / dt / 1e12, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+            "sample": f"{rows_per_head} seeded query rows per (batch, head) of {w.name} "
+                      f"({rows.size} rows, every visible key), {dt:.1f} s wall"}, dt
+
+
+def run_reference(args, w: wl.Workload):
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return 0
+    inp = wl.draw_workload(w)
+    per_step = []
+    cpu = None
+    for s in range(args.warmup + args.steps):
+        cpu, dt = time_oracle(w, inp, budget_s=args.ref_budget)
+        if s >= args.warmup:
+            per_step.append(cpu["value"])
+    value = statistics.median(per_step)
+    cpu["value"] = value
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": None, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f64", "data": "synthetic (seeded, bf16-rounded N(0,1))",
+        "config": workload_config(w),
+        "cpu_baseline": cpu,
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+        "gpu_launches": 0,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+METRIC = "attention fwd TFLOP/s (bf16, causal=1/2 FLOPs) and % of B200 dense BF16 peak"
+
+
+def workload_config(w: wl.Workload):
+    return {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "N": w.N, "d": w.d,
+            "causal": w.causal, "k_scale": w.k_scale, "scale": w.scale,
+            "seqlens": None if w.seqlen_range is None else f"uniform {w.seqlen_range}"}
+
+
+def run_mine(args, w: wl.Workload):
+    import torch
+    import torch.distributed as dist
+    from exact_io_aware_92_b200 import _lib, attention
+
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+    # Each rank: its own replica of the workload (seed offset by rank).
+    inp = wl.draw(w.B, w.Hq, w.Hkv, w.N, w.d, w.seed + 1000 * rank, k_scale=w.k_scale,
+                  seqlen_range=w.seqlen_range)
+    q, k, v = (torch.from_numpy(x).view(torch.bfloat16).to(dev)
+               for x in (inp.q_bits, inp.k_bits, inp.v_bits))
+    sl = None if inp.seqlens is None else torch.from_numpy(inp.seqlens).to(dev)
+    o = torch.empty_like(q)
+    lse = torch.empty((w.B, w.Hq, w.N), dtype=torch.float32, device=dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    flops = wl.flops(w, inp.seqlens)
+    in_bytes = sum(t.numel() * t.element_size() for t in (q, k, v))
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        attention.fwd(q, k, v, causal=w.causal, scale=w.scale, seqlens=sl, out=o, lse=lse,
+                      status=status)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    if attention.check_status(status) != 0:
+        raise RuntimeError("kernel reported a time-out during warm-up")
+
+    sampler = ClockSampler(local)
+    barrier()
+    torch.cuda.synchronize(dev)
+    sampler.start()
+    time.sleep(0.3)
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    start.record(stream)
+    for _ in range(args.steps):
+        step()
+    end.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    clocks = sampler.stop()
+    ms_total = start.elapsed_time(end)
+    if attention.check_status(status) != 0:
+        raise RuntimeError("kernel reported a time-out in the timed region")
+    ms_max = ms_total
+    if world > 1:
+        t = torch.tensor([ms_total], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_max = float(t.item())
+    ms_per_step = ms_max / args.steps
+    value = world * flops * args.steps / (ms_max * 1e-3) / 1e12
+    kernel_tflops = flops / (ms_total / args.steps * 1e-3) / 1e12
+
+    # End to end through the C ABI on host buffers: pinned host inputs are
+    # copied in, the forward runs, O and LSE are copied back, every step.
+    q_h, k_h, v_h = (torch.from_numpy(x).pin_memory() for x in (inp.q_bits, inp.k_bits, inp.v_bits))
+    o_h = torch.empty(q_h.shape, dtype=torch.int16).pin_memory()
+    lse_h = torch.empty(lse.shape, dtype=torch.float32).pin_memory()
+    sl_h = None if inp.seqlens is None else torch.from_numpy(inp.seqlens).pin_memory()
+    e2e_steps = max(2, min(args.steps, 10))
+    for _ in range(2):
+        attention.fwd_hostio(q_h, k_h, v_h, o_h, lse_h, q, k, v, o, lse, causal=w.causal,
+                             scale=w.scale, seqlens_h=sl_h, seqlens_d=sl)
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        attention.fwd_hostio(q_h, k_h, v_h, o_h, lse_h, q, k, v, o, lse, causal=w.causal,
+                             scale=w.scale, seqlens_h=sl_h, seqlens_d=sl)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = e0.elapsed_time(e1)
+    if world > 1:
+        t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    e2e_value = world * flops * e2e_steps / (e2e_ms * 1e-3) / 1e12
+    h2d = in_bytes + (0 if sl is None else sl.numel() * 4)
+    d2h = o.numel() * 2 + lse.numel() * 4
+
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return 0
+
+    peaks, src = load_peaks()
+    peak = float(peaks["bf16_tflops"])
+    traffic = None
+    traffic_file = os.path.join(ROOT, "profiles", "traffic.json")
+    if os.path.exists(traffic_file):
+        with open(traffic_file) as f:
+            traffic = json.load(f).get(w.name)
+    cpu, _ = time_oracle(w, inp, budget_s=args.cpu_budget) if not args.no_cpu_baseline else (
+        None, None)
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded, bf16-rounded N(0,1))",
+        "config": dict(workload_config(w),
+                       l2=f"no flush: inputs {in_bytes / 2**20:.0f} MiB > L2 126 MiB",
+                       parallelism=f"replicas x{world}" if world > 1 else "single GPU"),
+        "roofline": {"bound": "tensor", "achieved": kernel_tflops, "peak": peak,
+                     "unit": "TFLOP/s", "frac": kernel_tflops / peak, "traffic": traffic,
+                     "peak_source": f"{src} bf16_tflops (burst; kernel timed back to back)"},
+        "pct_of_peak": 100.0 * kernel_tflops / peak,
+        "clocks": clocks,
+        "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h},
+        "gpu_launches": args.steps,
+        "cpu_baseline": cpu,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=30)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["mine", "reference"], default="mine")
+    ap.add_argument("--workload", default=wl.LLAMA_GQA.name, choices=sorted(wl.BY_NAME))
+    ap.add_argument("--cpu-budget", type=float, default=15.0,
+                    help="seconds of CPU work for the oracle baseline sample")
+    ap.add_argument("--ref-budget", type=float, default=8.0,
+                    help="seconds of CPU work per reference-arm step")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--batch", type=int, default=None,
+                    help="override the workload's batch size (profiling a smaller case)")
+    args = ap.parse_args()
+    w = wl.BY_NAME[args.workload]
+    if args.batch is not None:
+        import dataclasses
+        w = dataclasses.replace(w, B=args.batch, name=f"{w.name}@B{args.batch}")
+    if args.impl == "reference":
+        return run_reference(args, w)
+    return run_mine(args, w)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

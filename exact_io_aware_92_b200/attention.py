@@ -1,0 +1,83 @@
+"""Python entry points over the C ABI.  Argument marshalling only: every step
+of the attention forward runs in the CUDA kernels of libfa_b200.so.
+
+PyTorch provides device memory and the current stream; nothing here computes.
+"""
+from __future__ import annotations
+
+import math
+
+import torch
+
+from . import _lib
+
+
+def _stream_handle(device: torch.device) -> int:
+    return torch.cuda.current_stream(device).cuda_stream
+
+
+def _check_qkv(q, k, v, dtype):
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        if not t.is_cuda:
+            raise ValueError(f"{name} must be a CUDA tensor")
+        if t.dtype != dtype:
+            raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+        if t.dim() != 4 or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous [B, H, N, d] tensor")
+    B, Hq, N, d = q.shape
+    if k.shape != v.shape or k.shape[0] != B or k.shape[2] != N or k.shape[3] != d:
+        raise ValueError("k and v must be [B, Hkv, N, d] matching q")
+    return B, Hq, k.shape[1], N, d
+
+
+def fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *, causal: bool = False,
+        scale: float | None = None, seqlens: torch.Tensor | None = None,
+        out: torch.Tensor | None = None, lse: torch.Tensor | None = None,
+        status: torch.Tensor | None = None):
+    """Exact attention forward.  q: [B, Hq, N, d], k, v: [B, Hkv, N, d], all
+    bf16 (tensor cores) or all fp32 (check mode), contiguous, on one CUDA
+    device.  seqlens: int32 [B] key lengths on the same device, or None.
+    Returns (o, lse): o like q, lse fp32 [B, Hq, N].  Runs on the current
+    stream; `status` (int32 [1] on the device) receives in-kernel time-outs."""
+    if q.dtype not in (torch.bfloat16, torch.float32):
+        raise TypeError("q, k, v must be bf16 or fp32")
+    B, Hq, Hkv, N, d = _check_qkv(q, k, v, q.dtype)
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, Hq, N), dtype=torch.float32, device=q.device)
+    sl_ptr = None
+    if seqlens is not None:
+        if seqlens.dtype != torch.int32 or seqlens.device != q.device or seqlens.numel() != B:
+            raise ValueError("seqlens must be int32 [B] on q's device")
+        sl_ptr = seqlens.data_ptr()
+    dtype = _lib.FA_DTYPE_BF16 if q.dtype == torch.bfloat16 else _lib.FA_DTYPE_F32
+    rc = _lib.load().fa_fwd_ex(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                               lse.data_ptr(), B, Hq, Hkv, N, d, scale, int(bool(causal)), sl_ptr,
+                               dtype, _stream_handle(q.device),
+                               None if status is None else status.data_ptr())
+    _lib.check(rc, "fa_fwd_ex")
+    return out, lse
+
+
+def check_status(status: torch.Tensor | None = None, device: torch.device | None = None) -> int:
+    """Synchronise the current stream and return the status word (0 = ok)."""
+    dev = status.device if status is not None else (device or torch.device("cuda"))
+    return _lib.load().fa_check_status(None if status is None else status.data_ptr(),
+                                       _stream_handle(dev))
+
+
+def fwd_hostio(q_h, k_h, v_h, o_h, lse_h, q_d, k_d, v_d, o_d, lse_d, *, causal: bool,
+               scale: float, seqlens_h=None, seqlens_d=None) -> None:
+    """End-to-end call on host tensors (pinned for asynchronous copies):
+    host->device copies, the forward, device->host copies, then a wait."""
+    B, Hq, N, d = q_h.shape
+    Hkv = k_h.shape[1]
+    rc = _lib.load().fa_fwd_hostio(
+        q_h.data_ptr(), k_h.data_ptr(), v_h.data_ptr(), o_h.data_ptr(), lse_h.data_ptr(),
+        None if seqlens_h is None else seqlens_h.data_ptr(), q_d.data_ptr(), k_d.data_ptr(),
+        v_d.data_ptr(), o_d.data_ptr(), lse_d.data_ptr(),
+        None if seqlens_d is None else seqlens_d.data_ptr(), B, Hq, Hkv, N, d, float(scale),
+        int(bool(causal)), _stream_handle(q_d.device))
+    _lib.check(rc, "fa_fwd_hostio")

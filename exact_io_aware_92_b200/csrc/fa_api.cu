@@ -1,0 +1,328 @@
+// C ABI of the attention-forward library (declared in include/fa.h).
+//
+// Host side only: argument checks, TMA tensor maps (cuTensorMapEncodeTiled,
+// reached through the runtime's driver entry point so the library does not
+// link libcuda), launch configuration, and the status word.  All attention
+// arithmetic runs in the kernels of fa_fwd_sm100.cuh and fa_fwd_f32.cuh.
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "fa.h"
+#include "fa_fwd_f32.cuh"
+#include "fa_fwd_sm100.cuh"
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+constexpr unsigned long long kWaitLimitNs = 2000000000ull;  // 2 s per wait
+constexpr float kLog2e = 1.4426950408889634f;
+
+// The library's own status word, used when the caller passes none.
+__device__ int g_status_word;
+
+struct DeviceState {
+  bool checked = false;
+  bool ok = false;
+  int num_sms = 0;
+  int *status_word = nullptr;  // device address of g_status_word
+  bool attr64 = false, attr128 = false;
+};
+DeviceState g_dev[kMaxDevices];
+std::mutex g_mu;
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                   const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                   const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn g_encode = nullptr;
+
+// Current device, checked once per device: must be sm_100 (B200).
+int current_device(DeviceState **out) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+    cudaGetLastError();
+    return FA_ERR_ARCH;
+  }
+  std::lock_guard<std::mutex> lock(g_mu);
+  DeviceState &s = g_dev[dev];
+  if (!s.checked) {
+    s.checked = true;
+    cudaDeviceProp prop;
+    if (cudaGetDeviceProperties(&prop, dev) != cudaSuccess) {
+      cudaGetLastError();
+      return FA_ERR_ARCH;
+    }
+    if (prop.major != 10 || prop.minor != 0) return FA_ERR_ARCH;
+    s.num_sms = prop.multiProcessorCount;
+    void *addr = nullptr;
+    if (cudaGetSymbolAddress(&addr, g_status_word) != cudaSuccess) {
+      cudaGetLastError();
+      return FA_ERR_CUDA;
+    }
+    s.status_word = static_cast<int *>(addr);
+    s.ok = true;
+  }
+  if (!s.ok) return FA_ERR_ARCH;
+  if (!g_encode) {
+    void *fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &fn, 12000, cudaEnableDefault,
+                                         &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess || !fn) {
+      cudaGetLastError();
+      return FA_ERR_CUDA;
+    }
+    g_encode = reinterpret_cast<EncodeTiledFn>(fn);
+  }
+  *out = &s;
+  return FA_OK;
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int check_args(const void *q, const void *k, const void *v, const void *o, const float *lse,
+               int B, int Hq, int Hkv, int N, int d, float scale) {
+  if (!q || !k || !v || !o || !lse) return FA_ERR_NULL;
+  if (B <= 0 || Hq <= 0 || Hkv <= 0 || N <= 0 || d <= 0) return FA_ERR_SHAPE;
+  if (!(std::isfinite(scale) && scale > 0.f)) return FA_ERR_SHAPE;
+  if (Hq % Hkv != 0) return FA_ERR_HEADS;
+  if (d != 64 && d != 128) return FA_ERR_HEADDIM;
+  // element counts must fit the kernels' 64-bit offsets and the 32-bit grid
+  const long long rows = static_cast<long long>(B) * Hq;
+  if (rows > (1ll << 30) || static_cast<long long>(N) * d > (1ll << 40)) return FA_ERR_SHAPE;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return FA_ERR_ALIGN;
+  if ((reinterpret_cast<uintptr_t>(lse) & 3u) != 0) return FA_ERR_ALIGN;
+  return FA_OK;
+}
+
+// 3-D map over a [planes, N, d] bf16 tensor: box = 64 columns x 128 rows x 1
+// plane, 128-byte swizzle; rows past N read as zero.
+int make_map(CUtensorMap *m, const void *ptr, int planes, int N, int d) {
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(N),
+                        static_cast<cuuint64_t>(planes)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2,
+                           static_cast<cuuint64_t>(N) * static_cast<cuuint64_t>(d) * 2};
+  cuuint32_t box[3] = {64, 128, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(ptr), dims,
+                        strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? FA_OK : FA_ERR_CUDA;
+}
+
+template <int D>
+int launch_bf16(DeviceState *ds, const void *q, const void *k, const void *v, void *o,
+                float *lse, int B, int Hq, int Hkv, int N, float scale, int causal,
+                const int *seqlens, cudaStream_t stream, int *status) {
+  using C = fa::Sm100Cfg<D>;
+  auto kernel = fa::fa_fwd_bf16_sm100_kernel<D>;
+  bool &attr = (D == 64) ? ds->attr64 : ds->attr128;
+  if (!attr) {
+    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             C::SMEM_ALLOC) != cudaSuccess) {
+      cudaGetLastError();
+      return FA_ERR_LAUNCH;
+    }
+    attr = true;
+  }
+  CUtensorMap tq, tk, tv;
+  if (make_map(&tq, q, B * Hq, N, D) != FA_OK || make_map(&tk, k, B * Hkv, N, D) != FA_OK ||
+      make_map(&tv, v, B * Hkv, N, D) != FA_OK)
+    return FA_ERR_CUDA;
+  fa::FwdParams p;
+  p.o = static_cast<uint16_t *>(o);
+  p.lse = lse;
+  p.seqlens = seqlens;
+  p.status = status;
+  p.B = B;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.N = N;
+  p.group = Hq / Hkv;
+  p.num_qpairs = (N + C::ROWS_PER_CTA - 1) / C::ROWS_PER_CTA;
+  p.causal = causal ? 1 : 0;
+  p.scale_log2 = scale * kLog2e;
+  p.wait_limit_ns = kWaitLimitNs;
+  const long long grid = static_cast<long long>(B) * Hq * p.num_qpairs;
+  if (grid > 0x7fffffffll) return FA_ERR_SHAPE;
+  kernel<<<static_cast<unsigned>(grid), C::THREADS, C::SMEM_ALLOC, stream>>>(tq, tk, tv, p);
+  if (cudaGetLastError() != cudaSuccess) return FA_ERR_LAUNCH;
+  return FA_OK;
+}
+
+template <int D>
+int launch_f32(const float *q, const float *k, const float *v, float *o, float *lse, int B,
+               int Hq, int Hkv, int N, float scale, int causal, const int *seqlens,
+               cudaStream_t stream) {
+  fa::F32Params p;
+  p.q = q;
+  p.k = k;
+  p.v = v;
+  p.o = o;
+  p.lse = lse;
+  p.seqlens = seqlens;
+  p.B = B;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.N = N;
+  p.group = Hq / Hkv;
+  p.causal = causal ? 1 : 0;
+  p.scale_log2 = scale * kLog2e;
+  const long long bh = static_cast<long long>(B) * Hq;
+  if (bh > 65535) return FA_ERR_SHAPE;
+  constexpr int ROWS = fa::F32Cfg<D>::ROWS;
+  dim3 grid((N + ROWS - 1) / ROWS, static_cast<unsigned>(bh));
+  fa::fa_fwd_f32_kernel<D><<<grid, ROWS, 0, stream>>>(p);
+  if (cudaGetLastError() != cudaSuccess) return FA_ERR_LAUNCH;
+  return FA_OK;
+}
+
+// Waits on a barrier that nothing arrives at; the bounded wait must give up.
+__global__ void bounded_wait_selftest_kernel(int *status, unsigned long long limit_ns) {
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x != 0) return;
+  abort_flag = 0;
+  fa::mbar_init(fa::smem_u32(&bar), 1);
+  fa::fence_barrier_init();
+  fa::mbar_wait_bounded(fa::smem_u32(&bar), 0, reinterpret_cast<volatile int *>(&abort_flag), status,
+                        limit_ns, fa::kErrTimeout);
+}
+
+}  // namespace
+
+extern "C" {
+
+int fa_version(void) { return 100; }
+
+const char *fa_status_string(int status) {
+  switch (status) {
+    case FA_OK: return "ok";
+    case FA_ERR_NULL: return "a required pointer is NULL";
+    case FA_ERR_SHAPE: return "bad shape or scale";
+    case FA_ERR_HEADS: return "Hq is not a multiple of Hkv";
+    case FA_ERR_HEADDIM: return "head dimension not supported (64 or 128)";
+    case FA_ERR_ALIGN: return "pointer not 16-byte aligned";
+    case FA_ERR_ARCH: return "no sm_100 (B200) CUDA device";
+    case FA_ERR_LAUNCH: return "kernel launch failed";
+    case FA_ERR_TIMEOUT: return "a bounded in-kernel wait ran out";
+    case FA_ERR_DTYPE: return "unknown dtype code";
+    case FA_ERR_CUDA: return "CUDA runtime error";
+    default: return "unknown status";
+  }
+}
+
+int fa_fwd_ex(const void *q, const void *k, const void *v, void *o, float *lse, int B, int Hq,
+              int Hkv, int N, int d, float scale, int causal, const int *seqlens, int dtype,
+              void *stream, int *status_dev) {
+  int rc = check_args(q, k, v, o, lse, B, Hq, Hkv, N, d, scale);
+  if (rc != FA_OK) return rc;
+  if (dtype != FA_DTYPE_BF16 && dtype != FA_DTYPE_F32) return FA_ERR_DTYPE;
+  DeviceState *ds = nullptr;
+  rc = current_device(&ds);
+  if (rc != FA_OK) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (dtype == FA_DTYPE_F32) {
+    const float *qf = static_cast<const float *>(q), *kf = static_cast<const float *>(k),
+                *vf = static_cast<const float *>(v);
+    float *of = static_cast<float *>(o);
+    return d == 64 ? launch_f32<64>(qf, kf, vf, of, lse, B, Hq, Hkv, N, scale, causal, seqlens, st)
+                   : launch_f32<128>(qf, kf, vf, of, lse, B, Hq, Hkv, N, scale, causal, seqlens,
+                                     st);
+  }
+  int *status = status_dev ? status_dev : ds->status_word;
+  return d == 64 ? launch_bf16<64>(ds, q, k, v, o, lse, B, Hq, Hkv, N, scale, causal, seqlens, st,
+                                   status)
+                 : launch_bf16<128>(ds, q, k, v, o, lse, B, Hq, Hkv, N, scale, causal, seqlens,
+                                    st, status);
+}
+
+int fa_fwd(const void *q, const void *k, const void *v, void *o, float *lse, int B, int Hq,
+           int Hkv, int N, int d, float scale, int causal, const int *seqlens) {
+  return fa_fwd_ex(q, k, v, o, lse, B, Hq, Hkv, N, d, scale, causal, seqlens, FA_DTYPE_BF16,
+                   nullptr, nullptr);
+}
+
+int fa_fwd_f32(const float *q, const float *k, const float *v, float *o, float *lse, int B,
+               int Hq, int Hkv, int N, int d, float scale, int causal, const int *seqlens) {
+  return fa_fwd_ex(q, k, v, o, lse, B, Hq, Hkv, N, d, scale, causal, seqlens, FA_DTYPE_F32,
+                   nullptr, nullptr);
+}
+
+int fa_check_status(const int *status_dev, void *stream) {
+  DeviceState *ds = nullptr;
+  int rc = current_device(&ds);
+  if (rc != FA_OK) return rc;
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) {
+    cudaGetLastError();
+    return FA_ERR_CUDA;
+  }
+  int word = 0;
+  if (status_dev) {
+    if (cudaMemcpy(&word, status_dev, sizeof word, cudaMemcpyDeviceToHost) != cudaSuccess) {
+      cudaGetLastError();
+      return FA_ERR_CUDA;
+    }
+  } else {
+    if (cudaMemcpyFromSymbol(&word, g_status_word, sizeof word) != cudaSuccess) {
+      cudaGetLastError();
+      return FA_ERR_CUDA;
+    }
+    const int zero = 0;
+    if (word != 0 && cudaMemcpyToSymbol(g_status_word, &zero, sizeof zero) != cudaSuccess) {
+      cudaGetLastError();
+      return FA_ERR_CUDA;
+    }
+  }
+  return word == 0 ? FA_OK : word;
+}
+
+int fa_fwd_hostio(const void *q_h, const void *k_h, const void *v_h, void *o_h, float *lse_h,
+                  const int *seqlens_h, void *q_d, void *k_d, void *v_d, void *o_d, float *lse_d,
+                  int *seqlens_d, int B, int Hq, int Hkv, int N, int d, float scale, int causal,
+                  void *stream) {
+  if (!q_h || !k_h || !v_h || !o_h || !lse_h) return FA_ERR_NULL;
+  if (seqlens_h && !seqlens_d) return FA_ERR_NULL;
+  int rc = check_args(q_d, k_d, v_d, o_d, lse_d, B, Hq, Hkv, N, d, scale);
+  if (rc != FA_OK) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const size_t qn = static_cast<size_t>(B) * Hq * N * d * 2;
+  const size_t kn = static_cast<size_t>(B) * Hkv * N * d * 2;
+  const size_t ln = static_cast<size_t>(B) * Hq * N * sizeof(float);
+  if (cudaMemcpyAsync(q_d, q_h, qn, cudaMemcpyHostToDevice, st) != cudaSuccess ||
+      cudaMemcpyAsync(k_d, k_h, kn, cudaMemcpyHostToDevice, st) != cudaSuccess ||
+      cudaMemcpyAsync(v_d, v_h, kn, cudaMemcpyHostToDevice, st) != cudaSuccess ||
+      (seqlens_h && cudaMemcpyAsync(seqlens_d, seqlens_h, sizeof(int) * B,
+                                    cudaMemcpyHostToDevice, st) != cudaSuccess)) {
+    cudaGetLastError();
+    return FA_ERR_CUDA;
+  }
+  rc = fa_fwd_ex(q_d, k_d, v_d, o_d, lse_d, B, Hq, Hkv, N, d, scale, causal,
+                 seqlens_h ? seqlens_d : nullptr, FA_DTYPE_BF16, stream, nullptr);
+  if (rc != FA_OK) return rc;
+  if (cudaMemcpyAsync(o_h, o_d, qn, cudaMemcpyDeviceToHost, st) != cudaSuccess ||
+      cudaMemcpyAsync(lse_h, lse_d, ln, cudaMemcpyDeviceToHost, st) != cudaSuccess) {
+    cudaGetLastError();
+    return FA_ERR_CUDA;
+  }
+  return fa_check_status(nullptr, stream);
+}
+
+int fa_selftest_bounded_wait(int *status_dev, unsigned long long limit_ns, void *stream) {
+  if (!status_dev) return FA_ERR_NULL;
+  DeviceState *ds = nullptr;
+  int rc = current_device(&ds);
+  if (rc != FA_OK) return rc;
+  bounded_wait_selftest_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(status_dev,
+                                                                              limit_ns);
+  if (cudaGetLastError() != cudaSuccess) return FA_ERR_LAUNCH;
+  return FA_OK;
+}
+
+}  // extern "C"

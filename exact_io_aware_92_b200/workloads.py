@@ -66,12 +66,23 @@ def round_to_bf16_bits(x: np.ndarray) -> np.ndarray:
     Inputs here are finite normal draws, so no NaN handling is needed; a NaN
     or an infinity is rejected rather than silently re-encoded."""
     x = np.ascontiguousarray(x, dtype=np.float32)
-    if not np.all(np.isfinite(x)):
+    if x.size <= (1 << 20):
+        if not np.all(np.isfinite(x)):
+            raise ValueError("round_to_bf16_bits: non-finite input")
+        # Finite fp32 bit patterns are <= 0xFF7FFFFF, so adding at most
+        # 0x8000 cannot overflow 32 bits.
+        u = x.view(np.uint32)
+        r = u + np.uint32(0x7FFF)
+        r += (u >> np.uint32(16)) & np.uint32(1)
+        r >>= np.uint32(16)
+        return r.astype(np.uint16)
+    # Large tensors: the same rounding (fp32 -> bf16 is round-to-nearest-even
+    # in PyTorch too; tests/test_workloads.py checks the two agree), multithreaded.
+    import torch
+    t = torch.from_numpy(x)
+    if not bool(torch.isfinite(t).all()):
         raise ValueError("round_to_bf16_bits: non-finite input")
-    u = x.view(np.uint32).astype(np.uint64)
-    lsb = (u >> 16) & 1
-    r = (u + 0x7FFF + lsb) >> 16
-    return r.astype(np.uint16)
+    return t.to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
 
 
 def bf16_bits_to_f32(b: np.ndarray) -> np.ndarray:

@@ -1,0 +1,155 @@
+/*
+ * fa.h - exact, IO-aware attention forward for NVIDIA B200 (sm_100a).
+ *
+ * One operation: for every batch b, query head h and query row i,
+ *
+ *     O[b,h,i,:] = softmax_j( scale * Q[b,h,i,:] . K[b,g,j,:] + mask(i,j) ) V[b,g,j,:]
+ *     LSE[b,h,i] = log sum_j exp( scale * Q[b,h,i,:] . K[b,g,j,:] + mask(i,j) )
+ *
+ * with g = h / (Hq / Hkv) (query heads [g*G, (g+1)*G) share kv head g) and
+ * mask(i,j) = -inf when j >= len_b or (causal and j > i), else 0.
+ *
+ * Sources, by page title and section:
+ *  - wiki note "FlashAttention", section "what it is": the formula
+ *    O = softmax(QK^T / sqrt(d)) V; the blockwise recurrence for the running
+ *    row max m, row sum l and output O when a new block S_b = Q_b K_b^T/sqrt(d)
+ *    arrives; causal mask, padding mask and multiple heads handled inside the
+ *    tile; the SDPA call with is_causal and enable_gqa that states the problem.
+ *  - explainer "FlashAttention" (liu-gong-zi): only the final result is stored.
+ * The result is exact up to floating-point rounding (same page; interview
+ * notes "Why is FlashAttention faster", section on exactness): no N x N
+ * score or probability matrix is ever written to device memory.
+ *
+ * LSE is not on the pages: it is the per-row statistic a backward pass
+ * recomputes from (interview notes, section on recomputation), exported in
+ * natural-log units.
+ *
+ * Common conventions for every fa_fwd* call
+ *  - Layout: all tensors contiguous, row-major, head dimension innermost.
+ *      q, o : [B, Hq, N, d]      k, v : [B, Hkv, N, d]      lse : [B, Hq, N] fp32
+ *  - Key padding: seqlens is NULL (every key of the N is visible) or a
+ *    DEVICE pointer to int32[B] with 0 <= seqlens[b] <= N; keys
+ *    j >= seqlens[b] are masked; every query row is still computed.  A row
+ *    with no visible key (seqlens[b] == 0) gets O = 0 and LSE = -inf.
+ *  - Causal: key j is visible to query i iff j <= i (queries and keys share
+ *    the index range [0, N)).
+ *  - Ownership: the caller allocates and owns every buffer; the library
+ *    allocates no device memory per call and keeps no pointer after the call
+ *    returns.  Device pointers must stay valid until the launched work ends.
+ *  - Streams: fa_fwd launches on the legacy default stream; the _ex forms
+ *    take a cudaStream_t (passed as void*, NULL = legacy default stream).
+ *    Launches are asynchronous.
+ *  - Errors: argument errors are reported synchronously and launch nothing.
+ *    Every wait inside a kernel is bounded; a wait that runs out makes the
+ *    kernel write FA_ERR_TIMEOUT into the status word and return, so no call
+ *    can hang the device.  fa_check_status() reads that word.  Nothing aborts,
+ *    traps or throws across this interface.
+ */
+#ifndef FA_B200_FA_H
+#define FA_B200_FA_H
+
+#if defined(__GNUC__)
+#define FA_API __attribute__((visibility("default")))
+#else
+#define FA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  FA_OK = 0,
+  FA_ERR_NULL = -1,      /* a required pointer is NULL */
+  FA_ERR_SHAPE = -2,     /* B, Hq, Hkv, N or d <= 0, scale not finite and > 0, or sizes overflow */
+  FA_ERR_HEADS = -3,     /* Hq is not a multiple of Hkv */
+  FA_ERR_HEADDIM = -4,   /* d not supported: the bf16 kernel takes d in {64, 128}, fp32 d in {64, 128} */
+  FA_ERR_ALIGN = -5,     /* a pointer is not 16-byte aligned (tensor-memory-access rule) */
+  FA_ERR_ARCH = -6,      /* no CUDA device, or the current device is not sm_100 */
+  FA_ERR_LAUNCH = -7,    /* the CUDA launch itself failed */
+  FA_ERR_TIMEOUT = -8,   /* a bounded in-kernel wait ran out (reported by fa_check_status) */
+  FA_ERR_DTYPE = -9,     /* unknown dtype code */
+  FA_ERR_CUDA = -10      /* another CUDA runtime error (copy, query, driver entry point) */
+} fa_status;
+
+/* dtype codes for fa_fwd_ex */
+#define FA_DTYPE_BF16 0
+#define FA_DTYPE_F32 1
+
+/*
+ * Attention forward, bf16 in / bf16 out, fp32 LSE, on the tensor cores.
+ *  q, k, v, o: bf16 device buffers in the layout above; lse: fp32 device.
+ *  B, Hq, Hkv, N, d: batch, query heads, kv heads, sequence length, head dim
+ *  (d in {64, 128}).  scale: multiplies Q.K (the pages use 1/sqrt(d)).
+ *  causal: 0 or 1.  seqlens: NULL or device int32[B].
+ * Returns FA_OK once the kernel is launched on the legacy default stream, or
+ * an fa_status code.  Device-side waits that run out are recorded in the
+ * library's own status word: read it with fa_check_status(NULL, stream).
+ */
+FA_API int fa_fwd(const void *q, const void *k, const void *v, void *o, float *lse, int B, int Hq,
+           int Hkv, int N, int d, float scale, int causal, const int *seqlens);
+
+/*
+ * Same operation with an explicit element type and stream.
+ *  dtype: FA_DTYPE_BF16 (tensor-core kernel) or FA_DTYPE_F32 (fp32 check
+ *         mode: q, k, v, o are fp32, plain CUDA-core arithmetic).
+ *  stream: cudaStream_t or NULL.
+ *  status_dev: NULL (use the library's status word) or a device int the
+ *         kernel sets to FA_ERR_TIMEOUT when a bounded wait runs out; the
+ *         caller zeroes it before the call and reads it with fa_check_status.
+ */
+FA_API int fa_fwd_ex(const void *q, const void *k, const void *v, void *o, float *lse, int B, int Hq,
+              int Hkv, int N, int d, float scale, int causal, const int *seqlens, int dtype,
+              void *stream, int *status_dev);
+
+/*
+ * fp32 check mode: same operation with fp32 q, k, v, o.  The online-softmax
+ * recurrence runs in fp32 on CUDA cores with accurate exp2f, for comparisons
+ * at 1e-5.  Same stream and status rules as fa_fwd.
+ */
+FA_API int fa_fwd_f32(const float *q, const float *k, const float *v, float *o, float *lse, int B,
+               int Hq, int Hkv, int N, int d, float scale, int causal, const int *seqlens);
+
+/*
+ * End-to-end call on HOST buffers: copies q, k, v (and seqlens) from host to
+ * the caller's device buffers, runs the bf16 forward and copies o and lse
+ * back, all on `stream`, then waits for the stream.
+ *  q_h, k_h, v_h, o_h, lse_h, seqlens_h: host buffers (pinned memory gives
+ *  asynchronous copies; seqlens_h may be NULL).
+ *  q_d, k_d, v_d, o_d, lse_d, seqlens_d: device buffers of the same sizes
+ *  (seqlens_d only when seqlens_h is given).
+ * Returns FA_OK when everything, including the device work, has finished
+ * without error; a bounded wait that ran out is returned as FA_ERR_TIMEOUT.
+ */
+FA_API int fa_fwd_hostio(const void *q_h, const void *k_h, const void *v_h, void *o_h, float *lse_h,
+                  const int *seqlens_h, void *q_d, void *k_d, void *v_d, void *o_d, float *lse_d,
+                  int *seqlens_d, int B, int Hq, int Hkv, int N, int d, float scale, int causal,
+                  void *stream);
+
+/*
+ * Waits for `stream` and reads a status word (status_dev, or the library's
+ * own when NULL).  Returns FA_OK, FA_ERR_TIMEOUT, or FA_ERR_CUDA when the
+ * stream reports an error.  Resets the library's own word to FA_OK.
+ */
+FA_API int fa_check_status(const int *status_dev, void *stream);
+
+/*
+ * Bounded-wait self test: launches one tiny kernel whose only work is to
+ * wait on a shared-memory barrier that nothing ever arrives at, with a limit
+ * of limit_ns nanoseconds.  The kernel must give up, write FA_ERR_TIMEOUT into
+ * status_dev (a device int the caller zeroes) and return.  Proves that an
+ * in-kernel wait cannot hang the device.  Returns the launch status.
+ */
+FA_API int fa_selftest_bounded_wait(int *status_dev, unsigned long long limit_ns, void *stream);
+
+/* Human-readable text for an fa_status code (static storage). */
+FA_API const char *fa_status_string(int status);
+
+/* Library version, as major*10000 + minor*100 + patch. */
+FA_API int fa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FA_B200_FA_H */

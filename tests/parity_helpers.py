@@ -1,0 +1,96 @@
+"""Shared pieces of the GPU parity tests: upload seeded inputs, run the CUDA
+path through the C ABI binding, run the oracle on the same values, compare.
+
+Tolerances (fixed by the problem statement):
+  bf16 path : max |O - O_ref| <= 1.5e-2 and max |LSE - LSE_ref| <= 2e-3
+  fp32 path : both <= 1e-5
+"""
+from __future__ import annotations
+
+import numpy as np
+
+import oracle
+from exact_io_aware_92_b200 import workloads as wl
+
+O_TOL_BF16 = 1.5e-2
+LSE_TOL_BF16 = 2e-3
+TOL_F32 = 1e-5
+
+
+def to_device_bf16(bits: np.ndarray):
+    import torch
+    return torch.from_numpy(np.ascontiguousarray(bits)).view(torch.bfloat16).cuda()
+
+
+def to_device_f32(x: np.ndarray):
+    import torch
+    return torch.from_numpy(np.ascontiguousarray(x, dtype=np.float32)).cuda()
+
+
+def run_bf16(inp: wl.Inputs, *, causal: bool, scale: float):
+    """CUDA path on bf16 inputs -> (O as fp64 numpy, LSE fp64 numpy)."""
+    import torch
+    from exact_io_aware_92_b200 import attention
+    q, k, v = (to_device_bf16(x) for x in (inp.q_bits, inp.k_bits, inp.v_bits))
+    sl = None if inp.seqlens is None else torch.from_numpy(inp.seqlens).cuda()
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    o, lse = attention.fwd(q, k, v, causal=causal, scale=scale, seqlens=sl, status=status)
+    rc = attention.check_status(status)
+    assert rc == 0, f"kernel status {rc}"
+    return o.float().cpu().numpy().astype(np.float64), lse.cpu().numpy().astype(np.float64)
+
+
+def run_f32(inp: wl.Inputs, *, causal: bool, scale: float):
+    import torch
+    from exact_io_aware_92_b200 import attention
+    q, k, v = (to_device_f32(x) for x in (inp.q_f32, inp.k_f32, inp.v_f32))
+    sl = None if inp.seqlens is None else torch.from_numpy(inp.seqlens).cuda()
+    o, lse = attention.fwd(q, k, v, causal=causal, scale=scale, seqlens=sl)
+    torch.cuda.synchronize()
+    return o.cpu().numpy().astype(np.float64), lse.cpu().numpy().astype(np.float64)
+
+
+def reference(inp: wl.Inputs, *, causal: bool, scale: float, rows=None):
+    """Oracle on exactly the bf16 values the kernel read (fp32-rounded scale,
+    as the kernel receives it)."""
+    return oracle.attention_forward(inp.q_bits, inp.k_bits, inp.v_bits, causal=causal,
+                                    scale=float(np.float32(scale)), seqlens=inp.seqlens,
+                                    rows=rows)
+
+
+def bf16_ulp(x: np.ndarray) -> np.ndarray:
+    """Spacing of bf16 numbers at |x| (8 significant bits)."""
+    a = np.maximum(np.abs(x), 2.0 ** -126)
+    return 2.0 ** (np.floor(np.log2(a)) - 7)
+
+
+def gather_rows(o, lse, rows):
+    """Pick per-(b, h) rows out of full [B, H, N, ...] outputs."""
+    B, H = o.shape[:2]
+    og = np.stack([o[bh // H, bh % H, rows[bh]] for bh in range(B * H)]).reshape(
+        B, H, rows.shape[1], o.shape[-1])
+    lg = np.stack([lse[bh // H, bh % H, rows[bh]] for bh in range(B * H)]).reshape(
+        B, H, rows.shape[1])
+    return og, lg
+
+
+def compare(o, lse, o_ref, lse_ref, *, o_tol, lse_tol, what=""):
+    """Element-by-element check.  Rows with no visible key must be O = 0 and
+    LSE = -inf exactly on both sides."""
+    dead = np.isneginf(lse_ref)
+    assert np.array_equal(np.isneginf(lse), dead), f"{what}: -inf LSE rows differ"
+    assert np.all(o[dead] == 0.0), f"{what}: fully masked rows must be 0"
+    assert np.all(np.isfinite(o)), f"{what}: non-finite O"
+    live = ~dead
+    err_o = np.abs(o - o_ref)
+    err_l = np.abs(lse[live] - lse_ref[live]) if np.any(live) else np.zeros(1)
+    max_o = float(err_o.max()) if err_o.size else 0.0
+    max_l = float(err_l.max()) if err_l.size else 0.0
+    if max_o > o_tol:
+        idx = np.unravel_index(np.argmax(err_o), err_o.shape)
+        ulps = err_o[idx] / bf16_ulp(o_ref[idx])
+        raise AssertionError(
+            f"{what}: max|dO| = {max_o:.3e} > {o_tol} at {idx}: gpu {o[idx]!r} ref "
+            f"{o_ref[idx]!r} ({ulps:.2f} bf16 ulps of the reference)")
+    assert max_l <= lse_tol, f"{what}: max|dLSE| = {max_l:.3e} > {lse_tol}"
+    return max_o, max_l

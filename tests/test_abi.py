@@ -1,0 +1,86 @@
+"""The C ABI library: it loads, exports every entry point include/fa.h
+declares, and rejects bad arguments synchronously (no GPU needed: argument
+checks run before any CUDA call)."""
+import os
+import re
+
+import pytest
+
+from exact_io_aware_92_b200 import _lib
+from exact_io_aware_92_b200 import build as fa_build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "fa.h")
+
+
+def declared_entry_points():
+    text = open(HEADER).read()
+    return re.findall(r"FA_API\s+[\w\s\*]*?\b(fa_\w+)\s*\(", text)
+
+
+@pytest.fixture(scope="module")
+def lib():
+    fa_build.build()
+    return _lib.load()
+
+
+def test_header_declares_the_entry_points():
+    names = declared_entry_points()
+    assert "fa_fwd" in names and "fa_fwd_ex" in names and "fa_check_status" in names
+    assert len(names) == len(set(names))
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declared_entry_points():
+        assert hasattr(lib, name), name
+        assert name in _lib.SIGNATURES, f"binding lacks a signature for {name}"
+
+
+def test_status_strings(lib):
+    for code in range(0, -11, -1):
+        assert _lib.status_string(code) != "unknown status"
+    assert _lib.status_string(-8) == "a bounded in-kernel wait ran out"
+    assert _lib.status_string(12345) == "unknown status"
+    assert lib.fa_version() == 100
+
+
+A = 4096  # a 16-byte aligned fake address: never dereferenced, checks come first
+
+
+@pytest.mark.parametrize("args,code", [
+    ((None, A, A, A, A, 1, 2, 1, 128, 64, 0.125, 0, None), _lib.FA_ERR_NULL),
+    ((A, A, A, A, None, 1, 2, 1, 128, 64, 0.125, 0, None), _lib.FA_ERR_NULL),
+    ((A, A, A, A, A, 0, 2, 1, 128, 64, 0.125, 0, None), _lib.FA_ERR_SHAPE),
+    ((A, A, A, A, A, 1, 2, 1, 0, 64, 0.125, 0, None), _lib.FA_ERR_SHAPE),
+    ((A, A, A, A, A, 1, 2, 1, 128, 64, 0.0, 0, None), _lib.FA_ERR_SHAPE),
+    ((A, A, A, A, A, 1, 2, 1, 128, 64, -1.0, 0, None), _lib.FA_ERR_SHAPE),
+    ((A, A, A, A, A, 1, 2, 1, 128, 64, float("nan"), 0, None), _lib.FA_ERR_SHAPE),
+    ((A, A, A, A, A, 1, 3, 2, 128, 64, 0.125, 0, None), _lib.FA_ERR_HEADS),
+    ((A, A, A, A, A, 1, 2, 1, 128, 96, 0.125, 0, None), _lib.FA_ERR_HEADDIM),
+    ((A, A, A, A, A, 1, 2, 1, 128, 32, 0.125, 0, None), _lib.FA_ERR_HEADDIM),
+    ((A + 8, A, A, A, A, 1, 2, 1, 128, 64, 0.125, 0, None), _lib.FA_ERR_ALIGN),
+    ((A, A, A, A + 2, A, 1, 2, 1, 128, 64, 0.125, 0, None), _lib.FA_ERR_ALIGN),
+    ((A, A, A, A, A + 2, 1, 2, 1, 128, 64, 0.125, 0, None), _lib.FA_ERR_ALIGN),
+])
+def test_bad_arguments_rejected_before_launch(lib, args, code):
+    assert lib.fa_fwd(*args) == code
+    assert lib.fa_fwd_f32(*args) == code
+
+
+def test_unknown_dtype_rejected(lib):
+    rc = lib.fa_fwd_ex(A, A, A, A, A, 1, 2, 1, 128, 64, 0.125, 0, None, 7, None, None)
+    assert rc == _lib.FA_ERR_DTYPE
+
+
+def test_hostio_requires_device_seqlens_with_host_seqlens(lib):
+    rc = lib.fa_fwd_hostio(A, A, A, A, A, A, A, A, A, A, A, None, 1, 2, 1, 128, 64, 0.125, 0, None)
+    assert rc == _lib.FA_ERR_NULL
+
+
+def test_without_a_b200_valid_calls_report_arch():
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present; covered by the gpu tests")
+    lib = _lib.load()
+    assert lib.fa_fwd(A, A, A, A, A, 1, 2, 1, 128, 64, 0.125, 0, None) == _lib.FA_ERR_ARCH
+    assert lib.fa_check_status(None, None) == _lib.FA_ERR_ARCH

@@ -1,0 +1,80 @@
+"""C ABI entry points on the GPU: the plain fa_fwd call, the host-buffer
+call, the status word and the bounded-wait self test (a wait that nothing
+satisfies must give up with FA_ERR_TIMEOUT and leave the context usable)."""
+import numpy as np
+import pytest
+
+from exact_io_aware_92_b200 import _lib
+from exact_io_aware_92_b200 import workloads as wl
+from parity_helpers import run_bf16, to_device_bf16
+
+pytestmark = pytest.mark.gpu
+
+
+def _torch():
+    import torch
+    return torch
+
+
+def test_plain_entry_point_matches_stream_entry_point():
+    torch = _torch()
+    inp = wl.draw(2, 4, 2, 333, 64, seed=8)
+    o_ref, lse_ref = run_bf16(inp, causal=True, scale=0.125)
+    q, k, v = (to_device_bf16(x) for x in (inp.q_bits, inp.k_bits, inp.v_bits))
+    o = torch.empty_like(q)
+    lse = torch.empty((2, 4, 333), dtype=torch.float32, device="cuda")
+    torch.cuda.synchronize()
+    lib = _lib.load()
+    rc = lib.fa_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
+                    2, 4, 2, 333, 64, 0.125, 1, None)
+    assert rc == _lib.FA_OK
+    assert lib.fa_check_status(None, None) == _lib.FA_OK
+    assert np.array_equal(o.float().cpu().numpy(), o_ref.astype(np.float32))
+    assert np.array_equal(lse.cpu().numpy(), lse_ref.astype(np.float32))
+
+
+def test_hostio_matches_device_call():
+    torch = _torch()
+    inp = wl.draw(3, 4, 4, 200, 128, seed=9)
+    inp.seqlens = np.array([200, 5, 130], np.int32)
+    o_ref, lse_ref = run_bf16(inp, causal=False, scale=0.0883)
+    pin = lambda a: torch.from_numpy(a).pin_memory()  # noqa: E731
+    q_h, k_h, v_h = (pin(x) for x in (inp.q_bits, inp.k_bits, inp.v_bits))
+    sl_h = pin(inp.seqlens)
+    o_h = torch.empty(q_h.shape, dtype=torch.int16).pin_memory()
+    lse_h = torch.empty((3, 4, 200), dtype=torch.float32).pin_memory()
+    q_d, k_d, v_d = (torch.empty(x.shape, dtype=torch.int16, device="cuda") for x in (q_h, k_h, v_h))
+    o_d = torch.empty_like(q_d)
+    lse_d = torch.empty((3, 4, 200), dtype=torch.float32, device="cuda")
+    sl_d = torch.empty(3, dtype=torch.int32, device="cuda")
+    from exact_io_aware_92_b200 import attention
+    attention.fwd_hostio(q_h, k_h, v_h, o_h, lse_h, q_d, k_d, v_d, o_d, lse_d, causal=False,
+                         scale=0.0883, seqlens_h=sl_h, seqlens_d=sl_d)
+    o = o_h.view(torch.bfloat16).float().numpy()
+    assert np.array_equal(o, o_ref.astype(np.float32))
+    assert np.array_equal(lse_h.numpy(), lse_ref.astype(np.float32))
+
+
+def test_bounded_wait_gives_up_and_context_survives():
+    torch = _torch()
+    lib = _lib.load()
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    stream = torch.cuda.current_stream().cuda_stream
+    assert lib.fa_selftest_bounded_wait(status.data_ptr(), 50_000_000, stream) == _lib.FA_OK
+    assert lib.fa_check_status(status.data_ptr(), stream) == _lib.FA_ERR_TIMEOUT
+    # the context is still usable afterwards
+    inp = wl.draw(1, 2, 2, 130, 64, seed=3)
+    o, lse = run_bf16(inp, causal=False, scale=0.125)
+    assert np.all(np.isfinite(o)) and np.all(np.isfinite(lse))
+
+
+def test_launch_errors_are_returned_not_raised_on_device():
+    torch = _torch()
+    lib = _lib.load()
+    q = torch.zeros((1, 2, 64, 64), dtype=torch.bfloat16, device="cuda")
+    lse = torch.zeros((1, 2, 64), dtype=torch.float32, device="cuda")
+    # misaligned output pointer: rejected before launch
+    rc = lib.fa_fwd(q.data_ptr(), q.data_ptr(), q.data_ptr(), q.data_ptr() + 2, lse.data_ptr(),
+                    1, 2, 2, 64, 64, 0.125, 0, None)
+    assert rc == _lib.FA_ERR_ALIGN
+    assert lib.fa_check_status(None, None) == _lib.FA_OK

@@ -1,0 +1,109 @@
+"""CUDA path vs the fp64 oracle, element by element, through the C ABI.
+
+Small shapes span several tiles and ragged tails (every row checked); the five
+workloads run at their full sizes in the launch configuration the benchmark
+uses, checked on every row where the oracle is quick and on seeded samples of
+rows where it is not.
+"""
+import numpy as np
+import pytest
+
+from exact_io_aware_92_b200 import workloads as wl
+from parity_helpers import (LSE_TOL_BF16, O_TOL_BF16, TOL_F32, compare, gather_rows, reference,
+                            run_bf16, run_f32)
+
+pytestmark = pytest.mark.gpu
+
+
+def _case(B, Hq, Hkv, N, d, causal, seed, seqlens=None, k_scale=1.0):
+    inp = wl.draw(B, Hq, Hkv, N, d, seed, k_scale=k_scale)
+    if seqlens is not None:
+        inp.seqlens = np.asarray(seqlens, dtype=np.int32)
+    scale = 1.0 / np.sqrt(d)
+    o, lse = run_bf16(inp, causal=causal, scale=scale)
+    o_ref, lse_ref = reference(inp, causal=causal, scale=scale)
+    return compare(o, lse, o_ref, lse_ref, o_tol=O_TOL_BF16, lse_tol=LSE_TOL_BF16,
+                   what=f"B{B} Hq{Hq} Hkv{Hkv} N{N} d{d} causal{causal} sl{seqlens}")
+
+
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("N", [1, 17, 127, 128, 129, 255, 256, 257, 383, 640])
+def test_ragged_lengths(N, d, causal):
+    _case(1, 2, 1, N, d, causal, seed=1000 + N)
+
+
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("causal", [False, True])
+def test_key_padding_edges(d, causal):
+    # lengths at 0 (no visible key), 1, around one tile, and the full N
+    _case(7, 2, 2, 512, d, causal, seed=77, seqlens=[0, 1, 63, 127, 128, 129, 512])
+
+
+@pytest.mark.parametrize("group", [1, 4, 8])
+@pytest.mark.parametrize("causal", [False, True])
+def test_gqa_groups(group, causal):
+    _case(2, 8, 8 // group, 300, 128, causal, seed=90 + group)
+
+
+def test_sharpened_scores():
+    # K scaled by 8: near one-hot rows, frequent rescaling of the running max
+    _case(1, 4, 2, 700, 128, True, seed=5, k_scale=8.0)
+    _case(1, 4, 2, 700, 64, False, seed=6, k_scale=8.0)
+
+
+def test_tiny_bf16():
+    w = wl.TINY
+    inp = wl.draw_workload(w)
+    o, lse = run_bf16(inp, causal=w.causal, scale=w.scale)
+    o_ref, lse_ref = reference(inp, causal=w.causal, scale=w.scale)
+    compare(o, lse, o_ref, lse_ref, o_tol=O_TOL_BF16, lse_tol=LSE_TOL_BF16, what=w.name)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_tiny_fp32_check_mode(causal):
+    w = wl.TINY
+    inp = wl.draw_workload(w)
+    o, lse = run_f32(inp, causal=causal, scale=w.scale)
+    o_ref, lse_ref = reference(inp, causal=causal, scale=w.scale)
+    compare(o, lse, o_ref, lse_ref, o_tol=TOL_F32, lse_tol=TOL_F32, what="tiny fp32")
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_fp32_check_mode_masks(d):
+    inp = wl.draw(2, 4, 2, 300, d, seed=321)
+    inp.seqlens = np.array([300, 77], dtype=np.int32)
+    for causal in (False, True):
+        o, lse = run_f32(inp, causal=causal, scale=1.0 / np.sqrt(d))
+        o_ref, lse_ref = reference(inp, causal=causal, scale=1.0 / np.sqrt(d))
+        compare(o, lse, o_ref, lse_ref, o_tol=TOL_F32, lse_tol=TOL_F32, what=f"fp32 d{d}")
+
+
+@pytest.mark.parametrize("w", [wl.GPT2, wl.BERT], ids=lambda w: w.name)
+def test_full_workload_every_row(w):
+    inp = wl.draw_workload(w)
+    o, lse = run_bf16(inp, causal=w.causal, scale=w.scale)
+    o_ref, lse_ref = reference(inp, causal=w.causal, scale=w.scale)
+    compare(o, lse, o_ref, lse_ref, o_tol=O_TOL_BF16, lse_tol=LSE_TOL_BF16, what=w.name)
+
+
+@pytest.mark.parametrize("w", [wl.LLAMA_GQA, wl.LONG], ids=lambda w: w.name)
+def test_full_workload_sampled_rows(w):
+    inp = wl.draw_workload(w)
+    o, lse = run_bf16(inp, causal=w.causal, scale=w.scale)
+    assert np.all(np.isfinite(o)) and np.all(np.isfinite(lse))
+    rows = wl.sample_rows(w)
+    # always include the first and last rows of every head
+    rows[:, 0] = 0
+    rows[:, -1] = w.N - 1
+    rows.sort(axis=1)
+    o_ref, lse_ref = reference(inp, causal=w.causal, scale=w.scale, rows=rows)
+    og, lg = gather_rows(o, lse, rows)
+    compare(og, lg, o_ref, lse_ref, o_tol=O_TOL_BF16, lse_tol=LSE_TOL_BF16, what=w.name)
+
+
+def test_deterministic():
+    inp = wl.draw(2, 8, 2, 1000, 128, seed=55)
+    a = run_bf16(inp, causal=True, scale=0.088)
+    b = run_bf16(inp, causal=True, scale=0.088)
+    assert np.array_equal(a[0], b[0]) and np.array_equal(a[1], b[1])
