@@ -45,6 +45,18 @@ def load_peaks():
         return FALLBACK_PEAKS, "fallback"
 
 
+def kernel_source_hash() -> str:
+    import glob
+    import hashlib
+    files = sorted(glob.glob(os.path.join(ROOT, "exact_io_aware_92_b200", "csrc", "*")))
+    files.append(os.path.join(ROOT, "include", "fa.h"))
+    h = hashlib.sha256()
+    for f in files:
+        with open(f, "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
 def dist_env():
     return (int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")),
             int(os.environ.get("LOCAL_RANK", "0")))
@@ -281,7 +293,9 @@ def run_mine(args, w: wl.Workload):
     traffic_file = os.path.join(ROOT, "profiles", "traffic.json")
     if os.path.exists(traffic_file):
         with open(traffic_file) as f:
-            traffic = json.load(f).get(w.name)
+            tj = json.load(f)
+        if tj.get("kernel_source_sha256_16") == kernel_source_hash():
+            traffic = tj.get(w.name)
     cpu, _ = time_oracle(w, inp, budget_s=args.cpu_budget) if not args.no_cpu_baseline else (
         None, None)
     line = {

@@ -74,9 +74,16 @@ def gather_rows(o, lse, rows):
     return og, lg
 
 
-def compare(o, lse, o_ref, lse_ref, *, o_tol, lse_tol, what=""):
+def compare(o, lse, o_ref, lse_ref, *, o_tol, lse_tol, what="", rounding_bound=False):
     """Element-by-element check.  Rows with no visible key must be O = 0 and
-    LSE = -inf exactly on both sides."""
+    LSE = -inf exactly on both sides.
+
+    rounding_bound: for stress inputs outside the stated workloads, where
+    |O_ref| >= 4 makes half a bf16 ulp (1/64) exceed 1.5e-2 so that no bf16
+    output can meet it, an element also passes when its error is within the
+    bf16 output rounding plus the bf16 rounding of P:
+        |dO| <= 0.5 * ulp_bf16(O_ref) + 2^-8 * |O_ref|.
+    The count of elements that needed it is returned."""
     dead = np.isneginf(lse_ref)
     assert np.array_equal(np.isneginf(lse), dead), f"{what}: -inf LSE rows differ"
     assert np.all(o[dead] == 0.0), f"{what}: fully masked rows must be 0"
@@ -86,6 +93,13 @@ def compare(o, lse, o_ref, lse_ref, *, o_tol, lse_tol, what=""):
     err_l = np.abs(lse[live] - lse_ref[live]) if np.any(live) else np.zeros(1)
     max_o = float(err_o.max()) if err_o.size else 0.0
     max_l = float(err_l.max()) if err_l.size else 0.0
+    n_rounding = 0
+    if rounding_bound and max_o > o_tol:
+        bound = np.maximum(o_tol, 0.5 * bf16_ulp(o_ref) + 2.0 ** -8 * np.abs(o_ref))
+        over = err_o > o_tol
+        n_rounding = int(over.sum())
+        err_o = np.where(err_o <= bound, 0.0, err_o)
+        max_o = float(err_o.max())
     if max_o > o_tol:
         idx = np.unravel_index(np.argmax(err_o), err_o.shape)
         ulps = err_o[idx] / bf16_ulp(o_ref[idx])
@@ -93,4 +107,4 @@ def compare(o, lse, o_ref, lse_ref, *, o_tol, lse_tol, what=""):
             f"{what}: max|dO| = {max_o:.3e} > {o_tol} at {idx}: gpu {o[idx]!r} ref "
             f"{o_ref[idx]!r} ({ulps:.2f} bf16 ulps of the reference)")
     assert max_l <= lse_tol, f"{what}: max|dLSE| = {max_l:.3e} > {lse_tol}"
-    return max_o, max_l
+    return max_o, max_l, n_rounding
