@@ -145,13 +145,16 @@ int launch_bf16(DeviceState *ds, const void *q, const void *k, const void *v, vo
   p.Hkv = Hkv;
   p.N = N;
   p.group = Hq / Hkv;
-  p.num_qpairs = (N + C::ROWS_PER_CTA - 1) / C::ROWS_PER_CTA;
+  p.num_qpairs = (N + C::ROWS_PER_UNIT - 1) / C::ROWS_PER_UNIT;
   p.causal = causal ? 1 : 0;
   p.scale_log2 = scale * kLog2e;
   p.wait_limit_ns = kWaitLimitNs;
-  const long long grid = static_cast<long long>(B) * Hq * p.num_qpairs;
-  if (grid > 0x7fffffffll) return FA_ERR_SHAPE;
-  kernel<<<static_cast<unsigned>(grid), C::THREADS, C::SMEM_ALLOC, stream>>>(tq, tk, tv, p);
+  const long long units = static_cast<long long>(B) * Hq * p.num_qpairs;
+  if (units > 0x7fffffffll) return FA_ERR_SHAPE;
+  p.num_units = static_cast<int>(units);
+  // Persistent: one CTA per SM (or per unit when there are fewer units).
+  const int grid = static_cast<int>(units < ds->num_sms ? units : ds->num_sms);
+  kernel<<<grid, C::THREADS, C::SMEM_ALLOC, stream>>>(tq, tk, tv, p);
   if (cudaGetLastError() != cudaSuccess) return FA_ERR_LAUNCH;
   return FA_OK;
 }

@@ -49,6 +49,27 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
+// Per-warpgroup register budget (all four warps of a warpgroup execute it).
+template <uint32_t N>
+__device__ __forceinline__ void regs_increase() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <uint32_t N>
+__device__ __forceinline__ void regs_decrease() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+
+// One lane of a converged warp (the lowest active one) gets true.
+__device__ __forceinline__ bool elect_one() {
+  uint32_t is_leader;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "elect.sync _|p, 0xffffffff;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(is_leader));
+  return is_leader != 0;
+}
+
 __device__ __forceinline__ uint64_t global_timer_ns() {
   uint64_t t;
   asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
@@ -258,6 +279,39 @@ __device__ __forceinline__ uint64_t add_f32x2(uint64_t a, uint64_t b) {
   uint64_t r;
   asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
   return r;
+}
+
+// 2^x for a pair of arguments on the FMA pipe instead of the MUFU pipe.
+// x = n + f with n = round(x) (adding 1.5 * 2^23 rounds an fp32 to the
+// nearest integer and leaves n in the low mantissa bits), f in [-1/2, 1/2];
+// 2^f by a degree-3 minimax polynomial (relative error 7.5e-5, derived by
+// exp2_poly.py with the Remez exchange algorithm); n is added to the
+// exponent field.  x is clamped at -127 and results whose exponent field
+// would go negative become +0, so x = -inf gives exactly 0.
+struct Exp2Poly {
+  static constexpr float C0 = 0.9999280571937561f;
+  static constexpr float C1 = 0.6932609677314758f;
+  static constexpr float C2 = 0.2426111251115799f;
+  static constexpr float C3 = 0.0551716685295105f;
+  static constexpr float ROUND = 12582912.0f;  // 1.5 * 2^23
+};
+
+__device__ __forceinline__ void exp2_poly_pair(float x0, float x1, float &y0, float &y1) {
+  using E = Exp2Poly;
+  const uint64_t x2 = f32x2(fmaxf(x0, -127.0f), fmaxf(x1, -127.0f));
+  const uint64_t t2 = add_f32x2(x2, f32x2(E::ROUND, E::ROUND));
+  const uint64_t r2 = add_f32x2(t2, f32x2(-E::ROUND, -E::ROUND));
+  const uint64_t f2 = fma_f32x2(r2, f32x2(-1.0f, -1.0f), x2);
+  uint64_t p2 = fma_f32x2(f32x2(E::C3, E::C3), f2, f32x2(E::C2, E::C2));
+  p2 = fma_f32x2(p2, f2, f32x2(E::C1, E::C1));
+  p2 = fma_f32x2(p2, f2, f32x2(E::C0, E::C0));
+  float t0, t1, p0, p1;
+  f32x2_split(t2, t0, t1);
+  f32x2_split(p2, p0, p1);
+  const int b0 = (__float_as_int(t0) << 23) + __float_as_int(p0);
+  const int b1 = (__float_as_int(t1) << 23) + __float_as_int(p1);
+  y0 = __int_as_float(max(b0, 0));
+  y1 = __int_as_float(max(b1, 0));
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
