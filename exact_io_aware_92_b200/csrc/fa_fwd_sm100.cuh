@@ -401,8 +401,7 @@ __device__ void role_softmax(const Sm100Ctx<D> &x, const FwdParams &p, int t) {
     const int limit = p.causal ? min(w.L, i + 1) : w.L;  // visible keys are [0, limit)
 
     float m_ref = -INFINITY;  // reference max (log2 units) the exponentials use
-    float l_exact = 0.f;      // row sum of the fp32 probabilities (for LSE)
-    float l_round = 0.f;      // row sum of the bf16-rounded probabilities (divides O)
+    float l = 0.f;            // row sum of the fp32 probabilities relative to m_ref
     for (int j = 0; j < w.nkv; ++j) {
       if (!wait_all(C::BAR_S_FULL + t, static_cast<uint32_t>((g + j) & 1))) return;
       tc_fence_after();
@@ -440,20 +439,16 @@ __device__ void role_softmax(const Sm100Ctx<D> &x, const FwdParams &p, int t) {
       const bool need = m_new > m_ref + C::RESCALE_THRESHOLD;
       const float alpha = need ? ex2_approx(m_ref - m_new) : 1.0f;
       if (need) {
-        l_exact *= alpha;
-        l_round *= alpha;
+        l *= alpha;
         m_ref = m_new;
       }
       const float m_use = (m_ref == -INFINITY) ? 0.0f : m_ref;
-      // p = 2^(s * scale * log2(e) - m_ref), rounded to bf16 for the PV
-      // product.  l_round adds the same rounded values, so the weights applied
-      // to V sum to exactly one after the final division; l_exact keeps the
-      // unrounded sum for the log-sum-exp.  Each half of the keys is published
-      // as soon as it is in tensor memory.
+      // p = 2^(s * scale * log2(e) - m_ref); the row sum takes p in fp32
+      // and the PV product its bf16 rounding.  Each half of the keys is
+      // published as soon as it is in tensor memory.
       const uint64_t scale2 = f32x2(sl2, sl2);
       const uint64_t shift2 = f32x2(-m_use, -m_use);
-      uint64_t sum_e = f32x2(0.f, 0.f);
-      uint64_t sum_r = f32x2(0.f, 0.f);
+      uint64_t sum2 = f32x2(0.f, 0.f);
 #pragma unroll
       for (int half = 0; half < 2; ++half) {
         uint32_t pk[32];
@@ -471,9 +466,7 @@ __device__ void role_softmax(const Sm100Ctx<D> &x, const FwdParams &p, int t) {
             p1 = ex2_approx(x1);
           }
           pk[e] = pack_bf16x2(p0, p1);
-          sum_e = add_f32x2(sum_e, f32x2(p0, p1));
-          sum_r = add_f32x2(sum_r, f32x2(__uint_as_float(pk[e] << 16),
-                                         __uint_as_float(pk[e] & 0xFFFF0000u)));
+          sum2 = add_f32x2(sum2, f32x2(p0, p1));
         }
         tmem_st32(tS + 32 * half, pk);
         // O holds earlier tiles' sum only for j > 0; nothing writes it until
@@ -495,16 +488,14 @@ __device__ void role_softmax(const Sm100Ctx<D> &x, const FwdParams &p, int t) {
         mbar_arrive(x.bar(C::BAR_P_HALF + 2 * t + half));
       }
       float a0, a1;
-      f32x2_split(sum_e, a0, a1);
-      l_exact += a0 + a1;
-      f32x2_split(sum_r, a0, a1);
-      l_round += a0 + a1;
+      f32x2_split(sum2, a0, a1);
+      l += a0 + a1;
     }
 
-    // Epilogue: O = O~ / l_round in bf16, LSE = (m_ref + log2 l_exact) * ln 2.
+    // Epilogue: O = O~ / l in bf16, LSE = (m_ref + log2 l) * ln 2.
     if (!wait_all(C::BAR_O_FULL + t, static_cast<uint32_t>(qi & 1))) return;
     tc_fence_after();
-    const float inv_l = l_round > 0.f ? 1.0f / l_round : 0.0f;
+    const float inv_l = l > 0.f ? 1.0f / l : 0.0f;
     uint16_t *orow = p.o + (static_cast<size_t>(w.bh) * p.N + (valid ? i : 0)) * D;
 #pragma unroll
     for (int c = 0; c < D / 32; ++c) {
@@ -525,7 +516,7 @@ __device__ void role_softmax(const Sm100Ctx<D> &x, const FwdParams &p, int t) {
     }
     if (valid)
       p.lse[static_cast<size_t>(w.bh) * p.N + i] =
-          l_exact > 0.f ? (m_ref + __log2f(l_exact)) * 0.69314718055994530942f : -INFINITY;
+          l > 0.f ? (m_ref + __log2f(l)) * 0.69314718055994530942f : -INFINITY;
     g += w.nkv;
     ++qi;
   }
