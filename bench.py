@@ -323,6 +323,46 @@ def run_mine(args, w: wl.Workload):
     return 0
 
 
+def report_all_workloads(args):
+    """Throughput of the forward on each of the five workloads (one GPU),
+    one JSON object per line; not the contract line."""
+    import torch
+    from exact_io_aware_92_b200 import attention
+    peaks, src = load_peaks()
+    peak = float(peaks["bf16_tflops"])
+    dev = torch.device("cuda", 0)
+    for w in wl.ALL:
+        inp = wl.draw_workload(w)
+        q, k, v = (torch.from_numpy(x).view(torch.bfloat16).to(dev)
+                   for x in (inp.q_bits, inp.k_bits, inp.v_bits))
+        sl = None if inp.seqlens is None else torch.from_numpy(inp.seqlens).to(dev)
+        o = torch.empty_like(q)
+        lse = torch.empty((w.B, w.Hq, w.N), dtype=torch.float32, device=dev)
+        flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
+        in_bytes = sum(t.numel() * t.element_size() for t in (q, k, v))
+        for _ in range(args.warmup):
+            attention.fwd(q, k, v, causal=w.causal, scale=w.scale, seqlens=sl, out=o, lse=lse)
+        torch.cuda.synchronize(dev)
+        times = []
+        for _ in range(args.steps):
+            if in_bytes < L2_BYTES:
+                flush.zero_()  # inputs smaller than L2: evict them between steps
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            attention.fwd(q, k, v, causal=w.causal, scale=w.scale, seqlens=sl, out=o, lse=lse)
+            e1.record()
+            e1.synchronize()
+            times.append(e0.elapsed_time(e1))
+        ms = statistics.median(times)
+        f = wl.flops(w, inp.seqlens)
+        algo_bytes = in_bytes + o.numel() * 2 + lse.numel() * 4
+        print(json.dumps({"workload": w.name, "ms_median": ms, "tflops": f / ms / 1e9,
+                          "frac_of_peak": f / ms / 1e9 / peak, "hbm_gbs": algo_bytes / ms / 1e6,
+                          "flops": f, "algorithmic_bytes": algo_bytes,
+                          "l2": "flushed between steps" if in_bytes < L2_BYTES else "inputs > L2",
+                          "peak_source": src}), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -335,9 +375,13 @@ def main():
     ap.add_argument("--ref-budget", type=float, default=8.0,
                     help="seconds of CPU work per reference-arm step")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--all-workloads", action="store_true",
+                    help="report per-workload throughput for the five workloads instead")
     ap.add_argument("--batch", type=int, default=None,
                     help="override the workload's batch size (profiling a smaller case)")
     args = ap.parse_args()
+    if args.all_workloads:
+        return report_all_workloads(args)
     w = wl.BY_NAME[args.workload]
     if args.batch is not None:
         import dataclasses

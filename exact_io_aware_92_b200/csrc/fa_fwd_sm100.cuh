@@ -420,38 +420,11 @@ __device__ void role_softmax(const Sm100Ctx<D> &x, const FwdParams &p, int t) {
         for (int c = 0; c < 128; ++c)
           if (kbase + c >= limit) s[c] = __float_as_uint(-INFINITY);
       }
-      // Row max in eight independent chains of 3-input maxima.
-      float mq[8];
-#pragma unroll
-      for (int q = 0; q < 8; ++q) {
-        const uint32_t *sq = s + 16 * q;
-        mq[q] = fmax3(__uint_as_float(sq[0]), __uint_as_float(sq[1]), __uint_as_float(sq[2]));
-#pragma unroll
-        for (int c = 3; c < 15; c += 2)
-          mq[q] = fmax3(mq[q], __uint_as_float(sq[c]), __uint_as_float(sq[c + 1]));
-        mq[q] = fmaxf(mq[q], __uint_as_float(sq[15]));
-      }
-      const float mx =
-          fmaxf(fmax3(mq[0], mq[1], mq[2]), fmax3(fmax3(mq[3], mq[4], mq[5]), mq[6], mq[7]));
-      const float m_new = fmaxf(m_ref, mx * sl2);
-
-      // Lazy correction: move m_ref (and rescale l and O) only on a big jump.
-      const bool need = m_new > m_ref + C::RESCALE_THRESHOLD;
-      const float alpha = need ? ex2_approx(m_ref - m_new) : 1.0f;
-      if (need) {
-        l *= alpha;
-        m_ref = m_new;
-      }
-      const float m_use = (m_ref == -INFINITY) ? 0.0f : m_ref;
-      // p = 2^(s * scale * log2(e) - m_ref); the row sum takes p in fp32
-      // and the PV product its bf16 rounding.  Each half of the keys is
-      // published as soon as it is in tensor memory.
+      // p = 2^(s * scale * log2(e) - m_ref) for 64 keys: the row sum takes
+      // p in fp32 and the PV product its bf16 rounding.
       const uint64_t scale2 = f32x2(sl2, sl2);
-      const uint64_t shift2 = f32x2(-m_use, -m_use);
-      uint64_t sum2 = f32x2(0.f, 0.f);
-#pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        uint32_t pk[32];
+      auto exp_half = [&](int half, float m_use, uint32_t(&pk)[32], uint64_t &sum2) {
+        const uint64_t shift2 = f32x2(-m_use, -m_use);
 #pragma unroll
         for (int e = 0; e < 32; ++e) {
           const int c = half * 64 + 2 * e;
@@ -468,25 +441,76 @@ __device__ void role_softmax(const Sm100Ctx<D> &x, const FwdParams &p, int t) {
           pk[e] = pack_bf16x2(p0, p1);
           sum2 = add_f32x2(sum2, f32x2(p0, p1));
         }
-        tmem_st32(tS + 32 * half, pk);
-        // O holds earlier tiles' sum only for j > 0; nothing writes it until
-        // this warpgroup publishes P (the PV product of tile j-1 finished
-        // before S_j did).  It is rescaled before the first half goes out.
-        if (half == 0 && j > 0 && __any_sync(0xffffffffu, need)) {
+      };
+      // Row max in eight independent chains of 3-input maxima.
+      auto row_max = [&]() {
+        float mq[8];
 #pragma unroll
-          for (int c = 0; c < D / 32; ++c) {
-            uint32_t o[32];
-            tmem_ld32(tO + 32 * c, o);
-            tmem_wait_ld();
+        for (int q = 0; q < 8; ++q) {
+          const uint32_t *sq = s + 16 * q;
+          mq[q] = fmax3(__uint_as_float(sq[0]), __uint_as_float(sq[1]), __uint_as_float(sq[2]));
 #pragma unroll
-            for (int e2 = 0; e2 < 32; ++e2) o[e2] = __float_as_uint(__uint_as_float(o[e2]) * alpha);
-            tmem_st32(tO + 32 * c, o);
-          }
+          for (int c = 3; c < 15; c += 2)
+            mq[q] = fmax3(mq[q], __uint_as_float(sq[c]), __uint_as_float(sq[c + 1]));
+          mq[q] = fmaxf(mq[q], __uint_as_float(sq[15]));
         }
-        tmem_wait_st();
-        tc_fence_before();
-        mbar_arrive(x.bar(C::BAR_P_HALF + 2 * t + half));
+        return fmaxf(fmax3(mq[0], mq[1], mq[2]), fmax3(fmax3(mq[3], mq[4], mq[5]), mq[6], mq[7]));
+      };
+
+      uint32_t pk[32];
+      uint64_t sum2 = f32x2(0.f, 0.f);
+      bool need;
+      float alpha = 1.0f;
+      if (j > 0) {
+        // The first half's exponentials start against the current reference
+        // while the row max is found: the reference moves only when the max
+        // rose by more than the threshold, which after the first tile is rare.
+        exp_half(0, (m_ref == -INFINITY) ? 0.0f : m_ref, pk, sum2);
+        const float m_new = fmaxf(m_ref, row_max() * sl2);
+        need = m_new > m_ref + C::RESCALE_THRESHOLD;
+        if (__any_sync(0xffffffffu, need)) {
+          if (need) {
+            alpha = ex2_approx(m_ref - m_new);
+            l *= alpha;
+            m_ref = m_new;
+          }
+          const float m_use = (m_ref == -INFINITY) ? 0.0f : m_ref;
+          sum2 = f32x2(0.f, 0.f);
+          exp_half(0, m_use, pk, sum2);
+        }
+      } else {
+        // First tile of the unit: the reference is the tile's row max.
+        const float m_new = row_max() * sl2;
+        need = true;
+        m_ref = m_new;
+        l = 0.f;
+        exp_half(0, (m_ref == -INFINITY) ? 0.0f : m_ref, pk, sum2);
       }
+      const float m_use = (m_ref == -INFINITY) ? 0.0f : m_ref;
+      tmem_st32(tS, pk);
+      // O holds earlier tiles' sum only for j > 0; nothing writes it until
+      // this warpgroup publishes P (the PV product of tile j-1 finished
+      // before S_j did).  It is rescaled before the first half goes out.
+      if (j > 0 && __any_sync(0xffffffffu, need)) {
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t o[32];
+          tmem_ld32(tO + 32 * c, o);
+          tmem_wait_ld();
+#pragma unroll
+          for (int e2 = 0; e2 < 32; ++e2) o[e2] = __float_as_uint(__uint_as_float(o[e2]) * alpha);
+          tmem_st32(tO + 32 * c, o);
+        }
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(x.bar(C::BAR_P_HALF + 2 * t));
+      // Second half of the keys.
+      exp_half(1, m_use, pk, sum2);
+      tmem_st32(tS + 32, pk);
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(x.bar(C::BAR_P_HALF + 2 * t + 1));
       float a0, a1;
       f32x2_split(sum2, a0, a1);
       l += a0 + a1;
