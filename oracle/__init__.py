@@ -26,6 +26,13 @@ def open_library(path: str):
     """Bind a compiled copy of attention_ref.c (the default one, or a test's
     deliberately mutated copy)."""
     lib = ctypes.CDLL(path)
+    lib.oracle_attention_fwd_general.restype = ctypes.c_int
+    lib.oracle_attention_fwd_general.argtypes = [
+        ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int,
+        ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+        ctypes.c_double, ctypes.c_int, ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p,
+        ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int,
+    ]
     lib.oracle_attention_fwd.restype = ctypes.c_int
     lib.oracle_attention_fwd.argtypes = [
         ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int,
@@ -51,14 +58,16 @@ def num_threads() -> int:
 
 def attention_forward(q, k, v, *, causal: bool, scale: float, seqlens=None, rows=None,
                       return_probs: bool = False, threads: int | None = None,
-                      _lib_override=None):
+                      causal_bottom_right: bool = False, _lib_override=None):
     """Exact softmax attention in fp64.
 
-    q: [B, Hq, N, d]; k, v: [B, Hkv, N, d]; dtype float64, float32 or uint16
+    q: [B, Hq, Nq, d]; k, v: [B, Hkv, Nk, d]; dtype float64, float32 or uint16
     (bf16 bit patterns).  seqlens: int [B] key lengths or None.  rows: int
     [B*Hq, R] query rows per (batch, head) or None for all rows.
+    causal_bottom_right: with causal, query i sits at position len_b - Nq + i
+    (key j visible iff j <= i + len_b - Nq); otherwise causal is top-left.
 
-    Returns (o [B, Hq, R, d], lse [B, Hq, R]) in fp64, plus P [B, Hq, R, N]
+    Returns (o [B, Hq, R, d], lse [B, Hq, R]) in fp64, plus P [B, Hq, R, Nk]
     when return_probs is set (small cases only).
     """
     q = np.ascontiguousarray(q)
@@ -66,37 +75,37 @@ def attention_forward(q, k, v, *, causal: bool, scale: float, seqlens=None, rows
     v = np.ascontiguousarray(v)
     if not (q.dtype == k.dtype == v.dtype) or q.dtype not in _IN_KIND:
         raise TypeError("q, k, v must share one dtype among float64, float32, uint16(bf16)")
-    B, Hq, N, d = q.shape
+    B, Hq, Nq, d = q.shape
     Bk, Hkv, Nk, dk = k.shape
-    if (Bk, Nk, dk) != (B, N, d) or v.shape != k.shape:
+    if (Bk, dk) != (B, d) or v.shape != k.shape:
         raise ValueError("shape mismatch between q and k/v")
     if Hq % Hkv:
         raise ValueError("Hq must be a multiple of Hkv")
     sl = None
     if seqlens is not None:
         sl = np.ascontiguousarray(seqlens, dtype=np.int32)
-        if sl.shape != (B,) or np.any(sl < 0) or np.any(sl > N):
-            raise ValueError("seqlens must be int[B] within [0, N]")
+        if sl.shape != (B,) or np.any(sl < 0) or np.any(sl > Nk):
+            raise ValueError("seqlens must be int[B] within [0, Nk]")
     if rows is None:
-        R = N
+        R = Nq
         rw = None
     else:
         rw = np.ascontiguousarray(rows, dtype=np.int64)
-        if rw.ndim != 2 or rw.shape[0] != B * Hq or np.any(rw < 0) or np.any(rw >= N):
-            raise ValueError("rows must be int[B*Hq, R] within [0, N)")
+        if rw.ndim != 2 or rw.shape[0] != B * Hq or np.any(rw < 0) or np.any(rw >= Nq):
+            raise ValueError("rows must be int[B*Hq, R] within [0, Nq)")
         R = rw.shape[1]
     o = np.empty((B, Hq, R, d), dtype=np.float64)
     lse = np.empty((B, Hq, R), dtype=np.float64)
-    p = np.empty((B, Hq, R, N), dtype=np.float64) if return_probs else None
+    p = np.empty((B, Hq, R, Nk), dtype=np.float64) if return_probs else None
 
     def ptr(a):
         return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
 
     lib = _lib_override if _lib_override is not None else _load()
-    rc = lib.oracle_attention_fwd(
-        ptr(q), ptr(k), ptr(v), _IN_KIND[q.dtype], B, Hq, Hkv, N, d, float(scale),
-        int(bool(causal)), ptr(sl), ptr(rw), R, ptr(o), ptr(lse), ptr(p),
-        int(threads or num_threads()))
+    rc = lib.oracle_attention_fwd_general(
+        ptr(q), ptr(k), ptr(v), _IN_KIND[q.dtype], B, Hq, Hkv, Nq, Nk, d, float(scale),
+        int(bool(causal)), int(bool(causal_bottom_right)), ptr(sl), ptr(rw), R, ptr(o),
+        ptr(lse), ptr(p), int(threads or num_threads()))
     if rc != 0:
         raise RuntimeError(f"oracle_attention_fwd failed ({rc})")
     return (o, lse, p) if return_probs else (o, lse)

@@ -32,6 +32,12 @@
  * contiguous (query heads [g*G, (g+1)*G) share kv head g), LSE is the
  * natural log.
  *
+ * Queries and keys may have different lengths (Nq query rows against Nk keys,
+ * the decode case the wiki note's "common misconceptions" section mentions):
+ * with causal_bottom_right set, query i is the (len_b - Nq + i)-th position
+ * of its sequence, so key j is visible iff j <= i + len_b - Nq; otherwise
+ * causal stays top-left (j <= i).
+ *
  * S and P are materialised per block of query rows, exactly as defined.
  * Blocks are independent and run on a pool of POSIX threads.
  */
@@ -57,7 +63,7 @@ static double in_at(const void *base, int kind, int64_t idx) {
 
 typedef struct {
   const void *q, *k, *v;
-  int in_kind, B, Hq, Hkv, N, d, causal, R, nblk;
+  int in_kind, B, Hq, Hkv, Nq, N, d, causal, bottom_right, R, nblk;
   double scale;
   const int32_t *seqlens;
   const int64_t *rows;
@@ -78,7 +84,8 @@ static void run_block(const job_t *J, int64_t t, double *S, double *qrow) {
   int len = J->seqlens ? J->seqlens[b] : N;
   if (len < 0) len = 0;
   if (len > N) len = N;
-  const int64_t qbase = ((int64_t)b * J->Hq + h) * N * d;
+  const int64_t qbase = ((int64_t)b * J->Hq + h) * J->Nq * d;
+  const int64_t off = J->bottom_right ? (int64_t)len - J->Nq : 0;
   const int64_t kvbase = ((int64_t)b * J->Hkv + g) * N * d;
   const int r0 = blk * ORACLE_ROW_BLOCK;
   const int r1 = (r0 + ORACLE_ROW_BLOCK < R) ? r0 + ORACLE_ROW_BLOCK : R;
@@ -89,7 +96,7 @@ static void run_block(const job_t *J, int64_t t, double *S, double *qrow) {
     double *Srow = S + (size_t)(r - r0) * N;
     for (int c = 0; c < d; ++c) qrow[c] = in_at(J->q, J->in_kind, qbase + i * d + c);
     for (int j = 0; j < N; ++j) {
-      const int visible = (j < len) && (!J->causal || j <= i);
+      const int visible = (j < len) && (!J->causal || j <= i + off);
       if (!visible) {
         Srow[j] = -INFINITY;
         continue;
@@ -147,29 +154,33 @@ static void *worker(void *arg) {
 }
 
 /*
- * q: [B, Hq, N, d]; k, v: [B, Hkv, N, d]; element type given by in_kind.
- * seqlens: int32 [B] key lengths (0 <= len_b <= N) or NULL for N.
- * rows: int64 [B*Hq, R] query rows to compute per (b, h), or NULL for all N
- *       (then R must equal N).
+ * q: [B, Hq, Nq, d]; k, v: [B, Hkv, Nk, d]; element type given by in_kind.
+ * seqlens: int32 [B] key lengths (0 <= len_b <= Nk) or NULL for Nk.
+ * causal: 0/1; causal_bottom_right: 0 = top-left (j <= i), 1 = bottom-right
+ *       (j <= i + len_b - Nq).
+ * rows: int64 [B*Hq, R] query rows to compute per (b, h), or NULL for all Nq
+ *       (then R must equal Nq).
  * o: fp64 [B*Hq, R, d]; lse: fp64 [B*Hq, R].
- * p_out: optional fp64 [B*Hq, R, N], the probability rows P[i][:].
+ * p_out: optional fp64 [B*Hq, R, Nk], the probability rows P[i][:].
  * nthreads: worker threads (>= 1); tasks are independent blocks of rows, so
  *           the result does not depend on it.
  * Returns 0, or -1 on a bad argument or an allocation failure.
  */
-int oracle_attention_fwd(const void *q, const void *k, const void *v, int in_kind, int B, int Hq,
-                         int Hkv, int N, int d, double scale, int causal,
-                         const int32_t *seqlens, const int64_t *rows, int R, double *o,
-                         double *lse, double *p_out, int nthreads) {
+int oracle_attention_fwd_general(const void *q, const void *k, const void *v, int in_kind, int B,
+                                 int Hq, int Hkv, int Nq, int Nk, int d, double scale, int causal,
+                                 int causal_bottom_right, const int32_t *seqlens,
+                                 const int64_t *rows, int R, double *o, double *lse,
+                                 double *p_out, int nthreads) {
   if (!q || !k || !v || !o || !lse) return -1;
-  if (B <= 0 || Hq <= 0 || Hkv <= 0 || N <= 0 || d <= 0 || R <= 0) return -1;
+  if (B <= 0 || Hq <= 0 || Hkv <= 0 || Nq <= 0 || Nk <= 0 || d <= 0 || R <= 0) return -1;
   if (Hq % Hkv != 0) return -1;
-  if (!rows && R != N) return -1;
+  if (!rows && R != Nq) return -1;
   if (in_kind < ORACLE_IN_F64 || in_kind > ORACLE_IN_BF16) return -1;
   job_t J;
   memset(&J, 0, sizeof J);
   J.q = q; J.k = k; J.v = v; J.in_kind = in_kind;
-  J.B = B; J.Hq = Hq; J.Hkv = Hkv; J.N = N; J.d = d; J.causal = causal; J.R = R;
+  J.B = B; J.Hq = Hq; J.Hkv = Hkv; J.Nq = Nq; J.N = Nk; J.d = d; J.causal = causal;
+  J.bottom_right = causal_bottom_right; J.R = R;
   J.scale = scale; J.seqlens = seqlens; J.rows = rows; J.o = o; J.lse = lse; J.p_out = p_out;
   J.nblk = (R + ORACLE_ROW_BLOCK - 1) / ORACLE_ROW_BLOCK;
   J.total = (int64_t)B * Hq * J.nblk;
@@ -186,4 +197,13 @@ int oracle_attention_fwd(const void *q, const void *k, const void *v, int in_kin
   for (int t = 1; t <= started; ++t) pthread_join(th[t], NULL);
   free(th);
   return J.bad ? -1 : 0;
+}
+
+/* Square case (Nq = Nk = N, causal top-left): the problem the pages state. */
+int oracle_attention_fwd(const void *q, const void *k, const void *v, int in_kind, int B, int Hq,
+                         int Hkv, int N, int d, double scale, int causal,
+                         const int32_t *seqlens, const int64_t *rows, int R, double *o,
+                         double *lse, double *p_out, int nthreads) {
+  return oracle_attention_fwd_general(q, k, v, in_kind, B, Hq, Hkv, N, N, d, scale, causal, 0,
+                                      seqlens, rows, R, o, lse, p_out, nthreads);
 }

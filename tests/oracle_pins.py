@@ -141,18 +141,19 @@ def pin_matches_torch_sdpa(fwd):
         np.testing.assert_allclose(lse, torch.logsumexp(s, dim=-1).numpy(), rtol=0, atol=1e-12)
 
 
-def _brute(q, k, v, causal, scale, seqlens):
+def _brute(q, k, v, causal, scale, seqlens, bottom_right=False):
     """Two passes per row in plain Python with math.exp: max, then sums."""
-    B, Hq, N, d = q.shape
-    Hkv = k.shape[1]
+    B, Hq, Nq, d = q.shape
+    Hkv, Nk = k.shape[1], k.shape[2]
     o = np.zeros_like(q)
-    lse = np.zeros((B, Hq, N))
+    lse = np.zeros((B, Hq, Nq))
     for b in range(B):
-        L = N if seqlens is None else int(seqlens[b])
+        L = Nk if seqlens is None else int(seqlens[b])
+        off = L - Nq if bottom_right else 0
         for h in range(Hq):
             g = h // (Hq // Hkv)
-            for i in range(N):
-                vis = [j for j in range(N) if j < L and (not causal or j <= i)]
+            for i in range(Nq):
+                vis = [j for j in range(Nk) if j < L and (not causal or j <= i + off)]
                 s = {j: scale * math.fsum(float(q[b, h, i, c]) * float(k[b, g, j, c])
                                           for c in range(d)) for j in vis}
                 mx = max(s.values())
@@ -263,9 +264,69 @@ def pin_input_encodings_agree(fwd):
         np.testing.assert_array_equal(l, res[0][1])
 
 
+def pin_cross_length_matches_torch_sdpa(fwd):
+    """Nq query rows against Nk keys (the decode shape), causal aligned to the
+    end of each sequence's keys, against torch SDPA in fp64 with the same
+    explicit mask, and against the pure-Python two-pass softmax."""
+    import torch
+    import torch.nn.functional as F
+
+    for (B, Hq, Hkv, Nq, Nk, d, causal, sl, seed) in [
+        (2, 4, 2, 1, 37, 8, True, [37, 9], 51),
+        (2, 4, 1, 3, 50, 16, True, [50, 4], 52),
+        (1, 2, 2, 5, 23, 4, False, None, 53),
+        (3, 6, 3, 2, 40, 12, True, None, 54),
+    ]:
+        rng = np.random.default_rng(seed)
+        q = rng.standard_normal((B, Hq, Nq, d))
+        k = rng.standard_normal((B, Hkv, Nk, d)) * 1.7
+        v = rng.standard_normal((B, Hkv, Nk, d))
+        sln = None if sl is None else np.array(sl, np.int32)
+        o, lse = fwd(q, k, v, causal=causal, scale=0.4, seqlens=sln, causal_bottom_right=True)
+        lens = torch.tensor(sl if sl is not None else [Nk] * B)
+        i = torch.arange(Nq)[None, :, None]
+        j = torch.arange(Nk)[None, None, :]
+        allowed = j < lens[:, None, None]
+        if causal:
+            allowed = allowed & (j <= i + (lens - Nq)[:, None, None])
+        allowed = allowed[:, None]
+        tq, tk, tv = (torch.from_numpy(x) for x in (q, k, v))
+        dead = ~allowed.any(-1)  # rows with no visible key
+        ref = F.scaled_dot_product_attention(tq, tk, tv, attn_mask=allowed, scale=0.4,
+                                             enable_gqa=True)
+        ref = torch.where(dead[..., None], torch.zeros_like(ref), ref)
+        np.testing.assert_allclose(o, ref.numpy(), rtol=0, atol=1e-12)
+        ob, lb = _brute(q, k, v, causal, 0.4, sln, bottom_right=True)
+        np.testing.assert_allclose(o, ob, rtol=0, atol=1e-13)
+        live = np.isfinite(lb)
+        np.testing.assert_allclose(lse[live], lb[live], rtol=0, atol=1e-13)
+        assert np.all(np.isneginf(lse[~live]))
+
+
+def pin_single_query_is_last_causal_row(fwd):
+    """A single query at the end of a sequence (causal, bottom-right) sees
+    every key, so it equals the last row of the square causal forward, and
+    its LSE is the log-sum-exp of that whole row."""
+    B, Hq, Hkv, N, d = 2, 4, 2, 33, 8
+    q, k, v = _rng_inputs(55, B, Hq, Hkv, N, d, 1.3)
+    o_full, l_full = fwd(q, k, v, causal=True, scale=0.3)
+    o1, l1 = fwd(np.ascontiguousarray(q[:, :, -1:]), k, v, causal=True, scale=0.3,
+                 causal_bottom_right=True)
+    np.testing.assert_allclose(o1[:, :, 0], o_full[:, :, -1], rtol=0, atol=1e-13)
+    np.testing.assert_allclose(l1[:, :, 0], l_full[:, :, -1], rtol=0, atol=1e-13)
+    # with key lengths, the query sits at position len_b - 1
+    sl = np.array([33, 12], np.int32)
+    o1, l1 = fwd(np.ascontiguousarray(q[:, :, 11:12]), k, v, causal=True, scale=0.3,
+                 seqlens=np.array([12, 12], np.int32), causal_bottom_right=True)
+    o_s, l_s = fwd(q, k, v, causal=True, scale=0.3, seqlens=sl)
+    np.testing.assert_allclose(o1[1, :, 0], o_s[1, :, 11], rtol=0, atol=1e-13)
+    np.testing.assert_allclose(l1[1, :, 0], l_s[1, :, 11], rtol=0, atol=1e-13)
+
+
 ALL_PINS = [
     pin_golden, pin_probs_are_a_row_softmax, pin_constant_v, pin_single_visible_key,
     pin_causal_first_row, pin_matches_torch_sdpa, pin_brute_force,
     pin_key_permutation_invariance, pin_linear_in_v, pin_shift_invariance,
     pin_fully_masked_row, pin_row_subset, pin_input_encodings_agree,
+    pin_cross_length_matches_torch_sdpa, pin_single_query_is_last_causal_row,
 ]

@@ -17,7 +17,9 @@ SRC = os.path.join(ROOT, "oracle", "attention_ref.c")
 RUNNER = os.path.join(os.path.dirname(os.path.abspath(__file__)), "_mutant_runner.py")
 
 MUTANTS = {
-    "causal_off_by_one": ("(!J->causal || j <= i)", "(!J->causal || j < i)"),
+    "causal_off_by_one": ("(!J->causal || j <= i + off)", "(!J->causal || j < i + off)"),
+    "bottom_right_offset_off_by_one": ("(int64_t)len - J->Nq : 0", "(int64_t)len - J->Nq + 1 : 0"),
+    "bottom_right_ignores_length": ("(int64_t)len - J->Nq : 0", "(int64_t)J->N - J->Nq : 0"),
     "padding_off_by_one": ("(j < len) &&", "(j <= len) &&"),
     "scale_dropped": ("Srow[j] = J->scale * acc;", "Srow[j] = acc;"),
     "gqa_interleaved": ("const int g = h / (J->Hq / J->Hkv);", "const int g = h % J->Hkv;"),
@@ -29,7 +31,8 @@ MUTANTS = {
     "lse_drops_max": ("= m + log(denom);", "= log(denom);"),
     "lse_log2": ("= m + log(denom);", "= m + log2(denom);"),
     "o_overwritten_not_accumulated": ("orow[c] += p *", "orow[c] = p *"),
-    "head_batch_swapped": ("((int64_t)b * J->Hq + h) * N * d", "((int64_t)h * J->B + b) * N * d"),
+    "head_batch_swapped": ("((int64_t)b * J->Hq + h) * J->Nq * d",
+                           "((int64_t)h * J->B + b) * J->Nq * d"),
     "kv_head_dropped": ("((int64_t)b * J->Hkv + g) * N * d", "((int64_t)b * J->Hkv) * N * d"),
     "seqlen_of_batch_0": ("J->seqlens ? J->seqlens[b] : N", "J->seqlens ? J->seqlens[0] : N"),
     "masked_row_not_zeroed": ("for (int j = 0; j < N; ++j) Srow[j] = 0.0;",
