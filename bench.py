@@ -361,6 +361,49 @@ def report_all_workloads(args):
                           "flops": f, "algorithmic_bytes": algo_bytes,
                           "l2": "flushed between steps" if in_bytes < L2_BYTES else "inputs > L2",
                           "peak_source": src}), flush=True)
+    report_decode(args, dev)
+
+
+def report_decode(args, dev):
+    """The split-KV decode path: HBM bandwidth against the measured copy rate."""
+    import torch
+    from exact_io_aware_92_b200 import attention
+    peaks, src = load_peaks()
+    w = wl.DECODE
+    inp = wl.draw_workload(w)
+    q, k, v = (torch.from_numpy(x).view(torch.bfloat16).to(dev)
+               for x in (inp.q_bits, inp.k_bits, inp.v_bits))
+    sl = torch.from_numpy(inp.seqlens).to(dev)
+    o = torch.empty_like(q)
+    lse = torch.empty((w.B, w.Hq, w.nq), dtype=torch.float32, device=dev)
+    ws = torch.empty(attention.decode_workspace_size(w.B, w.Hq, w.Hkv, w.nq, w.N, w.d),
+                     dtype=torch.uint8, device=dev)
+    flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
+    for _ in range(args.warmup):
+        attention.fwd_decode(q, k, v, causal=w.causal, scale=w.scale, seqlens=sl, workspace=ws,
+                             out=o, lse=lse)
+    torch.cuda.synchronize(dev)
+    times = []
+    for _ in range(args.steps):
+        flush.zero_()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        attention.fwd_decode(q, k, v, causal=w.causal, scale=w.scale, seqlens=sl, workspace=ws,
+                             out=o, lse=lse)
+        e1.record()
+        e1.synchronize()
+        times.append(e0.elapsed_time(e1))
+    ms = statistics.median(times)
+    # algorithmic bytes: the valid cache rows of K and V, Q, O and LSE
+    kv = 2 * int(np.sum(inp.seqlens)) * w.Hkv * w.d * 2
+    qo = 2 * q.numel() * 2 + lse.numel() * 4
+    gbs = (kv + qo) / ms / 1e6
+    flops = 4.0 * w.Hq * w.nq * w.d * float(np.sum(inp.seqlens))
+    print(json.dumps({"workload": w.name, "ms_median": ms, "hbm_gbs": gbs,
+                      "frac_of_hbm_peak": gbs / float(peaks["hbm_gbs"]),
+                      "algorithmic_bytes": kv + qo, "tflops": flops / ms / 1e9,
+                      "launches_per_call": 2, "l2": "flushed between steps",
+                      "peak_source": src}), flush=True)
 
 
 def main():

@@ -22,6 +22,7 @@ FA_ERR_LAUNCH = -7
 FA_ERR_TIMEOUT = -8
 FA_ERR_DTYPE = -9
 FA_ERR_CUDA = -10
+FA_ERR_WORKSPACE = -11
 FA_DTYPE_BF16 = 0
 FA_DTYPE_F32 = 1
 
@@ -35,6 +36,9 @@ SIGNATURES = {
     "fa_fwd_f32": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _I, _P]),
     "fa_fwd_hostio": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P,
                            _I, _I, _I, _I, _I, _F, _I, _P]),
+    "fa_decode_workspace_size": (ctypes.c_size_t, [_I, _I, _I, _I, _I, _I, _I]),
+    "fa_fwd_decode": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _I, _P, _I, _P,
+                           ctypes.c_size_t, _P, _P]),
     "fa_check_status": (_I, [_P, _P]),
     "fa_selftest_bounded_wait": (_I, [_P, ctypes.c_ulonglong, _P]),
     "fa_status_string": (ctypes.c_char_p, [_I]),

@@ -61,6 +61,52 @@ def fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *, causal: bool = Fal
     return out, lse
 
 
+def decode_workspace_size(B: int, Hq: int, Hkv: int, Nq: int, Nk: int, d: int,
+                          num_splits: int = 0) -> int:
+    """Bytes of device workspace fwd_decode needs for this shape."""
+    return int(_lib.load().fa_decode_workspace_size(B, Hq, Hkv, Nq, Nk, d, num_splits))
+
+
+def fwd_decode(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *, causal: bool = False,
+               scale: float | None = None, seqlens: torch.Tensor | None = None,
+               num_splits: int = 0, workspace: torch.Tensor | None = None,
+               out: torch.Tensor | None = None, lse: torch.Tensor | None = None,
+               status: torch.Tensor | None = None):
+    """Split-KV decode forward.  q: [B, Hq, Nq, d], k, v: [B, Hkv, Nk, d]
+    (the cache), bf16, contiguous, one CUDA device.  seqlens: int32 [B]
+    valid cache lengths or None.  Causal queries sit at the end of their
+    sequence.  workspace: a byte tensor of at least decode_workspace_size()
+    bytes (allocated here when None).  Returns (o, lse)."""
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        if not t.is_cuda or t.dtype != torch.bfloat16 or t.dim() != 4 or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous bf16 [B, H, N, d] CUDA tensor")
+    B, Hq, Nq, d = q.shape
+    Bk, Hkv, Nk, dk = k.shape
+    if (Bk, dk) != (B, d) or v.shape != k.shape:
+        raise ValueError("k and v must be [B, Hkv, Nk, d] matching q")
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, Hq, Nq), dtype=torch.float32, device=q.device)
+    need = decode_workspace_size(B, Hq, Hkv, Nq, Nk, d, num_splits)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    sl_ptr = None
+    if seqlens is not None:
+        if seqlens.dtype != torch.int32 or seqlens.device != q.device or seqlens.numel() != B:
+            raise ValueError("seqlens must be int32 [B] on q's device")
+        sl_ptr = seqlens.data_ptr()
+    rc = _lib.load().fa_fwd_decode(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                                   lse.data_ptr(), B, Hq, Hkv, Nq, Nk, d, scale,
+                                   int(bool(causal)), sl_ptr, int(num_splits),
+                                   workspace.data_ptr(), workspace.numel() * workspace.element_size(),
+                                   _stream_handle(q.device),
+                                   None if status is None else status.data_ptr())
+    _lib.check(rc, "fa_fwd_decode")
+    return out, lse
+
+
 def check_status(status: torch.Tensor | None = None, device: torch.device | None = None) -> int:
     """Synchronise the current stream and return the status word (0 = ok)."""
     dev = status.device if status is not None else (device or torch.device("cuda"))

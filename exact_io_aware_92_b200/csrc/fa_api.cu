@@ -6,6 +6,7 @@
 // arithmetic runs in the kernels of fa_fwd_sm100.cuh and fa_fwd_f32.cuh.
 #include <cmath>
 #include <cstdint>
+#include <algorithm>
 #include <cstring>
 #include <mutex>
 
@@ -13,6 +14,7 @@
 #include <cuda_runtime.h>
 
 #include "fa.h"
+#include "fa_decode.cuh"
 #include "fa_fwd_f32.cuh"
 #include "fa_fwd_sm100.cuh"
 
@@ -31,6 +33,7 @@ struct DeviceState {
   int num_sms = 0;
   int *status_word = nullptr;  // device address of g_status_word
   bool attr64 = false, attr128 = false;
+  bool dec_attr64 = false, dec_attr128 = false;
 };
 DeviceState g_dev[kMaxDevices];
 std::mutex g_mu;
@@ -186,6 +189,101 @@ int launch_f32(const float *q, const float *k, const float *v, float *o, float *
   return FA_OK;
 }
 
+// Decode: how many key ranges, and how many keys each (a multiple of the
+// kernel's chunk).  The automatic choice aims at about 16 CTAs per SM of a
+// B200 (148 SMs, two resident at a time), so the last wave is a small part of
+// the work, with at least 256 keys per range.
+struct DecodeSplit {
+  int splits, keys_per_split;
+};
+DecodeSplit decode_split(int B, int Hkv, int groups, int Nk, int d, int requested) {
+  const int chunk = 16384 / (d * 2);
+  const long long ctas_per_split = static_cast<long long>(B) * Hkv * groups;
+  int s = requested > 0 ? requested
+                        : static_cast<int>((16 * 148 + ctas_per_split - 1) / ctas_per_split);
+  const int by_len = (Nk + 255) / 256;
+  s = std::max(1, std::min(s, std::min(128, std::max(1, by_len))));
+  int kps = (Nk + s - 1) / s;
+  kps = (kps + chunk - 1) / chunk * chunk;
+  DecodeSplit r;
+  r.keys_per_split = kps;
+  r.splits = (Nk + kps - 1) / kps;
+  return r;
+}
+
+size_t decode_workspace_bytes(int B, int Hq, int Nq, int d, int splits) {
+  const size_t rows = static_cast<size_t>(B) * Hq * Nq;
+  const size_t o_bytes = static_cast<size_t>(splits) * rows * d * sizeof(float);
+  const size_t ml_bytes = static_cast<size_t>(splits) * rows * 2 * sizeof(float);
+  return ((o_bytes + 255) / 256) * 256 + ml_bytes;
+}
+
+int check_decode_args(const void *q, const void *k, const void *v, const void *o,
+                      const float *lse, int B, int Hq, int Hkv, int Nq, int Nk, int d,
+                      float scale) {
+  if (!q || !k || !v || !o || !lse) return FA_ERR_NULL;
+  if (B <= 0 || Hq <= 0 || Hkv <= 0 || Nq <= 0 || Nk <= 0 || d <= 0) return FA_ERR_SHAPE;
+  if (!(std::isfinite(scale) && scale > 0.f)) return FA_ERR_SHAPE;
+  if (Hq % Hkv != 0) return FA_ERR_HEADS;
+  if (d != 64 && d != 128) return FA_ERR_HEADDIM;
+  const long long groups = (static_cast<long long>(Hq / Hkv) * Nq + 3) / 4;
+  if (static_cast<long long>(B) * Hkv > 65535 || groups > 65535) return FA_ERR_SHAPE;
+  if (static_cast<long long>(B) * Hq * Nq > (1ll << 30)) return FA_ERR_SHAPE;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return FA_ERR_ALIGN;
+  if ((reinterpret_cast<uintptr_t>(lse) & 3u) != 0) return FA_ERR_ALIGN;
+  return FA_OK;
+}
+
+template <int D>
+int launch_decode(DeviceState *ds, const void *q, const void *k, const void *v, void *o,
+                  float *lse, int B, int Hq, int Hkv, int Nq, int Nk, float scale, int causal,
+                  const int *seqlens, const DecodeSplit &sp, void *workspace,
+                  cudaStream_t stream, int *status) {
+  using C = fa::DecodeCfg<D>;
+  auto kernel = fa::fa_decode_split_kernel<D>;
+  bool &attr = (D == 64) ? ds->dec_attr64 : ds->dec_attr128;
+  if (!attr) {
+    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM) !=
+        cudaSuccess) {
+      cudaGetLastError();
+      return FA_ERR_LAUNCH;
+    }
+    attr = true;
+  }
+  const size_t rows = static_cast<size_t>(B) * Hq * Nq;
+  fa::DecodeParams p;
+  p.q = static_cast<const uint16_t *>(q);
+  p.k = static_cast<const uint16_t *>(k);
+  p.v = static_cast<const uint16_t *>(v);
+  p.o = static_cast<uint16_t *>(o);
+  p.lse = lse;
+  p.seqlens = seqlens;
+  p.part_o = static_cast<float *>(workspace);
+  p.part_ml = reinterpret_cast<float *>(
+      static_cast<char *>(workspace) +
+      ((static_cast<size_t>(sp.splits) * rows * D * sizeof(float) + 255) / 256) * 256);
+  p.status = status;
+  p.B = B;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.Nq = Nq;
+  p.Nk = Nk;
+  p.group = Hq / Hkv;
+  p.splits = sp.splits;
+  p.keys_per_split = sp.keys_per_split;
+  p.causal = causal ? 1 : 0;
+  p.scale_log2 = scale * kLog2e;
+  p.wait_limit_ns = kWaitLimitNs;
+  const int groups = (p.group * Nq + C::ROWS - 1) / C::ROWS;
+  dim3 grid(sp.splits, B * Hkv, groups);
+  kernel<<<grid, C::THREADS, C::SMEM, stream>>>(p);
+  if (cudaGetLastError() != cudaSuccess) return FA_ERR_LAUNCH;
+  const unsigned cblocks = static_cast<unsigned>((rows + 3) / 4);
+  fa::fa_decode_combine_kernel<D><<<cblocks, 128, 0, stream>>>(p);
+  if (cudaGetLastError() != cudaSuccess) return FA_ERR_LAUNCH;
+  return FA_OK;
+}
+
 // Waits on a barrier that nothing arrives at; the bounded wait must give up.
 __global__ void bounded_wait_selftest_kernel(int *status, unsigned long long limit_ns) {
   __shared__ __align__(8) uint64_t bar;
@@ -217,6 +315,7 @@ const char *fa_status_string(int status) {
     case FA_ERR_TIMEOUT: return "a bounded in-kernel wait ran out";
     case FA_ERR_DTYPE: return "unknown dtype code";
     case FA_ERR_CUDA: return "CUDA runtime error";
+    case FA_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
     default: return "unknown status";
   }
 }
@@ -315,6 +414,38 @@ int fa_fwd_hostio(const void *q_h, const void *k_h, const void *v_h, void *o_h, 
     return FA_ERR_CUDA;
   }
   return fa_check_status(nullptr, stream);
+}
+
+size_t fa_decode_workspace_size(int B, int Hq, int Hkv, int Nq, int Nk, int d, int num_splits) {
+  if (B <= 0 || Hq <= 0 || Hkv <= 0 || Nq <= 0 || Nk <= 0 || (d != 64 && d != 128) ||
+      Hq % Hkv != 0 || num_splits < 0)
+    return 0;
+  const int groups = ((Hq / Hkv) * Nq + 3) / 4;
+  const DecodeSplit sp = decode_split(B, Hkv, groups, Nk, d, num_splits);
+  return decode_workspace_bytes(B, Hq, Nq, d, sp.splits);
+}
+
+int fa_fwd_decode(const void *q, const void *k, const void *v, void *o, float *lse, int B,
+                  int Hq, int Hkv, int Nq, int Nk, int d, float scale, int causal,
+                  const int *seqlens_k, int num_splits, void *workspace, size_t workspace_bytes,
+                  void *stream, int *status_dev) {
+  int rc = check_decode_args(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, scale);
+  if (rc != FA_OK) return rc;
+  if (num_splits < 0 || num_splits > 128) return FA_ERR_SHAPE;
+  const int groups = ((Hq / Hkv) * Nq + 3) / 4;
+  const DecodeSplit sp = decode_split(B, Hkv, groups, Nk, d, num_splits);
+  if (!workspace || !aligned16(workspace) ||
+      workspace_bytes < decode_workspace_bytes(B, Hq, Nq, d, sp.splits))
+    return FA_ERR_WORKSPACE;
+  DeviceState *ds = nullptr;
+  rc = current_device(&ds);
+  if (rc != FA_OK) return rc;
+  int *status = status_dev ? status_dev : ds->status_word;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  return d == 64 ? launch_decode<64>(ds, q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, scale, causal,
+                                     seqlens_k, sp, workspace, st, status)
+                 : launch_decode<128>(ds, q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, scale, causal,
+                                      seqlens_k, sp, workspace, st, status);
 }
 
 int fa_selftest_bounded_wait(int *status_dev, unsigned long long limit_ns, void *stream) {

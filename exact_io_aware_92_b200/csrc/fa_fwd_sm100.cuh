@@ -52,9 +52,6 @@ struct FwdParams {
   unsigned long long wait_limit_ns;
 };
 
-// Status codes written by the kernel (negative, matching fa_status).
-constexpr int kErrTimeout = -8;
-
 template <int D>
 struct Sm100Cfg {
   static_assert(D == 64 || D == 128, "head dim 64 or 128");

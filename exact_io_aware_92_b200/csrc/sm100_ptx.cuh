@@ -9,6 +9,9 @@
 
 namespace fa {
 
+// Status code the kernels write when a bounded wait runs out (FA_ERR_TIMEOUT).
+constexpr int kErrTimeout = -8;
+
 // ---------------------------------------------------------------------------
 // Shared-memory addresses and barriers
 // ---------------------------------------------------------------------------

@@ -38,6 +38,7 @@ class Workload:
     k_scale: float = 1.0
     seqlen_range: tuple[int, int] | None = None  # inclusive [lo, hi] key lengths
     sample_rows: int | None = None  # oracle rows per head for large cases
+    nq: int | None = None  # query rows for the decode shape (keys: N); None = N
 
     @property
     def scale(self) -> float:
@@ -56,8 +57,13 @@ LLAMA_GQA = Workload("llama_gqa_causal_b2_hq32_hkv8_n8192_d128", 2, 32, 8, 8192,
 LONG = Workload("long_causal_b1_h16_n32768_d128", 1, 16, 16, 32768, 128, True, seed=5,
                 sample_rows=256)
 
+# Decode against a KV cache (SURVEY "next" row): one new token per sequence,
+# the Llama-style GQA heads, caches of 16K-32K tokens.
+DECODE = Workload("llama_gqa_decode_b8_hq32_hkv8_nq1_nk32768_d128", 8, 32, 8, 32768, 128, True,
+                  seed=6, seqlen_range=(16384, 32768), nq=1)
+
 ALL = (TINY, GPT2, BERT, LLAMA_GQA, LONG)
-BY_NAME = {w.name: w for w in ALL}
+BY_NAME = {w.name: w for w in ALL + (DECODE,)}
 
 
 def round_to_bf16_bits(x: np.ndarray) -> np.ndarray:
@@ -115,9 +121,10 @@ class Inputs:
 
 
 def draw(B: int, Hq: int, Hkv: int, N: int, d: int, seed: int, *, k_scale: float = 1.0,
-         seqlen_range: tuple[int, int] | None = None) -> Inputs:
+         seqlen_range: tuple[int, int] | None = None, nq: int | None = None) -> Inputs:
+    """Q has nq rows (default N: self-attention); K and V have N rows."""
     rng = np.random.default_rng(seed)
-    q = rng.standard_normal((B, Hq, N, d), dtype=np.float32)
+    q = rng.standard_normal((B, Hq, N if nq is None else nq, d), dtype=np.float32)
     k = rng.standard_normal((B, Hkv, N, d), dtype=np.float32)
     v = rng.standard_normal((B, Hkv, N, d), dtype=np.float32)
     if k_scale != 1.0:
@@ -131,7 +138,7 @@ def draw(B: int, Hq: int, Hkv: int, N: int, d: int, seed: int, *, k_scale: float
 
 def draw_workload(w: Workload) -> Inputs:
     return draw(w.B, w.Hq, w.Hkv, w.N, w.d, w.seed, k_scale=w.k_scale,
-                seqlen_range=w.seqlen_range)
+                seqlen_range=w.seqlen_range, nq=w.nq)
 
 
 def sample_rows(w: Workload, rows_per_head: int | None = None) -> np.ndarray:

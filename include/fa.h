@@ -48,6 +48,8 @@
 #ifndef FA_B200_FA_H
 #define FA_B200_FA_H
 
+#include <stddef.h>
+
 #if defined(__GNUC__)
 #define FA_API __attribute__((visibility("default")))
 #else
@@ -69,7 +71,8 @@ typedef enum {
   FA_ERR_LAUNCH = -7,    /* the CUDA launch itself failed */
   FA_ERR_TIMEOUT = -8,   /* a bounded in-kernel wait ran out (reported by fa_check_status) */
   FA_ERR_DTYPE = -9,     /* unknown dtype code */
-  FA_ERR_CUDA = -10      /* another CUDA runtime error (copy, query, driver entry point) */
+  FA_ERR_CUDA = -10,     /* another CUDA runtime error (copy, query, driver entry point) */
+  FA_ERR_WORKSPACE = -11 /* workspace missing, misaligned or smaller than required */
 } fa_status;
 
 /* dtype codes for fa_fwd_ex */
@@ -125,6 +128,38 @@ FA_API int fa_fwd_hostio(const void *q_h, const void *k_h, const void *v_h, void
                   const int *seqlens_h, void *q_d, void *k_d, void *v_d, void *o_d, float *lse_d,
                   int *seqlens_d, int B, int Hq, int Hkv, int N, int d, float scale, int causal,
                   void *stream);
+
+/*
+ * Split-KV decode forward: Nq query rows per (batch, query head) against Nk
+ * cached keys.  Same operation as fa_fwd with two differences of shape:
+ *  q, o : [B, Hq, Nq, d] bf16      k, v : [B, Hkv, Nk, d] bf16 (the cache)
+ *  lse  : [B, Hq, Nq] fp32
+ *  seqlens_k: NULL or device int32[B], 0 <= seqlens_k[b] <= Nk, the number of
+ *         valid cached keys of sequence b (keys past it are ignored).
+ *  causal: 0/1; query i is position len_b - Nq + i of its sequence, so it sees
+ *         keys j <= len_b - Nq + i (with Nq = 1: every valid key).
+ *  num_splits: key ranges processed in parallel per (batch, kv head), 1..128,
+ *         or 0 for an automatic choice (about 16 CTAs per SM of a B200 in
+ *         all, at least 256 keys per range).
+ *  workspace: DEVICE buffer of at least fa_decode_workspace_size() bytes,
+ *         16-byte aligned, owned by the caller; it holds each key range's
+ *         partial output, row max and row sum, merged by a second kernel
+ *         through their log-sum-exp.  It may be reused across calls that are
+ *         ordered on one stream.
+ * Reference: wiki note "FlashAttention", common misconceptions: generating a
+ * single token is bound by reading the cached K/V, and needs decode-oriented
+ * kernels; the merge is the same online-softmax update (section "what it
+ * is") applied to whole key ranges.
+ * Returns FA_OK when both kernels are launched on `stream`, FA_ERR_WORKSPACE
+ * when the workspace is missing, misaligned or too small, or another
+ * fa_status.  d must be 64 or 128.
+ */
+FA_API size_t fa_decode_workspace_size(int B, int Hq, int Hkv, int Nq, int Nk, int d,
+                                       int num_splits);
+FA_API int fa_fwd_decode(const void *q, const void *k, const void *v, void *o, float *lse, int B,
+                         int Hq, int Hkv, int Nq, int Nk, int d, float scale, int causal,
+                         const int *seqlens_k, int num_splits, void *workspace,
+                         size_t workspace_bytes, void *stream, int *status_dev);
 
 /*
  * Waits for `stream` and reads a status word (status_dev, or the library's

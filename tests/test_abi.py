@@ -77,6 +77,23 @@ def test_hostio_requires_device_seqlens_with_host_seqlens(lib):
     assert rc == _lib.FA_ERR_NULL
 
 
+def test_decode_workspace_size_and_errors(lib):
+    n = lib.fa_decode_workspace_size(8, 32, 8, 1, 32768, 128, 0)
+    assert n > 0 and n % 4 == 0
+    assert lib.fa_decode_workspace_size(8, 32, 8, 1, 32768, 96, 0) == 0  # bad head dim
+    assert lib.fa_decode_workspace_size(8, 30, 8, 1, 32768, 128, 0) == 0  # Hq % Hkv
+    more = lib.fa_decode_workspace_size(8, 32, 8, 1, 32768, 128, 64)
+    assert more >= lib.fa_decode_workspace_size(8, 32, 8, 1, 32768, 128, 1)
+    args = (A, A, A, A, A, 2, 8, 2, 1, 1000, 128, 0.088, 0)
+    # missing or too-small workspace is reported before anything touches the device
+    assert lib.fa_fwd_decode(*args, None, 0, None, 0, None, None) == _lib.FA_ERR_WORKSPACE
+    assert lib.fa_fwd_decode(*args, None, 0, A, 16, None, None) == _lib.FA_ERR_WORKSPACE
+    assert lib.fa_fwd_decode(*args, None, 0, A + 4, 1 << 30, None, None) == _lib.FA_ERR_WORKSPACE
+    assert lib.fa_fwd_decode(*args, None, 200, A, 1 << 30, None, None) == _lib.FA_ERR_SHAPE
+    assert lib.fa_fwd_decode(A, A, A, A, A, 2, 8, 3, 1, 1000, 128, 0.088, 0, None, 0, A, 1 << 30,
+                             None, None) == _lib.FA_ERR_HEADS
+
+
 def test_without_a_b200_valid_calls_report_arch():
     import torch
     if torch.cuda.is_available():

@@ -1,0 +1,81 @@
+"""Split-KV decode forward (fa_fwd_decode) vs the fp64 oracle with queries at
+the end of their sequences, element by element."""
+import numpy as np
+import pytest
+
+from exact_io_aware_92_b200 import workloads as wl
+from parity_helpers import LSE_TOL_BF16, O_TOL_BF16, compare, to_device_bf16
+
+pytestmark = pytest.mark.gpu
+
+import oracle  # noqa: E402
+
+
+def run_decode(inp, *, causal, scale, num_splits=0):
+    import torch
+    from exact_io_aware_92_b200 import attention
+    q, k, v = (to_device_bf16(x) for x in (inp.q_bits, inp.k_bits, inp.v_bits))
+    sl = None if inp.seqlens is None else torch.from_numpy(inp.seqlens).cuda()
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    o, lse = attention.fwd_decode(q, k, v, causal=causal, scale=scale, seqlens=sl,
+                                  num_splits=num_splits, status=status)
+    assert attention.check_status(status) == 0
+    return o.float().cpu().numpy().astype(np.float64), lse.cpu().numpy().astype(np.float64)
+
+
+def ref_decode(inp, *, causal, scale):
+    return oracle.attention_forward(inp.q_bits, inp.k_bits, inp.v_bits, causal=causal,
+                                    scale=float(np.float32(scale)), seqlens=inp.seqlens,
+                                    causal_bottom_right=True)
+
+
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("Nk", [1, 17, 64, 65, 129, 1000, 4097])
+def test_single_query_lengths(Nk, d):
+    inp = wl.draw(2, 8, 2, Nk, d, seed=600 + Nk, nq=1)
+    o, lse = run_decode(inp, causal=True, scale=1 / np.sqrt(d))
+    o_r, l_r = ref_decode(inp, causal=True, scale=1 / np.sqrt(d))
+    compare(o, lse, o_r, l_r, o_tol=O_TOL_BF16, lse_tol=LSE_TOL_BF16, what=f"Nk{Nk} d{d}")
+
+
+@pytest.mark.parametrize("splits", [1, 3, 7, 0])
+@pytest.mark.parametrize("group,nq", [(1, 1), (4, 1), (8, 1), (4, 3), (1, 5)])
+def test_groups_rows_and_splits(group, nq, splits):
+    inp = wl.draw(3, 8, 8 // group, 2000, 128, seed=700 + group * 10 + nq, nq=nq)
+    inp.seqlens = np.array([2000, 1, 777], dtype=np.int32)
+    for causal in (False, True):
+        o, lse = run_decode(inp, causal=causal, scale=0.09, num_splits=splits)
+        o_r, l_r = ref_decode(inp, causal=causal, scale=0.09)
+        compare(o, lse, o_r, l_r, o_tol=O_TOL_BF16, lse_tol=LSE_TOL_BF16,
+                what=f"G{group} nq{nq} splits{splits} causal{causal}")
+
+
+def test_empty_and_short_caches():
+    inp = wl.draw(4, 4, 2, 300, 64, seed=801, nq=2)
+    inp.seqlens = np.array([0, 1, 2, 300], dtype=np.int32)
+    o, lse = run_decode(inp, causal=True, scale=0.125, num_splits=4)
+    o_r, l_r = ref_decode(inp, causal=True, scale=0.125)
+    compare(o, lse, o_r, l_r, o_tol=O_TOL_BF16, lse_tol=LSE_TOL_BF16, what="short caches")
+
+
+def test_decode_workload_every_row():
+    w = wl.DECODE
+    inp = wl.draw_workload(w)
+    o, lse = run_decode(inp, causal=w.causal, scale=w.scale)
+    o_r, l_r = ref_decode(inp, causal=w.causal, scale=w.scale)
+    compare(o, lse, o_r, l_r, o_tol=O_TOL_BF16, lse_tol=LSE_TOL_BF16, what=w.name)
+
+
+def test_decode_matches_last_row_of_full_forward():
+    """A single query at the end of a sequence equals the last causal row of
+    the tensor-core forward over the same keys (two kernels, same answer
+    within rounding)."""
+    import torch
+    from exact_io_aware_92_b200 import attention
+    full = wl.draw(2, 8, 2, 1000, 128, seed=802)
+    q, k, v = (to_device_bf16(x) for x in (full.q_bits, full.k_bits, full.v_bits))
+    o_full, l_full = attention.fwd(q, k, v, causal=True, scale=0.088)
+    o_dec, l_dec = attention.fwd_decode(q[:, :, -1:].contiguous(), k, v, causal=True, scale=0.088)
+    torch.cuda.synchronize()
+    assert torch.allclose(o_dec[:, :, 0].float(), o_full[:, :, -1].float(), atol=2e-2)
+    assert torch.allclose(l_dec[:, :, 0], l_full[:, :, -1], atol=1e-3)
