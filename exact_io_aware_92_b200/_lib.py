@@ -39,6 +39,8 @@ SIGNATURES = {
     "fa_decode_workspace_size": (ctypes.c_size_t, [_I, _I, _I, _I, _I, _I, _I]),
     "fa_fwd_decode": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _I, _P, _I, _P,
                            ctypes.c_size_t, _P, _P]),
+    "fa_fwd_decode_noalloc": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _I, _P, _I,
+                                   _P, _P]),
     "fa_check_status": (_I, [_P, _P]),
     "fa_selftest_bounded_wait": (_I, [_P, ctypes.c_ulonglong, _P]),
     "fa_status_string": (ctypes.c_char_p, [_I]),

@@ -460,3 +460,65 @@ int fa_selftest_bounded_wait(int *status_dev, unsigned long long limit_ns, void 
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Decode for callers that cannot allocate device memory (fa_fwd_decode_noalloc)
+// ---------------------------------------------------------------------------
+// The per-range partials live in one fixed array owned by this library
+// instead of a caller-provided workspace.  Every GPU that loads the library
+// keeps these 8 MiB until the process exits.  In host code the symbol is a
+// host-side stand-in, so its device address is looked up once per device.
+static __device__ __align__(256) float g_decode_noalloc_scratch[(8u << 20) / sizeof(float)];
+
+namespace {
+constexpr size_t kNoAllocScratchBytes = 8u << 20;
+void *g_noalloc_scratch_addr[kMaxDevices];
+std::mutex g_noalloc_mu;
+
+// With `dev` current: the device address of the scratch array, looked up on
+// the first call for that device and remembered.
+int noalloc_scratch(int dev, void **out) {
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (!g_noalloc_scratch_addr[dev]) {
+    void *ptr = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&ptr, g_decode_noalloc_scratch);
+    if (e != cudaSuccess || !ptr) {
+      cudaGetLastError();
+      return FA_ERR_CUDA;
+    }
+    g_noalloc_scratch_addr[dev] = ptr;
+  }
+  *out = g_noalloc_scratch_addr[dev];
+  return FA_OK;
+}
+}  // namespace
+
+extern "C" int fa_fwd_decode_noalloc(const void *q, const void *k, const void *v, void *o,
+                                     float *lse, int B, int Hq, int Hkv, int Nq, int Nk, int d,
+                                     float scale, int causal, const int *seqlens_k,
+                                     int num_splits, void *stream, int *status_dev) {
+  int rc = check_decode_args(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, scale);
+  if (rc != FA_OK) return rc;
+  if (num_splits < 0 || num_splits > 128) return FA_ERR_SHAPE;
+  const int groups = ((Hq / Hkv) * Nq + 3) / 4;
+  const DecodeSplit sp = decode_split(B, Hkv, groups, Nk, d, num_splits);
+  if (decode_workspace_bytes(B, Hq, Nq, d, sp.splits) > kNoAllocScratchBytes)
+    return FA_ERR_WORKSPACE;
+  DeviceState *ds = nullptr;
+  rc = current_device(&ds);
+  if (rc != FA_OK) return rc;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    cudaGetLastError();
+    return FA_ERR_CUDA;
+  }
+  void *scratch = nullptr;
+  rc = noalloc_scratch(dev, &scratch);
+  if (rc != FA_OK) return rc;
+  int *status = status_dev ? status_dev : ds->status_word;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  return d == 64 ? launch_decode<64>(ds, q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, scale, causal,
+                                     seqlens_k, sp, scratch, st, status)
+                 : launch_decode<128>(ds, q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, scale, causal,
+                                      seqlens_k, sp, scratch, st, status);
+}

@@ -162,6 +162,34 @@ FA_API int fa_fwd_decode(const void *q, const void *k, const void *v, void *o, f
                          size_t workspace_bytes, void *stream, int *status_dev);
 
 /*
+ * fa_fwd_decode without a workspace argument, for callers that cannot
+ * allocate device memory on the call path: code that runs where the
+ * allocator must not be touched (an inference loop with a fixed memory
+ * budget, a host framework that owns every device allocation, or a latency
+ * path where cudaMalloc's implicit device synchronisation is not acceptable).
+ * The pages have no counterpart to this call; it only changes where the
+ * decode partials are kept.
+ *
+ * Same arguments and results as fa_fwd_decode, minus workspace and
+ * workspace_bytes.  The partials go to one 8 MiB array that the library
+ * defines in device memory; every GPU that loads the library holds it until
+ * the process exits.  A shape whose partials need more than 8 MiB
+ * (fa_decode_workspace_size() > 8388608) is rejected with FA_ERR_WORKSPACE;
+ * nothing is launched then.  No call allocates or frees device memory.
+ *
+ * The first call on a device looks up the array's device address (with that
+ * device current) and remembers it; make that first call before any stream
+ * capture.  The array keeps the last call's contents: every call writes all
+ * the partials it reads, so nothing needs clearing, but all calls share the
+ * one array, so calls that overlap on the GPU (on different streams, or from
+ * several host threads) race; order them on one stream.
+ */
+FA_API int fa_fwd_decode_noalloc(const void *q, const void *k, const void *v, void *o,
+                                 float *lse, int B, int Hq, int Hkv, int Nq, int Nk, int d,
+                                 float scale, int causal, const int *seqlens_k, int num_splits,
+                                 void *stream, int *status_dev);
+
+/*
  * Waits for `stream` and reads a status word (status_dev, or the library's
  * own when NULL).  Returns FA_OK, FA_ERR_TIMEOUT, or FA_ERR_CUDA when the
  * stream reports an error.  Resets the library's own word to FA_OK.
