@@ -361,7 +361,45 @@ def report_all_workloads(args):
                           "flops": f, "algorithmic_bytes": algo_bytes,
                           "l2": "flushed between steps" if in_bytes < L2_BYTES else "inputs > L2",
                           "peak_source": src}), flush=True)
+    report_varlen(args, dev)
     report_decode(args, dev)
+
+
+def report_varlen(args, dev):
+    """The BERT-shaped workload in the packed layout (no padded rows)."""
+    import torch
+    from exact_io_aware_92_b200 import attention
+    peaks, src = load_peaks()
+    w = wl.BERT
+    inp = wl.draw_workload(w)
+    lengths = [int(x) for x in inp.seqlens]
+    q, k, v = (torch.from_numpy(wl.pack(x, lengths)).view(torch.bfloat16).to(dev)
+               for x in (inp.q_bits, inp.k_bits, inp.v_bits))
+    cu = torch.from_numpy(wl.cu_seqlens(lengths)).to(dev)
+    o = torch.empty_like(q)
+    lse = torch.empty((w.Hq, q.shape[0]), dtype=torch.float32, device=dev)
+    flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
+    for _ in range(args.warmup):
+        attention.fwd_varlen(q, k, v, cu, max(lengths), causal=False, scale=w.scale, out=o,
+                             lse=lse)
+    torch.cuda.synchronize(dev)
+    times = []
+    for _ in range(args.steps):
+        flush.zero_()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        attention.fwd_varlen(q, k, v, cu, max(lengths), causal=False, scale=w.scale, out=o,
+                             lse=lse)
+        e1.record()
+        e1.synchronize()
+        times.append(e0.elapsed_time(e1))
+    ms = statistics.median(times)
+    useful = 4.0 * w.Hq * w.d * float(sum(L * L for L in lengths))
+    print(json.dumps({"workload": w.name + "@packed", "ms_median": ms,
+                      "tflops_useful": useful / ms / 1e9,
+                      "frac_of_peak": useful / ms / 1e9 / float(peaks["bf16_tflops"]),
+                      "flops_useful": useful, "l2": "flushed between steps",
+                      "peak_source": src}), flush=True)
 
 
 def report_decode(args, dev):

@@ -7,12 +7,12 @@ inputs (``workloads``).
 """
 from . import workloads  # noqa: F401
 
-__all__ = ["fwd", "fwd_decode", "decode_workspace_size", "check_status", "fwd_hostio",
+__all__ = ["fwd", "fwd_varlen", "fwd_decode", "decode_workspace_size", "check_status", "fwd_hostio",
            "workloads"]
 
 
 def __getattr__(name):
-    if name in ("fwd", "fwd_decode", "decode_workspace_size", "check_status", "fwd_hostio"):
+    if name in ("fwd", "fwd_varlen", "fwd_decode", "decode_workspace_size", "check_status", "fwd_hostio"):
         from . import attention
         return getattr(attention, name)
     raise AttributeError(name)

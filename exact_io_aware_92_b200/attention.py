@@ -61,6 +61,37 @@ def fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *, causal: bool = Fal
     return out, lse
 
 
+def fwd_varlen(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, cu_seqlens: torch.Tensor,
+               max_seqlen: int, *, causal: bool = False, scale: float | None = None,
+               out: torch.Tensor | None = None, lse: torch.Tensor | None = None,
+               status: torch.Tensor | None = None):
+    """Packed variable-length forward.  q: [total, Hq, d], k, v: [total, Hkv, d]
+    bf16 contiguous; cu_seqlens: int32 [B+1] token offsets on the device;
+    max_seqlen >= every sequence length.  Returns (o [total, Hq, d],
+    lse [Hq, total])."""
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        if not t.is_cuda or t.dtype != torch.bfloat16 or t.dim() != 3 or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous bf16 [total, H, d] CUDA tensor")
+    total, Hq, d = q.shape
+    if k.shape != v.shape or k.shape[0] != total or k.shape[2] != d:
+        raise ValueError("k and v must be [total, Hkv, d] matching q")
+    if cu_seqlens.dtype != torch.int32 or cu_seqlens.device != q.device or cu_seqlens.dim() != 1:
+        raise ValueError("cu_seqlens must be int32 [B+1] on q's device")
+    B = cu_seqlens.numel() - 1
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((Hq, total), dtype=torch.float32, device=q.device)
+    rc = _lib.load().fa_fwd_varlen(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                                   lse.data_ptr(), cu_seqlens.data_ptr(), B, Hq, k.shape[1],
+                                   total, int(max_seqlen), d, scale, int(bool(causal)),
+                                   _stream_handle(q.device),
+                                   None if status is None else status.data_ptr())
+    _lib.check(rc, "fa_fwd_varlen")
+    return out, lse
+
+
 def decode_workspace_size(B: int, Hq: int, Hkv: int, Nq: int, Nk: int, d: int,
                           num_splits: int = 0) -> int:
     """Bytes of device workspace fwd_decode needs for this shape."""

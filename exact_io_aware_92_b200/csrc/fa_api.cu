@@ -119,10 +119,28 @@ int make_map(CUtensorMap *m, const void *ptr, int planes, int N, int d) {
   return r == CUDA_SUCCESS ? FA_OK : FA_ERR_CUDA;
 }
 
+// Packed layout: a [total, H, d] tensor seen as (d, head, token), box of 64
+// columns x 1 head x 128 tokens, 128-byte swizzle; tokens past the end read
+// as zero.
+int make_map_packed(CUtensorMap *m, const void *ptr, int total, int H, int d) {
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(H),
+                        static_cast<cuuint64_t>(total)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2,
+                           static_cast<cuuint64_t>(H) * static_cast<cuuint64_t>(d) * 2};
+  cuuint32_t box[3] = {64, 1, 128};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(ptr), dims,
+                        strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? FA_OK : FA_ERR_CUDA;
+}
+
 template <int D>
 int launch_bf16(DeviceState *ds, const void *q, const void *k, const void *v, void *o,
                 float *lse, int B, int Hq, int Hkv, int N, float scale, int causal,
-                const int *seqlens, cudaStream_t stream, int *status) {
+                const int *seqlens, cudaStream_t stream, int *status,
+                const int *cu_seqlens = nullptr, int total = 0) {
   using C = fa::Sm100Cfg<D>;
   auto kernel = fa::fa_fwd_bf16_sm100_kernel<D>;
   bool &attr = (D == 64) ? ds->attr64 : ds->attr128;
@@ -135,13 +153,21 @@ int launch_bf16(DeviceState *ds, const void *q, const void *k, const void *v, vo
     attr = true;
   }
   CUtensorMap tq, tk, tv;
-  if (make_map(&tq, q, B * Hq, N, D) != FA_OK || make_map(&tk, k, B * Hkv, N, D) != FA_OK ||
-      make_map(&tv, v, B * Hkv, N, D) != FA_OK)
+  if (cu_seqlens) {
+    if (make_map_packed(&tq, q, total, Hq, D) != FA_OK ||
+        make_map_packed(&tk, k, total, Hkv, D) != FA_OK ||
+        make_map_packed(&tv, v, total, Hkv, D) != FA_OK)
+      return FA_ERR_CUDA;
+  } else if (make_map(&tq, q, B * Hq, N, D) != FA_OK || make_map(&tk, k, B * Hkv, N, D) != FA_OK ||
+             make_map(&tv, v, B * Hkv, N, D) != FA_OK) {
     return FA_ERR_CUDA;
+  }
   fa::FwdParams p;
   p.o = static_cast<uint16_t *>(o);
   p.lse = lse;
   p.seqlens = seqlens;
+  p.cu_seqlens = cu_seqlens;
+  p.total = total;
   p.status = status;
   p.B = B;
   p.Hq = Hq;
@@ -414,6 +440,24 @@ int fa_fwd_hostio(const void *q_h, const void *k_h, const void *v_h, void *o_h, 
     return FA_ERR_CUDA;
   }
   return fa_check_status(nullptr, stream);
+}
+
+int fa_fwd_varlen(const void *q, const void *k, const void *v, void *o, float *lse,
+                  const int *cu_seqlens, int B, int Hq, int Hkv, int total, int max_seqlen, int d,
+                  float scale, int causal, void *stream, int *status_dev) {
+  if (!cu_seqlens) return FA_ERR_NULL;
+  int rc = check_args(q, k, v, o, lse, B, Hq, Hkv, max_seqlen, d, scale);
+  if (rc != FA_OK) return rc;
+  if (total <= 0 || static_cast<long long>(total) * Hq * d > (1ll << 40)) return FA_ERR_SHAPE;
+  DeviceState *ds = nullptr;
+  rc = current_device(&ds);
+  if (rc != FA_OK) return rc;
+  int *status = status_dev ? status_dev : ds->status_word;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  return d == 64 ? launch_bf16<64>(ds, q, k, v, o, lse, B, Hq, Hkv, max_seqlen, scale, causal,
+                                   nullptr, st, status, cu_seqlens, total)
+                 : launch_bf16<128>(ds, q, k, v, o, lse, B, Hq, Hkv, max_seqlen, scale, causal,
+                                    nullptr, st, status, cu_seqlens, total);
 }
 
 size_t fa_decode_workspace_size(int B, int Hq, int Hkv, int Nq, int Nk, int d, int num_splits) {

@@ -40,9 +40,11 @@
 namespace fa {
 
 struct FwdParams {
-  uint16_t *o;           // bf16 [B, Hq, N, d]
-  float *lse;            // fp32 [B, Hq, N]
-  const int *seqlens;    // int32 [B] or nullptr
+  uint16_t *o;           // bf16 [B, Hq, N, d], or [total, Hq, d] when packed
+  float *lse;            // fp32 [B, Hq, N], or [Hq, total] when packed
+  const int *seqlens;    // int32 [B] key lengths or nullptr
+  const int *cu_seqlens; // packed layout: int32 [B+1] token offsets, else nullptr
+  int total;             // packed layout: tokens in all sequences
   int *status;           // device status word (time-outs)
   int B, Hq, Hkv, N, group;
   int num_qpairs;        // ceil(N / 256)
@@ -96,9 +98,18 @@ struct Sm100Cfg {
 #endif
 };
 
-// One work unit, as every role sees it.
+// One work unit, as every role sees it.  Rows and keys are counted from the
+// start of the unit's sequence; tok0 is where that sequence starts in the
+// packed layout (0 otherwise).
 struct Unit {
   int b, h, hkv, bh, row0, L, nkv;
+  int q_rows;      // query rows that exist (N, or the sequence length when packed)
+  int tok0;        // first token of the sequence (packed layout)
+  int q_plane;     // TMA plane of Q: b*Hq+h, or h when packed
+  int kv_plane;    // TMA plane of K/V: b*Hkv+hkv, or hkv when packed
+  size_t o_base;   // element offset of row 0 of this (sequence, head) in O
+  size_t o_stride; // elements between consecutive rows of O
+  size_t lse_base; // offset of row 0 in LSE
 };
 
 template <int D>
@@ -113,10 +124,29 @@ __device__ __forceinline__ Unit unit_at(const FwdParams &p, int u) {
   x.hkv = x.h / p.group;
   x.row0 = qp * C::ROWS_PER_UNIT;
   int L = p.N;
-  if (p.seqlens) L = min(max(p.seqlens[x.b], 0), p.N);
+  if (p.cu_seqlens) {
+    x.tok0 = p.cu_seqlens[x.b];
+    L = max(p.cu_seqlens[x.b + 1] - x.tok0, 0);
+    x.q_rows = L;
+    x.q_plane = x.h;
+    x.kv_plane = x.hkv;
+    x.o_base = (static_cast<size_t>(x.tok0) * p.Hq + x.h) * D;
+    x.o_stride = static_cast<size_t>(p.Hq) * D;
+    x.lse_base = static_cast<size_t>(x.h) * p.total + x.tok0;
+  } else {
+    if (p.seqlens) L = min(max(p.seqlens[x.b], 0), p.N);
+    x.tok0 = 0;
+    x.q_rows = p.N;
+    x.q_plane = x.bh;
+    x.kv_plane = x.b * p.Hkv + x.hkv;
+    x.o_base = static_cast<size_t>(x.bh) * p.N * D;
+    x.o_stride = D;
+    x.lse_base = static_cast<size_t>(x.bh) * p.N;
+  }
   x.L = L;
   const int kv_end = p.causal ? min(L, x.row0 + C::ROWS_PER_UNIT) : L;
-  x.nkv = (kv_end + C::BN - 1) / C::BN;
+  // A unit past the end of its sequence (packed layout) has no rows at all.
+  x.nkv = x.row0 < x.q_rows ? (kv_end + C::BN - 1) / C::BN : 0;
   return x;
 }
 
@@ -160,6 +190,7 @@ __device__ void role_producer(const Sm100Ctx<D> &x, const FwdParams &p, const CU
   using C = Sm100Cfg<D>;
   int seq = 0;  // K/V tiles put into the ring so far (K and V counted apart)
   int qi = 0;   // units with keys loaded so far
+  const bool packed = p.cu_seqlens != nullptr;
   bool ok = true;
   for (int k = 0; ok; ++k) {
     const int u = snake_unit(k, p.num_units);
@@ -176,13 +207,16 @@ __device__ void role_producer(const Sm100Ctx<D> &x, const FwdParams &p, const CU
         break;
       }
       mbar_arrive_expect_tx(x.bar(C::BAR_Q_FULL + t), C::TILE_BYTES);
+      // The padded layout's maps are (d, rows, plane); the packed layout's
+      // are (d, head, token), which keeps their strides increasing.
+      const int qrow = w.tok0 + w.row0 + t * C::BM;
       for (int half = 0; half < D / 64; ++half)
         tma_load_3d(x.q_tile(t) + half * C::HALF_BYTES, tm_q, x.bar(C::BAR_Q_FULL + t), half * 64,
-                    w.row0 + t * C::BM, w.bh);
+                    packed ? w.q_plane : qrow, packed ? qrow : w.q_plane);
     }
     if (!ok) break;
     ++qi;
-    const int kv_plane = w.b * p.Hkv + w.hkv;
+    const int kv_plane = w.kv_plane;
     for (int j = 0; j < w.nkv && ok; ++j) {
       for (int kv = 0; kv < 2; ++kv, ++seq) {
         const int slot = ring_slot<D>(seq);
@@ -194,9 +228,10 @@ __device__ void role_producer(const Sm100Ctx<D> &x, const FwdParams &p, const CU
         const uint32_t full = x.bar(C::BAR_KV_FULL + slot);
         mbar_arrive_expect_tx(full, C::TILE_BYTES);
         const CUtensorMap *m = kv ? tm_v : tm_k;
+        const int krow = w.tok0 + j * C::BN;
         for (int half = 0; half < D / 64; ++half)
-          tma_load_3d(x.kv_tile(slot) + half * C::HALF_BYTES, m, full, half * 64, j * C::BN,
-                      kv_plane);
+          tma_load_3d(x.kv_tile(slot) + half * C::HALF_BYTES, m, full, half * 64,
+                      packed ? kv_plane : krow, packed ? krow : kv_plane);
       }
     }
   }
@@ -384,14 +419,14 @@ __device__ void role_softmax(const Sm100Ctx<D> &x, const FwdParams &p, int t) {
     const Unit w = unit_at<D>(p, u);
     const int tile_row0 = w.row0 + t * C::BM;
     const int i = tile_row0 + r;  // this thread's query row
-    const bool valid = i < p.N;
+    const bool valid = i < w.q_rows;
     if (w.nkv == 0) {
       // No visible key at all (key length 0): O = 0, LSE = -inf.
       if (valid) {
-        uint4 *dst = reinterpret_cast<uint4 *>(p.o + (static_cast<size_t>(w.bh) * p.N + i) * D);
+        uint4 *dst = reinterpret_cast<uint4 *>(p.o + w.o_base + i * w.o_stride);
 #pragma unroll
         for (int v4 = 0; v4 < D / 8; ++v4) dst[v4] = make_uint4(0, 0, 0, 0);
-        p.lse[static_cast<size_t>(w.bh) * p.N + i] = -INFINITY;
+        p.lse[w.lse_base + i] = -INFINITY;
       }
       continue;
     }
@@ -517,7 +552,7 @@ __device__ void role_softmax(const Sm100Ctx<D> &x, const FwdParams &p, int t) {
     if (!wait_all(C::BAR_O_FULL + t, static_cast<uint32_t>(qi & 1))) return;
     tc_fence_after();
     const float inv_l = l > 0.f ? 1.0f / l : 0.0f;
-    uint16_t *orow = p.o + (static_cast<size_t>(w.bh) * p.N + (valid ? i : 0)) * D;
+    uint16_t *orow = p.o + w.o_base + (valid ? i : 0) * w.o_stride;
 #pragma unroll
     for (int c = 0; c < D / 32; ++c) {
       uint32_t o[32];
@@ -536,7 +571,7 @@ __device__ void role_softmax(const Sm100Ctx<D> &x, const FwdParams &p, int t) {
       }
     }
     if (valid)
-      p.lse[static_cast<size_t>(w.bh) * p.N + i] =
+      p.lse[w.lse_base + i] =
           l > 0.f ? (m_ref + __log2f(l)) * 0.69314718055994530942f : -INFINITY;
     g += w.nkv;
     ++qi;

@@ -136,6 +136,18 @@ def draw(B: int, Hq: int, Hkv: int, N: int, d: int, seed: int, *, k_scale: float
     return Inputs(round_to_bf16_bits(q), round_to_bf16_bits(k), round_to_bf16_bits(v), seqlens)
 
 
+def pack(x: np.ndarray, lengths) -> np.ndarray:
+    """[B, H, N, d] -> the packed layout [sum(lengths), H, d] (rows of each
+    sequence below its length, sequences back to back)."""
+    return np.ascontiguousarray(np.concatenate(
+        [np.transpose(x[b, :, :int(L), :], (1, 0, 2)) for b, L in enumerate(lengths)], axis=0))
+
+
+def cu_seqlens(lengths) -> np.ndarray:
+    """Token offsets [B+1] of sequences stored back to back."""
+    return np.concatenate([[0], np.cumsum(np.asarray(lengths, dtype=np.int64))]).astype(np.int32)
+
+
 def draw_workload(w: Workload) -> Inputs:
     return draw(w.B, w.Hq, w.Hkv, w.N, w.d, w.seed, k_scale=w.k_scale,
                 seqlen_range=w.seqlen_range, nq=w.nq)

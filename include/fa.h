@@ -130,6 +130,25 @@ FA_API int fa_fwd_hostio(const void *q_h, const void *k_h, const void *v_h, void
                   void *stream);
 
 /*
+ * Packed variable-length forward: the tokens of B sequences are stored back
+ * to back with no padding (the padding mask of the pages' statement, without
+ * padded rows).  Same operation as fa_fwd per sequence, self-attention
+ * (each sequence's queries attend to its own keys; causal is j <= i within
+ * the sequence).
+ *  q, o : [total, Hq, d] bf16      k, v : [total, Hkv, d] bf16
+ *  lse  : [Hq, total] fp32
+ *  cu_seqlens: DEVICE int32 [B+1], cu_seqlens[0] = 0, non-decreasing,
+ *         cu_seqlens[B] = total; sequence b holds tokens
+ *         [cu_seqlens[b], cu_seqlens[b+1]).
+ *  max_seqlen: an upper bound on every sequence length (it sizes the work
+ *         grid; rows past it would not be computed).
+ *  d in {64, 128}.  Returns FA_OK once launched on `stream`, else fa_status.
+ */
+FA_API int fa_fwd_varlen(const void *q, const void *k, const void *v, void *o, float *lse,
+                         const int *cu_seqlens, int B, int Hq, int Hkv, int total, int max_seqlen,
+                         int d, float scale, int causal, void *stream, int *status_dev);
+
+/*
  * Split-KV decode forward: Nq query rows per (batch, query head) against Nk
  * cached keys.  Same operation as fa_fwd with two differences of shape:
  *  q, o : [B, Hq, Nq, d] bf16      k, v : [B, Hkv, Nk, d] bf16 (the cache)
