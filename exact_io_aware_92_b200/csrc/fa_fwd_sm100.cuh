@@ -89,13 +89,16 @@ struct Sm100Cfg {
   static constexpr uint32_t COL_S0 = 0, COL_O0 = 256;
   static constexpr float RESCALE_THRESHOLD = 8.0f;         // log2 units
   // Of every 8 consecutive pairs of probabilities, this many are computed on
-  // the FMA pipe (exp2_poly_pair) instead of the MUFU pipe, which the
-  // exponentials alone would otherwise keep as busy as the tensor pipe.
-#ifdef FA_EXP2_EMU_PAIRS
-  static constexpr int EXP2_EMU_PAIRS = FA_EXP2_EMU_PAIRS;
-#else
-  static constexpr int EXP2_EMU_PAIRS = 2;
+  // the FMA pipe (exp2_poly_pair) instead of the MUFU pipe.  At d = 128 the
+  // exponentials alone keep the MUFU pipe as busy as the MMAs keep the
+  // tensor pipe; at d = 64 the MMAs take half as long, so more move over.
+#ifndef FA_EXP2_EMU_PAIRS_D64
+#define FA_EXP2_EMU_PAIRS_D64 2
 #endif
+#ifndef FA_EXP2_EMU_PAIRS_D128
+#define FA_EXP2_EMU_PAIRS_D128 2
+#endif
+  static constexpr int EXP2_EMU_PAIRS = D == 64 ? FA_EXP2_EMU_PAIRS_D64 : FA_EXP2_EMU_PAIRS_D128;
 };
 
 // One work unit, as every role sees it.  Rows and keys are counted from the
