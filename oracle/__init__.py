@@ -33,6 +33,13 @@ def open_library(path: str):
         ctypes.c_double, ctypes.c_int, ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p,
         ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int,
     ]
+    lib.oracle_attention_bwd.restype = ctypes.c_int
+    lib.oracle_attention_bwd.argtypes = [
+        ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int,
+        ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_double,
+        ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+        ctypes.c_int,
+    ]
     lib.oracle_attention_fwd.restype = ctypes.c_int
     lib.oracle_attention_fwd.argtypes = [
         ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int,
@@ -109,3 +116,40 @@ def attention_forward(q, k, v, *, causal: bool, scale: float, seqlens=None, rows
     if rc != 0:
         raise RuntimeError(f"oracle_attention_fwd failed ({rc})")
     return (o, lse, p) if return_probs else (o, lse)
+
+
+def attention_backward(q, k, v, dout, *, causal: bool, scale: float, seqlens=None,
+                       threads: int | None = None, _lib_override=None):
+    """Gradients (dq, dk, dv) in fp64 of sum(dout * O), O = attention_forward.
+
+    q, dout: [B, Hq, N, d]; k, v: [B, Hkv, N, d], one dtype among float64,
+    float32 and uint16 (bf16 bit patterns).  dk and dv sum over the query
+    heads that share each kv head."""
+    q, k, v, dout = (np.ascontiguousarray(x) for x in (q, k, v, dout))
+    if not (q.dtype == k.dtype == v.dtype == dout.dtype) or q.dtype not in _IN_KIND:
+        raise TypeError("q, k, v, dout must share one dtype among float64, float32, uint16(bf16)")
+    B, Hq, N, d = q.shape
+    Hkv = k.shape[1]
+    if k.shape != (B, Hkv, N, d) or v.shape != k.shape or dout.shape != q.shape:
+        raise ValueError("shape mismatch")
+    if Hq % Hkv:
+        raise ValueError("Hq must be a multiple of Hkv")
+    sl = None
+    if seqlens is not None:
+        sl = np.ascontiguousarray(seqlens, dtype=np.int32)
+        if sl.shape != (B,) or np.any(sl < 0) or np.any(sl > N):
+            raise ValueError("seqlens must be int[B] within [0, N]")
+    dq = np.empty(q.shape, dtype=np.float64)
+    dk = np.empty(k.shape, dtype=np.float64)
+    dv = np.empty(k.shape, dtype=np.float64)
+
+    def ptr(a):
+        return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+    lib = _lib_override if _lib_override is not None else _load()
+    rc = lib.oracle_attention_bwd(ptr(q), ptr(k), ptr(v), ptr(dout), _IN_KIND[q.dtype], B, Hq,
+                                  Hkv, N, d, float(scale), int(bool(causal)), ptr(sl), ptr(dq),
+                                  ptr(dk), ptr(dv), int(threads or num_threads()))
+    if rc != 0:
+        raise RuntimeError(f"oracle_attention_bwd failed ({rc})")
+    return dq, dk, dv

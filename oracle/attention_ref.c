@@ -38,6 +38,18 @@
  * of its sequence, so key j is visible iff j <= i + len_b - Nq; otherwise
  * causal stays top-left (j <= i).
  *
+ * Backward (oracle_attention_bwd): the gradients of sum(dO * O) with
+ * respect to Q, K and V, written out from the same definition by the chain
+ * rule (the pages' training path recomputes these from the inputs instead of
+ * storing P: interview notes, section on memory; exam explainer,
+ * "recomputation"):
+ *     dV[g]  += P^T dO                 (summed over the query heads of group g)
+ *     dP      = dO V^T
+ *     D_i     = sum_j P[i][j] dP[i][j]
+ *     dS      = P * (dP - D)           (elementwise, D broadcast over j)
+ *     dQ      = scale * dS K
+ *     dK[g]  += scale * dS^T Q
+ *
  * S and P are materialised per block of query rows, exactly as defined.
  * Blocks are independent and run on a pool of POSIX threads.
  */
@@ -194,6 +206,139 @@ int oracle_attention_fwd_general(const void *q, const void *k, const void *v, in
     ++started;
   }
   worker(&J);
+  for (int t = 1; t <= started; ++t) pthread_join(th[t], NULL);
+  free(th);
+  return J.bad ? -1 : 0;
+}
+
+/* ------------------------------------------------------------------------- */
+/* Backward                                                                  */
+/* ------------------------------------------------------------------------- */
+
+typedef struct {
+  const void *q, *k, *v, *dout;
+  int in_kind, B, Hq, Hkv, N, d, causal;
+  double scale;
+  const int32_t *seqlens;
+  double *dq, *dk, *dv;
+  int64_t total;
+  int64_t next;
+  int bad;
+} bwd_job_t;
+
+/* One task: one (batch, kv head) group: every query head of the group, every
+ * query row; the group's dK and dV rows are written by this task only. */
+static void run_bwd_group(const bwd_job_t *J, int64_t t, double *S, double *dP, double *qrow,
+                          double *dorow) {
+  const int N = J->N, d = J->d;
+  const int b = (int)(t / J->Hkv), g = (int)(t % J->Hkv);
+  const int G = J->Hq / J->Hkv;
+  int len = J->seqlens ? J->seqlens[b] : N;
+  if (len < 0) len = 0;
+  if (len > N) len = N;
+  const int64_t kvbase = ((int64_t)b * J->Hkv + g) * N * d;
+  double *dkg = J->dk + kvbase, *dvg = J->dv + kvbase;
+  for (int64_t e = 0; e < (int64_t)N * d; ++e) dkg[e] = dvg[e] = 0.0;
+  for (int hh = 0; hh < G; ++hh) {
+    const int h = g * G + hh;
+    const int64_t qbase = ((int64_t)b * J->Hq + h) * N * d;
+    for (int i = 0; i < N; ++i) {
+      for (int c = 0; c < d; ++c) {
+        qrow[c] = in_at(J->q, J->in_kind, qbase + (int64_t)i * d + c);
+        dorow[c] = in_at(J->dout, J->in_kind, qbase + (int64_t)i * d + c);
+      }
+      /* S row, P row (softmax), dP row */
+      double m = -INFINITY;
+      for (int j = 0; j < N; ++j) {
+        const int visible = (j < len) && (!J->causal || j <= i);
+        if (!visible) {
+          S[j] = -INFINITY;
+          continue;
+        }
+        double acc = 0.0;
+        for (int c = 0; c < d; ++c) acc += qrow[c] * in_at(J->k, J->in_kind, kvbase + (int64_t)j * d + c);
+        S[j] = J->scale * acc;
+        if (S[j] > m) m = S[j];
+      }
+      double *dqrow = J->dq + qbase + (int64_t)i * d;
+      for (int c = 0; c < d; ++c) dqrow[c] = 0.0;
+      if (m == -INFINITY) continue; /* no visible key: every gradient of the row is 0 */
+      double denom = 0.0;
+      for (int j = 0; j < N; ++j) denom += exp(S[j] - m);
+      double D = 0.0;
+      for (int j = 0; j < N; ++j) {
+        S[j] = exp(S[j] - m) / denom; /* P[i][j] */
+        double acc = 0.0;
+        if (S[j] != 0.0)
+          for (int c = 0; c < d; ++c) acc += dorow[c] * in_at(J->v, J->in_kind, kvbase + (int64_t)j * d + c);
+        dP[j] = acc;
+        D += S[j] * dP[j];
+      }
+      for (int j = 0; j < N; ++j) {
+        const double p = S[j];
+        if (p == 0.0) continue;
+        const double ds = p * (dP[j] - D);
+        for (int c = 0; c < d; ++c) {
+          dqrow[c] += J->scale * ds * in_at(J->k, J->in_kind, kvbase + (int64_t)j * d + c);
+          dkg[(int64_t)j * d + c] += J->scale * ds * qrow[c];
+          dvg[(int64_t)j * d + c] += p * dorow[c];
+        }
+      }
+    }
+  }
+}
+
+static void *bwd_worker(void *arg) {
+  bwd_job_t *J = (bwd_job_t *)arg;
+  double *S = (double *)malloc(sizeof(double) * (size_t)J->N);
+  double *dP = (double *)malloc(sizeof(double) * (size_t)J->N);
+  double *qrow = (double *)malloc(sizeof(double) * (size_t)J->d);
+  double *dorow = (double *)malloc(sizeof(double) * (size_t)J->d);
+  if (!S || !dP || !qrow || !dorow) {
+    __atomic_store_n(&J->bad, 1, __ATOMIC_RELAXED);
+  } else {
+    for (;;) {
+      const int64_t t = __atomic_fetch_add(&J->next, 1, __ATOMIC_RELAXED);
+      if (t >= J->total) break;
+      run_bwd_group(J, t, S, dP, qrow, dorow);
+    }
+  }
+  free(S);
+  free(dP);
+  free(qrow);
+  free(dorow);
+  return NULL;
+}
+
+/*
+ * Gradients of sum(dout * O) for O = attention(q, k, v) as defined above.
+ * q, dout: [B, Hq, N, d]; k, v: [B, Hkv, N, d]; element type in_kind.
+ * dq: fp64 [B, Hq, N, d]; dk, dv: fp64 [B, Hkv, N, d].
+ * Returns 0, or -1 on a bad argument or an allocation failure.
+ */
+int oracle_attention_bwd(const void *q, const void *k, const void *v, const void *dout,
+                         int in_kind, int B, int Hq, int Hkv, int N, int d, double scale,
+                         int causal, const int32_t *seqlens, double *dq, double *dk, double *dv,
+                         int nthreads) {
+  if (!q || !k || !v || !dout || !dq || !dk || !dv) return -1;
+  if (B <= 0 || Hq <= 0 || Hkv <= 0 || N <= 0 || d <= 0 || Hq % Hkv != 0) return -1;
+  if (in_kind < ORACLE_IN_F64 || in_kind > ORACLE_IN_BF16) return -1;
+  bwd_job_t J;
+  memset(&J, 0, sizeof J);
+  J.q = q; J.k = k; J.v = v; J.dout = dout; J.in_kind = in_kind;
+  J.B = B; J.Hq = Hq; J.Hkv = Hkv; J.N = N; J.d = d; J.causal = causal; J.scale = scale;
+  J.seqlens = seqlens; J.dq = dq; J.dk = dk; J.dv = dv;
+  J.total = (int64_t)B * Hkv;
+  if (nthreads < 1) nthreads = 1;
+  if ((int64_t)nthreads > J.total) nthreads = (int)J.total;
+  pthread_t *th = (pthread_t *)malloc(sizeof(pthread_t) * (size_t)nthreads);
+  if (!th) return -1;
+  int started = 0;
+  for (int t = 1; t < nthreads; ++t) {
+    if (pthread_create(&th[t], NULL, bwd_worker, &J) != 0) break;
+    ++started;
+  }
+  bwd_worker(&J);
   for (int t = 1; t <= started; ++t) pthread_join(th[t], NULL);
   free(th);
   return J.bad ? -1 : 0;

@@ -323,6 +323,89 @@ def pin_single_query_is_last_causal_row(fwd):
     np.testing.assert_allclose(l1[1, :, 0], l_s[1, :, 11], rtol=0, atol=1e-13)
 
 
+# ---------------------------------------------------------------------------
+# Backward pins: fn is a pair (fwd, bwd) for these.
+# ---------------------------------------------------------------------------
+def _bwd_inputs(seed, B, Hq, Hkv, N, d):
+    rng = np.random.default_rng(seed)
+    return (rng.standard_normal((B, Hq, N, d)), rng.standard_normal((B, Hkv, N, d)) * 1.4,
+            rng.standard_normal((B, Hkv, N, d)), rng.standard_normal((B, Hq, N, d)))
+
+
+def pin_bwd_matches_torch_autograd(fwd, bwd):
+    """Gradients against torch autograd through scaled_dot_product_attention
+    in fp64 with the same explicit mask and enable_gqa."""
+    import torch
+    import torch.nn.functional as F
+    for (B, Hq, Hkv, N, d, causal, sl, seed) in [
+        (2, 4, 2, 21, 8, True, [21, 6], 61),
+        (1, 6, 3, 30, 16, False, [11], 62),
+        (2, 2, 2, 17, 4, True, None, 63),
+    ]:
+        q, k, v, do = _bwd_inputs(seed, B, Hq, Hkv, N, d)
+        sln = None if sl is None else np.array(sl, np.int32)
+        dq, dk, dv = bwd(q, k, v, do, causal=causal, scale=0.35, seqlens=sln)
+        i = torch.arange(N)[:, None]
+        j = torch.arange(N)[None, :]
+        lens = torch.tensor(sl if sl is not None else [N] * B)
+        allowed = j[None] < lens[:, None, None]
+        if causal:
+            allowed = allowed & (j <= i)[None]
+        tq, tk, tv = (torch.from_numpy(x).requires_grad_() for x in (q, k, v))
+        o = F.scaled_dot_product_attention(tq, tk, tv, attn_mask=allowed[:, None], scale=0.35,
+                                           enable_gqa=True)
+        o.backward(torch.from_numpy(do))
+        np.testing.assert_allclose(dq, tq.grad.numpy(), rtol=0, atol=1e-11)
+        np.testing.assert_allclose(dk, tk.grad.numpy(), rtol=0, atol=1e-11)
+        np.testing.assert_allclose(dv, tv.grad.numpy(), rtol=0, atol=1e-11)
+
+
+def pin_bwd_finite_differences(fwd, bwd):
+    """Central differences of L = sum(dO * O) computed with the forward
+    oracle, along random directions in Q, K and V."""
+    B, Hq, Hkv, N, d = 1, 4, 2, 13, 6
+    q, k, v, do = _bwd_inputs(64, B, Hq, Hkv, N, d)
+    sl = np.array([10], np.int32)
+    dq, dk, dv = bwd(q, k, v, do, causal=True, scale=0.5, seqlens=sl)
+
+    def loss(qq, kk, vv):
+        o, _ = fwd(qq, kk, vv, causal=True, scale=0.5, seqlens=sl)
+        return float(np.sum(do * o))
+
+    rng = np.random.default_rng(65)
+    h = 1e-5
+    for which, grad in (("q", dq), ("k", dk), ("v", dv)):
+        for _ in range(3):
+            u = rng.standard_normal(grad.shape)
+            args = {"q": q, "k": k, "v": v}
+            plus = dict(args)
+            minus = dict(args)
+            plus[which] = args[which] + h * u
+            minus[which] = args[which] - h * u
+            fd = (loss(plus["q"], plus["k"], plus["v"]) - loss(minus["q"], minus["k"], minus["v"])) / (2 * h)
+            assert abs(fd - float(np.sum(grad * u))) <= 1e-6 * max(1.0, abs(fd)), which
+
+
+def pin_bwd_key_gradients_sum_to_zero(fwd, bwd):
+    """Adding one vector to every key shifts each row's scores by a constant,
+    which the softmax ignores, so the key gradients of each (batch, kv head)
+    sum to zero; keys that no query sees get zero gradients, and so do query
+    rows that see no key."""
+    B, Hq, Hkv, N, d = 2, 4, 2, 25, 8
+    q, k, v, do = _bwd_inputs(66, B, Hq, Hkv, N, d)
+    sl = np.array([25, 9], np.int32)
+    for causal in (False, True):
+        dq, dk, dv = bwd(q, k, v, do, causal=causal, scale=0.4, seqlens=sl)
+        np.testing.assert_allclose(dk.sum(axis=2), 0.0, rtol=0, atol=1e-12)
+        assert np.all(dk[1, :, 9:] == 0.0) and np.all(dv[1, :, 9:] == 0.0)
+    dq, dk, dv = bwd(q, k, v, do, causal=False, scale=0.4, seqlens=np.array([25, 0], np.int32))
+    assert np.all(dq[1] == 0.0) and np.all(dk[1] == 0.0) and np.all(dv[1] == 0.0)
+
+
+BWD_PINS = [pin_bwd_matches_torch_autograd, pin_bwd_finite_differences,
+            pin_bwd_key_gradients_sum_to_zero]
+
+
 ALL_PINS = [
     pin_golden, pin_probs_are_a_row_softmax, pin_constant_v, pin_single_visible_key,
     pin_causal_first_row, pin_matches_torch_sdpa, pin_brute_force,

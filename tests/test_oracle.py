@@ -2,12 +2,17 @@
 import pytest
 
 import oracle
-from oracle_pins import ALL_PINS
+from oracle_pins import ALL_PINS, BWD_PINS
 
 
 @pytest.mark.parametrize("pin", ALL_PINS, ids=lambda p: p.__name__)
 def test_oracle_pin(pin):
     pin(oracle.attention_forward)
+
+
+@pytest.mark.parametrize("pin", BWD_PINS, ids=lambda p: p.__name__)
+def test_oracle_backward_pin(pin):
+    pin(oracle.attention_forward, oracle.attention_backward)
 
 
 def test_oracle_rejects_bad_arguments():

@@ -35,6 +35,14 @@ MUTANTS = {
                            "((int64_t)h * J->B + b) * J->Nq * d"),
     "kv_head_dropped": ("((int64_t)b * J->Hkv + g) * N * d", "((int64_t)b * J->Hkv) * N * d"),
     "seqlen_of_batch_0": ("J->seqlens ? J->seqlens[b] : N", "J->seqlens ? J->seqlens[0] : N"),
+    "bwd_missing_row_term": ("const double ds = p * (dP[j] - D);", "const double ds = p * dP[j];"),
+    "bwd_dk_without_scale": ("dkg[(int64_t)j * d + c] += J->scale * ds * qrow[c];",
+                             "dkg[(int64_t)j * d + c] += ds * qrow[c];"),
+    "bwd_dv_from_ds": ("dvg[(int64_t)j * d + c] += p * dorow[c];",
+                       "dvg[(int64_t)j * d + c] += ds * dorow[c];"),
+    "bwd_dq_from_v": ("dqrow[c] += J->scale * ds * in_at(J->k,", "dqrow[c] += J->scale * ds * in_at(J->v,"),
+    "bwd_causal_off_by_one": ("(j < len) && (!J->causal || j <= i);",
+                              "(j < len) && (!J->causal || j < i);"),
     "masked_row_not_zeroed": ("for (int j = 0; j < N; ++j) Srow[j] = 0.0;",
                               "for (int j = 0; j < N; ++j) Srow[j] = 1.0 / N;"),
 }
@@ -53,7 +61,8 @@ def test_unmutated_copy_passes(tmp_path):
         text = f.read()
     lib = str(tmp_path / "clean.so")
     _compile(text, lib)
-    r = subprocess.run([sys.executable, RUNNER, lib], capture_output=True, text=True, timeout=600)
+    r = subprocess.run([sys.executable, RUNNER, lib, "--all"], capture_output=True, text=True,
+                       timeout=600)
     assert r.returncode == 0, r.stdout + r.stderr
 
 
