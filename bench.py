@@ -363,6 +363,47 @@ def report_all_workloads(args):
                           "peak_source": src}), flush=True)
     report_varlen(args, dev)
     report_decode(args, dev)
+    report_backward(args, dev)
+
+
+def report_backward(args, dev):
+    """The backward (fa_bwd) on the GPT-2 and Llama GQA workloads.  FLOPs are
+    counted as 2.5x the forward's (the five N^2 d products of the gradient);
+    this design executes seven, since the dQ kernel recomputes S and dP."""
+    import torch
+    from exact_io_aware_92_b200 import attention
+    peaks, src = load_peaks()
+    peak = float(peaks["bf16_tflops"])
+    for w in (wl.GPT2, wl.LLAMA_GQA):
+        inp = wl.draw_workload(w)
+        q, k, v = (torch.from_numpy(x).view(torch.bfloat16).to(dev)
+                   for x in (inp.q_bits, inp.k_bits, inp.v_bits))
+        g = torch.Generator(device=dev).manual_seed(w.seed + 100)
+        do = torch.randn(q.shape, generator=g, device=dev, dtype=torch.float32).to(torch.bfloat16)
+        o, lse = attention.fwd(q, k, v, causal=w.causal, scale=w.scale)
+        ws = torch.empty(attention.bwd_workspace_size(w.B, w.Hq, w.N), dtype=torch.uint8,
+                         device=dev)
+        flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
+        for _ in range(args.warmup):
+            attention.bwd(q, k, v, o, do, lse, causal=w.causal, scale=w.scale, workspace=ws)
+        torch.cuda.synchronize(dev)
+        times = []
+        for _ in range(args.steps):
+            flush.zero_()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            attention.bwd(q, k, v, o, do, lse, causal=w.causal, scale=w.scale, workspace=ws)
+            e1.record()
+            e1.synchronize()
+            times.append(e0.elapsed_time(e1))
+        ms = statistics.median(times)
+        f = 2.5 * wl.flops(w, inp.seqlens)
+        print(json.dumps({"workload": w.name + "@backward", "ms_median": ms,
+                          "tflops": f / ms / 1e9, "frac_of_peak": f / ms / 1e9 / peak,
+                          "tflops_executed": 1.4 * f / ms / 1e9, "flops": f,
+                          "launches_per_call": 3, "l2": "flushed between steps",
+                          "peak_source": src}), flush=True)
+        del q, k, v, do, o, lse, ws, flush
 
 
 def report_varlen(args, dev):

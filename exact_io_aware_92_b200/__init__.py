@@ -1,4 +1,5 @@
-"""Exact, IO-aware attention forward for B200 (sm_100a).
+"""Exact, IO-aware attention for B200 (sm_100a): forward, backward, packed
+variable-length and split-KV decode.
 
 The computation lives in hand-written CUDA kernels behind the C ABI of
 ``include/fa.h`` (``libfa_b200.so``); this package holds the ctypes binding
@@ -7,12 +8,13 @@ inputs (``workloads``).
 """
 from . import workloads  # noqa: F401
 
-__all__ = ["fwd", "fwd_varlen", "fwd_decode", "decode_workspace_size", "check_status", "fwd_hostio",
-           "workloads"]
+_API = ("fwd", "bwd", "fwd_varlen", "fwd_decode", "decode_workspace_size", "bwd_workspace_size",
+        "check_status", "fwd_hostio")
+__all__ = list(_API) + ["workloads"]
 
 
 def __getattr__(name):
-    if name in ("fwd", "fwd_varlen", "fwd_decode", "decode_workspace_size", "check_status", "fwd_hostio"):
+    if name in _API:
         from . import attention
         return getattr(attention, name)
     raise AttributeError(name)

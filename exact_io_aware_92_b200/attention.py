@@ -61,6 +61,38 @@ def fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *, causal: bool = Fal
     return out, lse
 
 
+def bwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: torch.Tensor,
+        dout: torch.Tensor, lse: torch.Tensor, *, causal: bool = False,
+        scale: float | None = None, seqlens: torch.Tensor | None = None,
+        workspace: torch.Tensor | None = None, status: torch.Tensor | None = None):
+    """Attention backward by recomputation.  q, o, dout: [B, Hq, N, d];
+    k, v: [B, Hkv, N, d] (bf16, contiguous); lse: fp32 [B, Hq, N] from fwd
+    with the same arguments.  Returns (dq, dk, dv) in bf16."""
+    B, Hq, Hkv, N, d = _check_qkv(q, k, v, torch.bfloat16)
+    for name, t in (("o", o), ("dout", dout)):
+        if t.shape != q.shape or t.dtype != torch.bfloat16 or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous bf16 tensor shaped like q")
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    dq = torch.empty_like(q)
+    dk = torch.empty_like(k)
+    dv = torch.empty_like(v)
+    if workspace is None:
+        workspace = torch.empty(bwd_workspace_size(B, Hq, N), dtype=torch.uint8, device=q.device)
+    sl_ptr = None
+    if seqlens is not None:
+        if seqlens.dtype != torch.int32 or seqlens.device != q.device or seqlens.numel() != B:
+            raise ValueError("seqlens must be int32 [B] on q's device")
+        sl_ptr = seqlens.data_ptr()
+    rc = _lib.load().fa_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
+                            dout.data_ptr(), lse.data_ptr(), dq.data_ptr(), dk.data_ptr(),
+                            dv.data_ptr(), B, Hq, Hkv, N, d, scale, int(bool(causal)), sl_ptr,
+                            workspace.data_ptr(), workspace.numel() * workspace.element_size(),
+                            _stream_handle(q.device),
+                            None if status is None else status.data_ptr())
+    _lib.check(rc, "fa_bwd")
+    return dq, dk, dv
+
+
 def fwd_varlen(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, cu_seqlens: torch.Tensor,
                max_seqlen: int, *, causal: bool = False, scale: float | None = None,
                out: torch.Tensor | None = None, lse: torch.Tensor | None = None,
@@ -90,6 +122,11 @@ def fwd_varlen(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, cu_seqlens: to
                                    None if status is None else status.data_ptr())
     _lib.check(rc, "fa_fwd_varlen")
     return out, lse
+
+
+def bwd_workspace_size(B: int, Hq: int, N: int) -> int:
+    """Bytes of device workspace bwd needs (per-row D and LSE*log2(e))."""
+    return int(_lib.load().fa_bwd_workspace_size(B, Hq, N))
 
 
 def decode_workspace_size(B: int, Hq: int, Hkv: int, Nq: int, Nk: int, d: int,

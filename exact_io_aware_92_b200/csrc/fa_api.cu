@@ -14,6 +14,7 @@
 #include <cuda_runtime.h>
 
 #include "fa.h"
+#include "fa_bwd_sm100.cuh"
 #include "fa_decode.cuh"
 #include "fa_fwd_f32.cuh"
 #include "fa_fwd_sm100.cuh"
@@ -34,6 +35,7 @@ struct DeviceState {
   int *status_word = nullptr;  // device address of g_status_word
   bool attr64 = false, attr128 = false;
   bool dec_attr64 = false, dec_attr128 = false;
+  bool bwd_attr64 = false, bwd_attr128 = false;
 };
 DeviceState g_dev[kMaxDevices];
 std::mutex g_mu;
@@ -310,6 +312,71 @@ int launch_decode(DeviceState *ds, const void *q, const void *k, const void *v, 
   return FA_OK;
 }
 
+size_t bwd_workspace_bytes(int B, int Hq, int N) {
+  const size_t npad = (static_cast<size_t>(N) + 127) / 128 * 128;
+  return 2 * static_cast<size_t>(B) * Hq * npad * sizeof(float);
+}
+
+template <int D>
+int launch_bwd(DeviceState *ds, const void *q, const void *k, const void *v, const void *o,
+               const void *dout, const float *lse, void *dq, void *dk, void *dv, int B, int Hq,
+               int Hkv, int N, float scale, int causal, const int *seqlens, void *workspace,
+               cudaStream_t stream, int *status) {
+  using C = fa::BwdCfg<D>;
+  bool &attr = (D == 64) ? ds->bwd_attr64 : ds->bwd_attr128;
+  if (!attr) {
+    if (cudaFuncSetAttribute(fa::fa_bwd_dkdv_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             C::SMEM_KV) != cudaSuccess ||
+        cudaFuncSetAttribute(fa::fa_bwd_dq_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             C::SMEM_Q) != cudaSuccess) {
+      cudaGetLastError();
+      return FA_ERR_LAUNCH;
+    }
+    attr = true;
+  }
+  CUtensorMap tq, tk, tv, tdo;
+  if (make_map(&tq, q, B * Hq, N, D) != FA_OK || make_map(&tk, k, B * Hkv, N, D) != FA_OK ||
+      make_map(&tv, v, B * Hkv, N, D) != FA_OK || make_map(&tdo, dout, B * Hq, N, D) != FA_OK)
+    return FA_ERR_CUDA;
+  fa::BwdParams p;
+  p.o = static_cast<const uint16_t *>(o);
+  p.dout = static_cast<const uint16_t *>(dout);
+  p.lse = lse;
+  p.dq = static_cast<uint16_t *>(dq);
+  p.dk = static_cast<uint16_t *>(dk);
+  p.dv = static_cast<uint16_t *>(dv);
+  p.Npad = (N + 127) / 128 * 128;
+  const size_t vec = static_cast<size_t>(B) * Hq * p.Npad;
+  p.ws_lse2 = static_cast<float *>(workspace);
+  p.ws_delta = p.ws_lse2 + vec;
+  p.seqlens = seqlens;
+  p.status = status;
+  p.B = B;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.N = N;
+  p.group = Hq / Hkv;
+  p.causal = causal ? 1 : 0;
+  p.q_tiles = p.Npad / 128;
+  p.scale = scale;
+  p.scale_log2 = scale * kLog2e;
+  p.wait_limit_ns = kWaitLimitNs;
+  const long long prep_blocks = (static_cast<long long>(vec) + 127) / 128;
+  const long long kv_units = static_cast<long long>(p.q_tiles) * B * Hkv;
+  const long long q_units = static_cast<long long>(p.q_tiles) * B * Hq;
+  if (prep_blocks > 0x7fffffffll || kv_units > 0x7fffffffll || q_units > 0x7fffffffll)
+    return FA_ERR_SHAPE;
+  fa::fa_bwd_prep_kernel<D><<<static_cast<unsigned>(prep_blocks), 128, 0, stream>>>(p);
+  if (cudaGetLastError() != cudaSuccess) return FA_ERR_LAUNCH;
+  fa::fa_bwd_dkdv_kernel<D><<<static_cast<unsigned>(kv_units), C::THREADS, C::SMEM_KV, stream>>>(
+      tq, tk, tv, tdo, p);
+  if (cudaGetLastError() != cudaSuccess) return FA_ERR_LAUNCH;
+  fa::fa_bwd_dq_kernel<D><<<static_cast<unsigned>(q_units), C::THREADS, C::SMEM_Q, stream>>>(
+      tq, tk, tv, tdo, p);
+  if (cudaGetLastError() != cudaSuccess) return FA_ERR_LAUNCH;
+  return FA_OK;
+}
+
 // Waits on a barrier that nothing arrives at; the bounded wait must give up.
 __global__ void bounded_wait_selftest_kernel(int *status, unsigned long long limit_ns) {
   __shared__ __align__(8) uint64_t bar;
@@ -458,6 +525,32 @@ int fa_fwd_varlen(const void *q, const void *k, const void *v, void *o, float *l
                                    nullptr, st, status, cu_seqlens, total)
                  : launch_bf16<128>(ds, q, k, v, o, lse, B, Hq, Hkv, max_seqlen, scale, causal,
                                     nullptr, st, status, cu_seqlens, total);
+}
+
+size_t fa_bwd_workspace_size(int B, int Hq, int N) {
+  if (B <= 0 || Hq <= 0 || N <= 0) return 0;
+  return bwd_workspace_bytes(B, Hq, N);
+}
+
+int fa_bwd(const void *q, const void *k, const void *v, const void *o, const void *dout,
+           const float *lse, void *dq, void *dk, void *dv, int B, int Hq, int Hkv, int N, int d,
+           float scale, int causal, const int *seqlens, void *workspace, size_t workspace_bytes,
+           void *stream, int *status_dev) {
+  int rc = check_args(q, k, v, o, lse, B, Hq, Hkv, N, d, scale);
+  if (rc != FA_OK) return rc;
+  if (!dout || !dq || !dk || !dv) return FA_ERR_NULL;
+  if (!aligned16(dout) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv)) return FA_ERR_ALIGN;
+  if (!workspace || !aligned16(workspace) || workspace_bytes < bwd_workspace_bytes(B, Hq, N))
+    return FA_ERR_WORKSPACE;
+  DeviceState *ds = nullptr;
+  rc = current_device(&ds);
+  if (rc != FA_OK) return rc;
+  int *status = status_dev ? status_dev : ds->status_word;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  return d == 64 ? launch_bwd<64>(ds, q, k, v, o, dout, lse, dq, dk, dv, B, Hq, Hkv, N, scale,
+                                  causal, seqlens, workspace, st, status)
+                 : launch_bwd<128>(ds, q, k, v, o, dout, lse, dq, dk, dv, B, Hq, Hkv, N, scale,
+                                   causal, seqlens, workspace, st, status);
 }
 
 size_t fa_decode_workspace_size(int B, int Hq, int Hkv, int Nq, int Nk, int d, int num_splits) {

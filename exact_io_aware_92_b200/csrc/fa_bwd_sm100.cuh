@@ -1,0 +1,602 @@
+// Attention backward on B200 tensor cores (sm_100a), by recomputation: the
+// probabilities are rebuilt from Q, K and the saved per-row log-sum-exp
+// instead of being stored (interview notes "Why is FlashAttention faster",
+// section on memory: training can store less by recomputing; exam explainer,
+// "recomputation": the backward pass recomputes what it needs).  With
+// P = exp(scale Q K^T - LSE), dP = dO V^T, D_i = sum_c dO_ic O_ic and
+// dS = P * (dP - D):  dV = P^T dO,  dK = scale dS^T Q,  dQ = scale dS K.
+//
+// fa_bwd_prep_kernel   D and LSE*log2(e) per query row, in a workspace padded
+//                      to whole 128-row tiles (padding: D = 0, LSE = +inf).
+// fa_bwd_dkdv_kernel   one CTA per 128-key tile of one (batch, kv head); it
+//                      walks the query tiles of every query head of the
+//                      group.  Per query tile:  S^T = K Q^T, dP^T = V dO^T
+//                      (tcgen05, TMEM); the softmax warpgroup (thread = key
+//                      row = TMEM lane) forms P^T and dS^T in bf16 over those
+//                      TMEM columns; then dV += P^T dO and dK += dS^T Q with
+//                      the left operand read from TMEM.
+// fa_bwd_dq_kernel     one CTA per 128-row query tile; per key tile:
+//                      S = Q K^T, dP = dO V^T, dS in bf16 over S, dQ += dS K.
+// Both tcgen05 kernels use 192 threads: warps 0-3 elementwise work, warp 4
+// TMA producer, warp 5 MMA issuer (one elected lane).  Every wait is bounded.
+#pragma once
+
+#include <cstdint>
+
+#include "sm100_ptx.cuh"
+
+namespace fa {
+
+struct BwdParams {
+  const uint16_t *o, *dout;   // bf16 [B,Hq,N,d]
+  const float *lse;           // fp32 [B,Hq,N]
+  uint16_t *dq, *dk, *dv;     // bf16 [B,Hq,N,d], [B,Hkv,N,d] x2
+  float *ws_lse2;             // [B*Hq][Npad]: LSE * log2(e); +inf on padding rows
+  float *ws_delta;            // [B*Hq][Npad]: D; 0 on padding rows
+  const int *seqlens;
+  int *status;
+  int B, Hq, Hkv, N, Npad, group, causal;
+  int q_tiles;                // Npad / 128
+  float scale, scale_log2;
+  unsigned long long wait_limit_ns;
+};
+
+template <int D>
+struct BwdCfg {
+  static constexpr int HALF_BYTES = 128 * 64 * 2;
+  static constexpr int TILE_BYTES = 128 * D * 2;
+  static constexpr int THREADS = 192;
+  static constexpr uint32_t COL_A = 0, COL_B = 128, COL_C = 256, COL_D = 384;
+  // dK/dV kernel: K, V resident; ring of (Q, dO, LSE2, D) stages.
+  static constexpr int KV_STAGES = 2;
+  static constexpr int OFF_K = 0, OFF_V = TILE_BYTES, OFF_RING = 2 * TILE_BYTES;
+  static constexpr int STAGE_BYTES = 2 * TILE_BYTES + 1024;  // Q, dO, 128 LSE2 + 128 D floats
+  static constexpr int OFF_BAR_KV = OFF_RING + KV_STAGES * STAGE_BYTES;
+  static constexpr int SMEM_KV = OFF_BAR_KV + 128 + 1024;
+  // dQ kernel: Q, dO resident; ring of (K, V) stages.
+  static constexpr int Q_STAGES = 2;
+  static constexpr int OFF_Q = 0, OFF_DO = TILE_BYTES, OFF_KVRING = 2 * TILE_BYTES;
+  static constexpr int KVSTAGE_BYTES = 2 * TILE_BYTES;
+  static constexpr int OFF_BAR_Q = OFF_KVRING + Q_STAGES * KVSTAGE_BYTES;
+  static constexpr int SMEM_Q = OFF_BAR_Q + 128 + 1024;
+};
+
+// ---------------------------------------------------------------------------
+// Preprocess: D_i = sum_c dO_ic O_ic, LSE2_i = LSE_i * log2(e)
+// ---------------------------------------------------------------------------
+template <int D>
+__global__ void __launch_bounds__(128) fa_bwd_prep_kernel(const BwdParams p) {
+  const long long row = static_cast<long long>(blockIdx.x) * 128 + threadIdx.x;  // over B*Hq*Npad
+  if (row >= static_cast<long long>(p.B) * p.Hq * p.Npad) return;
+  const int bh = static_cast<int>(row / p.Npad), i = static_cast<int>(row % p.Npad);
+  if (i >= p.N) {
+    p.ws_lse2[row] = INFINITY;
+    p.ws_delta[row] = 0.f;
+    return;
+  }
+  const size_t base = (static_cast<size_t>(bh) * p.N + i) * D;
+  const uint4 *po = reinterpret_cast<const uint4 *>(p.o + base);
+  const uint4 *pd = reinterpret_cast<const uint4 *>(p.dout + base);
+  float acc = 0.f;
+#pragma unroll
+  for (int c = 0; c < D / 8; ++c) {
+    const uint4 a = po[c], b = pd[c];
+    const uint32_t wa[4] = {a.x, a.y, a.z, a.w}, wb[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      acc = fmaf(__uint_as_float(wa[e] << 16), __uint_as_float(wb[e] << 16), acc);
+      acc = fmaf(__uint_as_float(wa[e] & 0xFFFF0000u), __uint_as_float(wb[e] & 0xFFFF0000u), acc);
+    }
+  }
+  p.ws_delta[row] = acc;
+  const float l = p.lse[static_cast<size_t>(bh) * p.N + i];
+  // A row that saw no key keeps no gradient: +inf makes its probabilities 0.
+  p.ws_lse2[row] = (l == -INFINITY) ? INFINITY : l * 1.4426950408889634f;
+}
+
+// Bulk copy of `bytes` (multiple of 16) global -> shared, completing on `bar`.
+__device__ __forceinline__ void bwd_bulk(uint32_t dst, const void *src, uint32_t bytes,
+                                         uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::
+          "r"(dst),
+      "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(bar)
+      : "memory");
+}
+
+// Load one 128-row x D bf16 tile (two 64-column boxes) with TMA.
+template <int D>
+__device__ __forceinline__ void load_tile(uint32_t dst, const CUtensorMap *m, uint32_t bar,
+                                          int row, int plane) {
+#pragma unroll
+  for (int half = 0; half < D / 64; ++half)
+    tma_load_3d(dst + half * BwdCfg<D>::HALF_BYTES, m, bar, half * 64, row, plane);
+}
+
+// ---------------------------------------------------------------------------
+// dK, dV
+// ---------------------------------------------------------------------------
+template <int D>
+__global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
+    fa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q,
+                       const __grid_constant__ CUtensorMap tm_k,
+                       const __grid_constant__ CUtensorMap tm_v,
+                       const __grid_constant__ CUtensorMap tm_do, const BwdParams p) {
+  using C = BwdCfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  uint8_t *smem = smem_raw + (base - raw);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  // Unit: (key tile, batch, kv head); causal units with the most query
+  // tiles (the first key tiles) run first.
+  const int BHkv = p.B * p.Hkv;
+  const int kt = static_cast<int>(blockIdx.x) / BHkv;
+  const int bkv = static_cast<int>(blockIdx.x) % BHkv;
+  const int b = bkv / p.Hkv, hkv = bkv % p.Hkv;
+  int L = p.N;
+  if (p.seqlens) L = min(max(p.seqlens[b], 0), p.N);
+  const int key0 = kt * 128;
+  const int qt0 = p.causal ? kt : 0;  // first query tile that sees these keys
+  const int nq_per_head = p.q_tiles - qt0;
+  const int nsteps = (key0 < L) ? p.group * nq_per_head : 0;
+
+  const uint32_t bar_kv = base + C::OFF_BAR_KV;         // K, V loaded
+  const uint32_t bar_full = bar_kv + 8;                  // [KV_STAGES]
+  const uint32_t bar_empty = bar_full + 8 * C::KV_STAGES;  // [KV_STAGES]
+  const uint32_t bar_st = bar_empty + 8 * C::KV_STAGES;  // S^T and dP^T in TMEM
+  const uint32_t bar_pds = bar_st + 8;                   // P^T and dS^T in TMEM
+  const uint32_t bar_done = bar_pds + 8;                 // all products finished
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + C::OFF_BAR_KV + 120);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + C::OFF_BAR_KV + 124);
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar_kv, 1);
+    for (int s = 0; s < C::KV_STAGES; ++s) {
+      mbar_init(bar_full + 8 * s, 1);
+      mbar_init(bar_empty + 8 * s, 1);
+    }
+    mbar_init(bar_st, 1);
+    mbar_init(bar_pds, 128);
+    mbar_init(bar_done, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(smem_u32(tmem_slot), 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *reinterpret_cast<volatile uint32_t *>(tmem_slot);
+
+  auto step_head = [&](int s) { return hkv * p.group + s / nq_per_head; };
+  auto step_qt = [&](int s) { return qt0 + s % nq_per_head; };
+
+  if (nsteps > 0 && warp == 4) {
+    if (lane == 0) {
+      // --- producer ---
+      mbar_arrive_expect_tx(bar_kv, 2 * C::TILE_BYTES);
+      load_tile<D>(base + C::OFF_K, &tm_k, bar_kv, key0, bkv);
+      load_tile<D>(base + C::OFF_V, &tm_v, bar_kv, key0, bkv);
+      int s = 0;
+      for (; s < nsteps; ++s) {
+        const int st = s % C::KV_STAGES;
+        if (!mbar_wait_bounded(bar_empty + 8 * st, ((s / C::KV_STAGES) & 1) ^ 1, abort_flag,
+                               p.status, p.wait_limit_ns, kErrTimeout))
+          break;
+        const int h = step_head(s), qt = step_qt(s);
+        const int bh = b * p.Hq + h;
+        const uint32_t dst = base + C::OFF_RING + st * C::STAGE_BYTES;
+        mbar_arrive_expect_tx(bar_full + 8 * st, 2 * C::TILE_BYTES + 1024);
+        load_tile<D>(dst, &tm_q, bar_full + 8 * st, qt * 128, bh);
+        load_tile<D>(dst + C::TILE_BYTES, &tm_do, bar_full + 8 * st, qt * 128, bh);
+        const size_t vrow = static_cast<size_t>(bh) * p.Npad + qt * 128;
+        bwd_bulk(dst + 2 * C::TILE_BYTES, p.ws_lse2 + vrow, 512, bar_full + 8 * st);
+        bwd_bulk(dst + 2 * C::TILE_BYTES + 512, p.ws_delta + vrow, 512, bar_full + 8 * st);
+      }
+      volatile int never = 0;
+      mbar_wait_bounded(bar_kv, 0, &never, p.status, p.wait_limit_ns, kErrTimeout);
+      for (int st = 0; st < C::KV_STAGES && st < s; ++st) {
+        const int last = st + C::KV_STAGES * ((s - 1 - st) / C::KV_STAGES);
+        mbar_wait_bounded(bar_full + 8 * st, (last / C::KV_STAGES) & 1, &never, p.status,
+                          p.wait_limit_ns, kErrTimeout);
+      }
+    }
+  } else if (nsteps > 0 && warp == 5) {
+    // --- MMA issuer ---
+    const bool leader = elect_one();
+    constexpr uint32_t IDESC_SS = idesc_bf16_f32(128, 128, 0, 0);  // K-major A and B
+    constexpr uint32_t IDESC_TS = idesc_bf16_f32(128, D, 0, 1);    // A in TMEM, B MN-major
+    const uint64_t dK = smem_desc_sw128(base + C::OFF_K, 16, 1024);
+    const uint64_t dV = smem_desc_sw128(base + C::OFF_V, 16, 1024);
+    auto wait = [&](uint32_t bar, uint32_t par) {
+      const bool ok = mbar_wait_bounded(bar, par, abort_flag, p.status, p.wait_limit_ns,
+                                        kErrTimeout);
+      return __all_sync(0xffffffffu, ok);
+    };
+    auto commit = [&](uint32_t bar) {
+      if (leader) tc_commit(bar);
+      __syncwarp();
+    };
+    if (wait(bar_kv, 0)) {
+      for (int s = 0; s < nsteps; ++s) {
+        const int st = s % C::KV_STAGES;
+        if (!wait(bar_full + 8 * st, (s / C::KV_STAGES) & 1)) break;
+        tc_fence_after();
+        const uint32_t stage = base + C::OFF_RING + st * C::STAGE_BYTES;
+        const uint64_t dQk = smem_desc_sw128(stage, 16, 1024);
+        const uint64_t dOk = smem_desc_sw128(stage + C::TILE_BYTES, 16, 1024);
+        // S^T = K Q^T and dP^T = V dO^T (K = d in steps of 16).
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = ((kk / 4) * C::HALF_BYTES + (kk % 4) * 32) >> 4;
+          if (leader) tc_mma_ss(tmem + C::COL_A, dK + off, dQk + off, IDESC_SS, kk > 0);
+        }
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = ((kk / 4) * C::HALF_BYTES + (kk % 4) * 32) >> 4;
+          if (leader) tc_mma_ss(tmem + C::COL_B, dV + off, dOk + off, IDESC_SS, kk > 0);
+        }
+        __syncwarp();
+        commit(bar_st);
+        if (!wait(bar_pds, s & 1)) break;
+        tc_fence_after();
+        // dV += P^T dO, dK += dS^T Q: K = 128 queries in steps of 16; the
+        // right operand is the tile read MN-major (queries as rows).
+        const uint64_t dOm = smem_desc_sw128(stage + C::TILE_BYTES, C::HALF_BYTES, 1024);
+        const uint64_t dQm = smem_desc_sw128(stage, C::HALF_BYTES, 1024);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          if (leader) {
+            tc_mma_ts(tmem + C::COL_D, tmem + C::COL_A + kk * 8, dOm + ((kk * 2048) >> 4),
+                      IDESC_TS, (s > 0 || kk > 0) ? 1u : 0u);
+            tc_mma_ts(tmem + C::COL_C, tmem + C::COL_B + kk * 8, dQm + ((kk * 2048) >> 4),
+                      IDESC_TS, (s > 0 || kk > 0) ? 1u : 0u);
+          }
+        }
+        __syncwarp();
+        commit(bar_empty + 8 * st);
+      }
+    }
+    commit(bar_done);
+    volatile int never = 0;
+    mbar_wait_bounded(bar_done, 0, &never, p.status, p.wait_limit_ns, kErrTimeout);
+  } else if (warp < 4) {
+    // --- elementwise warpgroup: thread = key row ---
+    const int j = key0 + threadIdx.x;
+    const uint32_t lane_base = static_cast<uint32_t>(warp) * 32u << 16;
+    const uint32_t tA = tmem + lane_base + C::COL_A, tB = tmem + lane_base + C::COL_B;
+    const bool key_ok = j < L;
+    bool ok = true;
+    for (int s = 0; s < nsteps && ok; ++s) {
+      const int st = s % C::KV_STAGES;
+      const bool got = mbar_wait_bounded(bar_st, s & 1, abort_flag, p.status, p.wait_limit_ns,
+                                         kErrTimeout);
+      if (!__all_sync(0xffffffffu, got)) {
+        ok = false;
+        break;
+      }
+      // The per-row vectors came with the stage's bulk copies: observe that
+      // stage's fill directly (it is refilled only after this step's P^T and
+      // dS^T are published, so the phase cannot have moved on).
+      const bool filled = mbar_wait_bounded(bar_full + 8 * st, (s / C::KV_STAGES) & 1, abort_flag,
+                                            p.status, p.wait_limit_ns, kErrTimeout);
+      if (!__all_sync(0xffffffffu, filled)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const int q0 = step_qt(s) * 128;
+      const float *lse2 =
+          reinterpret_cast<const float *>(smem + C::OFF_RING + st * C::STAGE_BYTES + 2 * C::TILE_BYTES);
+      const float *delta = lse2 + 128;
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+        uint32_t sv[64], dp[64];
+        tmem_ld32(tA + 64 * half, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
+        tmem_ld32(tA + 64 * half + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
+        tmem_ld32(tB + 64 * half, *reinterpret_cast<uint32_t(*)[32]>(&dp[0]));
+        tmem_ld32(tB + 64 * half + 32, *reinterpret_cast<uint32_t(*)[32]>(&dp[32]));
+        tmem_wait_ld();
+        uint32_t pk[32], dk[32];
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+          float pv[2], dv[2];
+#pragma unroll
+          for (int u = 0; u < 2; ++u) {
+            const int c = 64 * half + 2 * e + u;  // query column within the tile
+            const int i = q0 + c;
+            const bool vis = key_ok && (!p.causal || i >= j);
+            const float pp = vis ? ex2_approx(fmaf(__uint_as_float(sv[2 * e + u]), p.scale_log2,
+                                                   -lse2[c]))
+                                 : 0.f;
+            pv[u] = pp;
+            dv[u] = pp * (__uint_as_float(dp[2 * e + u]) - delta[c]);
+          }
+          pk[e] = pack_bf16x2(pv[0], pv[1]);
+          dk[e] = pack_bf16x2(dv[0], dv[1]);
+        }
+        // P^T over S^T's columns 32*half.., dS^T over dP^T's.
+        tmem_st32(tA + 32 * half, pk);
+        tmem_st32(tB + 32 * half, dk);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(bar_pds);
+    }
+    // Epilogue: dK = scale * sum dS^T Q, dV = sum P^T dO, in bf16.
+    if (ok && nsteps > 0) {
+      const bool got = mbar_wait_bounded(bar_done, 0, abort_flag, p.status, p.wait_limit_ns,
+                                         kErrTimeout);
+      ok = __all_sync(0xffffffffu, got);
+    }
+    // tcgen05.ld is warp-collective: every lane loads (ok is warp-uniform);
+    // only the stores are limited to rows that exist.
+    if (ok) {
+      const bool row_ok = j < p.N;
+      const size_t row = (static_cast<size_t>(bkv) * p.N + (row_ok ? j : 0)) * D;
+      if (nsteps > 0) tc_fence_after();
+#pragma unroll
+      for (int which = 0; which < 2; ++which) {
+        uint16_t *dst = (which == 0 ? p.dk : p.dv) + row;
+        const float mult = which == 0 ? p.scale : 1.0f;
+        const uint32_t tcol = tmem + lane_base + (which == 0 ? C::COL_C : C::COL_D);
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t r[32];
+          if (nsteps > 0) {
+            tmem_ld32(tcol + 32 * c, r);
+            tmem_wait_ld();
+          } else {
+#pragma unroll
+            for (int e = 0; e < 32; ++e) r[e] = 0u;  // keys past the length: no gradient
+          }
+          uint32_t w[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e)
+            w[e] = pack_bf16x2(__uint_as_float(r[2 * e]) * mult, __uint_as_float(r[2 * e + 1]) * mult);
+          uint4 *d4 = reinterpret_cast<uint4 *>(dst + 32 * c);
+          if (row_ok) {
+#pragma unroll
+            for (int v4 = 0; v4 < 4; ++v4)
+              d4[v4] = make_uint4(w[4 * v4], w[4 * v4 + 1], w[4 * v4 + 2], w[4 * v4 + 3]);
+          }
+        }
+      }
+    }
+  }
+  __syncwarp();
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// dQ
+// ---------------------------------------------------------------------------
+template <int D>
+__global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
+    fa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q,
+                     const __grid_constant__ CUtensorMap tm_k,
+                     const __grid_constant__ CUtensorMap tm_v,
+                     const __grid_constant__ CUtensorMap tm_do, const BwdParams p) {
+  using C = BwdCfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  uint8_t *smem = smem_raw + (base - raw);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  // Unit: (query tile, batch, head); causal units with the most key tiles
+  // (the last query tiles) first.
+  const int BH = p.B * p.Hq;
+  const int qt = p.q_tiles - 1 - static_cast<int>(blockIdx.x) / BH;
+  const int bh = static_cast<int>(blockIdx.x) % BH;
+  const int b = bh / p.Hq, h = bh % p.Hq, hkv = h / p.group;
+  const int bkv = b * p.Hkv + hkv;
+  int L = p.N;
+  if (p.seqlens) L = min(max(p.seqlens[b], 0), p.N);
+  const int row0 = qt * 128;
+  const int kv_end = p.causal ? min(L, row0 + 128) : L;
+  const int nkv = (kv_end + 127) / 128;
+
+  const uint32_t bar_q = base + C::OFF_BAR_Q;
+  const uint32_t bar_full = bar_q + 8;
+  const uint32_t bar_empty = bar_full + 8 * C::Q_STAGES;
+  const uint32_t bar_sd = bar_empty + 8 * C::Q_STAGES;  // S and dP in TMEM
+  const uint32_t bar_ds = bar_sd + 8;                    // dS in TMEM
+  const uint32_t bar_done = bar_ds + 8;
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + C::OFF_BAR_Q + 120);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + C::OFF_BAR_Q + 124);
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar_q, 1);
+    for (int s = 0; s < C::Q_STAGES; ++s) {
+      mbar_init(bar_full + 8 * s, 1);
+      mbar_init(bar_empty + 8 * s, 1);
+    }
+    mbar_init(bar_sd, 1);
+    mbar_init(bar_ds, 128);
+    mbar_init(bar_done, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(smem_u32(tmem_slot), 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *reinterpret_cast<volatile uint32_t *>(tmem_slot);
+
+  if (nkv > 0 && warp == 4) {
+    if (lane == 0) {
+      mbar_arrive_expect_tx(bar_q, 2 * C::TILE_BYTES);
+      load_tile<D>(base + C::OFF_Q, &tm_q, bar_q, row0, bh);
+      load_tile<D>(base + C::OFF_DO, &tm_do, bar_q, row0, bh);
+      int j = 0;
+      for (; j < nkv; ++j) {
+        const int st = j % C::Q_STAGES;
+        if (!mbar_wait_bounded(bar_empty + 8 * st, ((j / C::Q_STAGES) & 1) ^ 1, abort_flag,
+                               p.status, p.wait_limit_ns, kErrTimeout))
+          break;
+        const uint32_t dst = base + C::OFF_KVRING + st * C::KVSTAGE_BYTES;
+        mbar_arrive_expect_tx(bar_full + 8 * st, 2 * C::TILE_BYTES);
+        load_tile<D>(dst, &tm_k, bar_full + 8 * st, j * 128, bkv);
+        load_tile<D>(dst + C::TILE_BYTES, &tm_v, bar_full + 8 * st, j * 128, bkv);
+      }
+      volatile int never = 0;
+      mbar_wait_bounded(bar_q, 0, &never, p.status, p.wait_limit_ns, kErrTimeout);
+      for (int st = 0; st < C::Q_STAGES && st < j; ++st) {
+        const int last = st + C::Q_STAGES * ((j - 1 - st) / C::Q_STAGES);
+        mbar_wait_bounded(bar_full + 8 * st, (last / C::Q_STAGES) & 1, &never, p.status,
+                          p.wait_limit_ns, kErrTimeout);
+      }
+    }
+  } else if (nkv > 0 && warp == 5) {
+    const bool leader = elect_one();
+    constexpr uint32_t IDESC_SS = idesc_bf16_f32(128, 128, 0, 0);
+    constexpr uint32_t IDESC_TS = idesc_bf16_f32(128, D, 0, 1);
+    const uint64_t dQk = smem_desc_sw128(base + C::OFF_Q, 16, 1024);
+    const uint64_t dOk = smem_desc_sw128(base + C::OFF_DO, 16, 1024);
+    auto wait = [&](uint32_t bar, uint32_t par) {
+      const bool ok = mbar_wait_bounded(bar, par, abort_flag, p.status, p.wait_limit_ns,
+                                        kErrTimeout);
+      return __all_sync(0xffffffffu, ok);
+    };
+    auto commit = [&](uint32_t bar) {
+      if (leader) tc_commit(bar);
+      __syncwarp();
+    };
+    if (wait(bar_q, 0)) {
+      for (int j = 0; j < nkv; ++j) {
+        const int st = j % C::Q_STAGES;
+        if (!wait(bar_full + 8 * st, (j / C::Q_STAGES) & 1)) break;
+        tc_fence_after();
+        const uint32_t stage = base + C::OFF_KVRING + st * C::KVSTAGE_BYTES;
+        const uint64_t dKk = smem_desc_sw128(stage, 16, 1024);
+        const uint64_t dVk = smem_desc_sw128(stage + C::TILE_BYTES, 16, 1024);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = ((kk / 4) * C::HALF_BYTES + (kk % 4) * 32) >> 4;
+          if (leader) tc_mma_ss(tmem + C::COL_A, dQk + off, dKk + off, IDESC_SS, kk > 0);
+        }
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = ((kk / 4) * C::HALF_BYTES + (kk % 4) * 32) >> 4;
+          if (leader) tc_mma_ss(tmem + C::COL_B, dOk + off, dVk + off, IDESC_SS, kk > 0);
+        }
+        __syncwarp();
+        commit(bar_sd);
+        if (!wait(bar_ds, j & 1)) break;
+        tc_fence_after();
+        // dQ += dS K: K = 128 keys in steps of 16, K read MN-major.
+        const uint64_t dKm = smem_desc_sw128(stage, C::HALF_BYTES, 1024);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          if (leader)
+            tc_mma_ts(tmem + C::COL_C, tmem + C::COL_A + kk * 8, dKm + ((kk * 2048) >> 4),
+                      IDESC_TS, (j > 0 || kk > 0) ? 1u : 0u);
+        __syncwarp();
+        commit(bar_empty + 8 * st);
+      }
+    }
+    commit(bar_done);
+    volatile int never = 0;
+    mbar_wait_bounded(bar_done, 0, &never, p.status, p.wait_limit_ns, kErrTimeout);
+  } else if (warp < 4) {
+    const int i = row0 + threadIdx.x;
+    const uint32_t lane_base = static_cast<uint32_t>(warp) * 32u << 16;
+    const uint32_t tA = tmem + lane_base + C::COL_A, tB = tmem + lane_base + C::COL_B;
+    const size_t vrow = static_cast<size_t>(bh) * p.Npad + i;
+    const float lse2 = p.ws_lse2[vrow];
+    const float delta = p.ws_delta[vrow];
+    const int limit = p.causal ? min(L, i + 1) : L;
+    bool ok = true;
+    for (int j = 0; j < nkv && ok; ++j) {
+      const bool got = mbar_wait_bounded(bar_sd, j & 1, abort_flag, p.status, p.wait_limit_ns,
+                                         kErrTimeout);
+      if (!__all_sync(0xffffffffu, got)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+        uint32_t sv[64], dp[64];
+        tmem_ld32(tA + 64 * half, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
+        tmem_ld32(tA + 64 * half + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
+        tmem_ld32(tB + 64 * half, *reinterpret_cast<uint32_t(*)[32]>(&dp[0]));
+        tmem_ld32(tB + 64 * half + 32, *reinterpret_cast<uint32_t(*)[32]>(&dp[32]));
+        tmem_wait_ld();
+        uint32_t dk[32];
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+          float dv[2];
+#pragma unroll
+          for (int u = 0; u < 2; ++u) {
+            const int key = j * 128 + 64 * half + 2 * e + u;
+            const float pp = key < limit ? ex2_approx(fmaf(__uint_as_float(sv[2 * e + u]),
+                                                           p.scale_log2, -lse2))
+                                         : 0.f;
+            dv[u] = pp * (__uint_as_float(dp[2 * e + u]) - delta);
+          }
+          dk[e] = pack_bf16x2(dv[0], dv[1]);
+        }
+        tmem_st32(tA + 32 * half, dk);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(bar_ds);
+    }
+    if (ok && nkv > 0) {
+      const bool got = mbar_wait_bounded(bar_done, 0, abort_flag, p.status, p.wait_limit_ns,
+                                         kErrTimeout);
+      ok = __all_sync(0xffffffffu, got);
+    }
+    // Warp-collective TMEM loads on every lane; stores only for real rows.
+    if (ok) {
+      const bool row_ok = i < p.N;
+      uint16_t *dst = p.dq + (static_cast<size_t>(bh) * p.N + (row_ok ? i : 0)) * D;
+      if (nkv > 0) tc_fence_after();
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t r[32];
+        if (nkv > 0) {
+          tmem_ld32(tmem + lane_base + C::COL_C + 32 * c, r);
+          tmem_wait_ld();
+        } else {
+#pragma unroll
+          for (int e = 0; e < 32; ++e) r[e] = 0u;
+        }
+        uint32_t w[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e)
+          w[e] = pack_bf16x2(__uint_as_float(r[2 * e]) * p.scale,
+                             __uint_as_float(r[2 * e + 1]) * p.scale);
+        uint4 *d4 = reinterpret_cast<uint4 *>(dst + 32 * c);
+        if (row_ok) {
+#pragma unroll
+          for (int v4 = 0; v4 < 4; ++v4)
+            d4[v4] = make_uint4(w[4 * v4], w[4 * v4 + 1], w[4 * v4 + 2], w[4 * v4 + 3]);
+        }
+      }
+    }
+  }
+  __syncwarp();
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+}  // namespace fa

@@ -130,6 +130,27 @@ FA_API int fa_fwd_hostio(const void *q_h, const void *k_h, const void *v_h, void
                   void *stream);
 
 /*
+ * Attention backward by recomputation: the gradients of sum(dout * O) for
+ * O = fa_fwd(q, k, v, ...), rebuilt from q, k, v, o, dout and the forward's
+ * LSE without any stored probability matrix (interview notes "Why is
+ * FlashAttention faster", section on memory: training stores less by
+ * recomputing; exam explainer, "recomputation").
+ *  q, o, dout, dq : [B, Hq, N, d] bf16     k, v, dk, dv : [B, Hkv, N, d] bf16
+ *  lse : [B, Hq, N] fp32 from the forward with the same arguments.
+ *  dk, dv sum over the query heads that share each kv head.  causal and
+ *  seqlens as in fa_fwd.  d in {64, 128}.
+ *  workspace: DEVICE buffer of at least fa_bwd_workspace_size(B, Hq, N)
+ *  bytes, 16-byte aligned (per-row D = rowsum(dout * o) and LSE*log2(e)).
+ * Three kernels run on `stream`: the per-row preprocess, the dK/dV kernel
+ * (one CTA per 128-key tile) and the dQ kernel (one CTA per 128-row tile).
+ */
+FA_API size_t fa_bwd_workspace_size(int B, int Hq, int N);
+FA_API int fa_bwd(const void *q, const void *k, const void *v, const void *o, const void *dout,
+                  const float *lse, void *dq, void *dk, void *dv, int B, int Hq, int Hkv, int N,
+                  int d, float scale, int causal, const int *seqlens, void *workspace,
+                  size_t workspace_bytes, void *stream, int *status_dev);
+
+/*
  * Packed variable-length forward: the tokens of B sequences are stored back
  * to back with no padding (the padding mask of the pages' statement, without
  * padded rows).  Same operation as fa_fwd per sequence, self-attention
