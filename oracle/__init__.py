@@ -18,7 +18,9 @@ import numpy as np
 
 from . import build as _build
 
-_IN_KIND = {np.dtype(np.float64): 0, np.dtype(np.float32): 1, np.dtype(np.uint16): 2}
+# element encodings: fp64, fp32, bf16 bit patterns (uint16), FP8 E4M3 codes (uint8)
+_IN_KIND = {np.dtype(np.float64): 0, np.dtype(np.float32): 1, np.dtype(np.uint16): 2,
+            np.dtype(np.uint8): 3}
 _lib = None
 
 
@@ -68,8 +70,8 @@ def attention_forward(q, k, v, *, causal: bool, scale: float, seqlens=None, rows
                       causal_bottom_right: bool = False, _lib_override=None):
     """Exact softmax attention in fp64.
 
-    q: [B, Hq, Nq, d]; k, v: [B, Hkv, Nk, d]; dtype float64, float32 or uint16
-    (bf16 bit patterns).  seqlens: int [B] key lengths or None.  rows: int
+    q: [B, Hq, Nq, d]; k, v: [B, Hkv, Nk, d]; dtype float64, float32, uint16
+    (bf16 bit patterns) or uint8 (FP8 E4M3 codes).  seqlens: int [B] key lengths or None.  rows: int
     [B*Hq, R] query rows per (batch, head) or None for all rows.
     causal_bottom_right: with causal, query i sits at position len_b - Nq + i
     (key j visible iff j <= i + len_b - Nq); otherwise causal is top-left.
@@ -81,7 +83,8 @@ def attention_forward(q, k, v, *, causal: bool, scale: float, seqlens=None, rows
     k = np.ascontiguousarray(k)
     v = np.ascontiguousarray(v)
     if not (q.dtype == k.dtype == v.dtype) or q.dtype not in _IN_KIND:
-        raise TypeError("q, k, v must share one dtype among float64, float32, uint16(bf16)")
+        raise TypeError("q, k, v must share one dtype among float64, float32, uint16(bf16), "
+                        "uint8(e4m3)")
     B, Hq, Nq, d = q.shape
     Bk, Hkv, Nk, dk = k.shape
     if (Bk, dk) != (B, d) or v.shape != k.shape:

@@ -59,14 +59,33 @@
 #include <stdlib.h>
 #include <string.h>
 
-enum { ORACLE_IN_F64 = 0, ORACLE_IN_F32 = 1, ORACLE_IN_BF16 = 2 };
+enum { ORACLE_IN_F64 = 0, ORACLE_IN_F32 = 1, ORACLE_IN_BF16 = 2, ORACLE_IN_E4M3 = 3 };
 
 #define ORACLE_ROW_BLOCK 16
 
-/* Decode one input element to fp64.  bf16 and fp32 values widen exactly. */
+/*
+ * One FP8 E4M3 code (the OCP 8-bit format with 4 exponent bits, bias 7, 3
+ * mantissa bits, no infinities; S.1111.111 is NaN): normal values
+ * (1 + m/8) * 2^(e-7), subnormals (e = 0) m * 2^-9.  Every code is exact in
+ * fp64.
+ */
+static double e4m3_value(uint8_t c) {
+  const int s = c >> 7, e = (c >> 3) & 15, m = c & 7;
+  double x;
+  if (e == 15 && m == 7)
+    x = NAN;
+  else if (e == 0)
+    x = ldexp((double)m, -9);
+  else
+    x = ldexp(1.0 + m / 8.0, e - 7);
+  return s ? -x : x;
+}
+
+/* Decode one input element to fp64.  bf16, fp32 and e4m3 values widen exactly. */
 static double in_at(const void *base, int kind, int64_t idx) {
   if (kind == ORACLE_IN_F64) return ((const double *)base)[idx];
   if (kind == ORACLE_IN_F32) return (double)((const float *)base)[idx];
+  if (kind == ORACLE_IN_E4M3) return e4m3_value(((const uint8_t *)base)[idx]);
   uint32_t u = (uint32_t)((const uint16_t *)base)[idx] << 16;
   float f;
   memcpy(&f, &u, sizeof f);
@@ -187,7 +206,7 @@ int oracle_attention_fwd_general(const void *q, const void *k, const void *v, in
   if (B <= 0 || Hq <= 0 || Hkv <= 0 || Nq <= 0 || Nk <= 0 || d <= 0 || R <= 0) return -1;
   if (Hq % Hkv != 0) return -1;
   if (!rows && R != Nq) return -1;
-  if (in_kind < ORACLE_IN_F64 || in_kind > ORACLE_IN_BF16) return -1;
+  if (in_kind < ORACLE_IN_F64 || in_kind > ORACLE_IN_E4M3) return -1;
   job_t J;
   memset(&J, 0, sizeof J);
   J.q = q; J.k = k; J.v = v; J.in_kind = in_kind;
@@ -322,7 +341,7 @@ int oracle_attention_bwd(const void *q, const void *k, const void *v, const void
                          int nthreads) {
   if (!q || !k || !v || !dout || !dq || !dk || !dv) return -1;
   if (B <= 0 || Hq <= 0 || Hkv <= 0 || N <= 0 || d <= 0 || Hq % Hkv != 0) return -1;
-  if (in_kind < ORACLE_IN_F64 || in_kind > ORACLE_IN_BF16) return -1;
+  if (in_kind < ORACLE_IN_F64 || in_kind > ORACLE_IN_E4M3) return -1;
   bwd_job_t J;
   memset(&J, 0, sizeof J);
   J.q = q; J.k = k; J.v = v; J.dout = dout; J.in_kind = in_kind;

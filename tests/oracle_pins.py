@@ -264,6 +264,43 @@ def pin_input_encodings_agree(fwd):
         np.testing.assert_array_equal(l, res[0][1])
 
 
+def pin_e4m3_codes(fwd):
+    """FP8 E4M3 inputs (uint8 codes).  Through V: one visible key makes
+    O = V_0, so O shows the decoded value of every non-NaN code, which must
+    equal torch's float8_e4m3fn widening and, for a few codes, the values
+    worked out by hand from the format (bias 7, 3 mantissa bits, subnormals
+    m * 2^-9).  Through Q: one key of value 1 makes LSE = scale * q."""
+    import torch
+    codes = np.arange(256, dtype=np.uint8)
+    codes = codes[(codes & 0x7F) != 0x7F]  # S.1111.111 is NaN
+    n = codes.size
+    zeros = np.zeros((1, 1, 1, n), np.uint8)
+    o, _ = fwd(zeros, zeros, codes.reshape(1, 1, 1, n), causal=False, scale=1.0)
+    lib = torch.from_numpy(codes.copy()).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    np.testing.assert_array_equal(o.ravel(), lib)
+    by_hand = {0x00: 0.0, 0x38: 1.0, 0xB8: -1.0, 0x7E: 448.0, 0x01: 2.0 ** -9,
+               0x07: 7 * 2.0 ** -9, 0x08: 2.0 ** -6, 0x3C: 1.5, 0x40: 2.0, 0x46: 3.5, 0x4B: 5.5}
+    for c, val in by_hand.items():
+        assert o.ravel()[list(codes).index(c)] == val, hex(c)
+    one = np.full((1, 1, 1, 1), 0x38, np.uint8)
+    q = codes.reshape(1, 1, n, 1)
+    _, lse = fwd(q, one, one, causal=False, scale=0.5)
+    np.testing.assert_array_equal(lse.ravel(), 0.5 * lib)
+
+
+def pin_e4m3_matches_decoded_fp64(fwd):
+    """Attention on E4M3 codes equals attention on their values in fp64."""
+    import torch
+    rng = np.random.default_rng(57)
+    codes = rng.integers(0, 256, size=(3, 2, 1, 20, 16), dtype=np.uint8)
+    codes[(codes & 0x7F) == 0x7F] = 0x30  # no NaN codes
+    vals = torch.from_numpy(codes).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    a = fwd(codes[0], codes[1][:, :1], codes[2][:, :1], causal=True, scale=0.01)
+    b = fwd(vals[0], vals[1][:, :1], vals[2][:, :1], causal=True, scale=0.01)
+    np.testing.assert_array_equal(a[0], b[0])
+    np.testing.assert_array_equal(a[1], b[1])
+
+
 def pin_cross_length_matches_torch_sdpa(fwd):
     """Nq query rows against Nk keys (the decode shape), causal aligned to the
     end of each sequence's keys, against torch SDPA in fp64 with the same
@@ -412,4 +449,5 @@ ALL_PINS = [
     pin_key_permutation_invariance, pin_linear_in_v, pin_shift_invariance,
     pin_fully_masked_row, pin_row_subset, pin_input_encodings_agree,
     pin_cross_length_matches_torch_sdpa, pin_single_query_is_last_causal_row,
+    pin_e4m3_codes, pin_e4m3_matches_decoded_fp64,
 ]

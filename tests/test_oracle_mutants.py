@@ -43,6 +43,8 @@ MUTANTS = {
     "bwd_dq_from_v": ("dqrow[c] += J->scale * ds * in_at(J->k,", "dqrow[c] += J->scale * ds * in_at(J->v,"),
     "bwd_causal_off_by_one": ("(j < len) && (!J->causal || j <= i);",
                               "(j < len) && (!J->causal || j < i);"),
+    "e4m3_bias_off_by_one": ("ldexp(1.0 + m / 8.0, e - 7)", "ldexp(1.0 + m / 8.0, e - 8)"),
+    "e4m3_subnormal_scale": ("ldexp((double)m, -9)", "ldexp((double)m, -10)"),
     "masked_row_not_zeroed": ("for (int j = 0; j < N; ++j) Srow[j] = 0.0;",
                               "for (int j = 0; j < N; ++j) Srow[j] = 1.0 / N;"),
 }
