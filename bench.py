@@ -364,6 +364,44 @@ def report_all_workloads(args):
     report_varlen(args, dev)
     report_decode(args, dev)
     report_backward(args, dev)
+    report_fp8(args, dev)
+
+
+def report_fp8(args, dev):
+    """The FP8 E4M3 forward (fa_fwd_fp8) on the GQA workload; FLOPs counted
+    as for the bf16 forward, against the measured bf16 peak and twice it
+    (the nominal FP8:bf16 dense ratio)."""
+    import torch
+    from exact_io_aware_92_b200 import attention
+    peaks, src = load_peaks()
+    w = wl.LLAMA_GQA_FP8
+    inp = wl.draw_fp8_workload(w)
+    q, k = torch.from_numpy(inp.q).to(dev), torch.from_numpy(inp.k).to(dev)
+    vt = torch.from_numpy(inp.vt()).to(dev)
+    o = torch.empty((w.B, w.Hq, w.N, w.d), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((w.B, w.Hq, w.N), dtype=torch.float32, device=dev)
+    kw = dict(descale_q=inp.descale_q, descale_k=inp.descale_k, descale_v=inp.descale_v,
+              causal=w.causal, scale=w.scale, out=o, lse=lse)
+    flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
+    for _ in range(args.warmup):
+        attention.fwd_fp8(q, k, vt, **kw)
+    torch.cuda.synchronize(dev)
+    times = []
+    for _ in range(args.steps):
+        flush.zero_()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        attention.fwd_fp8(q, k, vt, **kw)
+        e1.record()
+        e1.synchronize()
+        times.append(e0.elapsed_time(e1))
+    ms = statistics.median(times)
+    f = wl.flops(w)
+    tf = f / ms / 1e9
+    print(json.dumps({"workload": w.name, "ms_median": ms, "tflops": tf,
+                      "frac_of_bf16_peak": tf / float(peaks["bf16_tflops"]),
+                      "frac_of_fp8_peak_2x_bf16": tf / (2 * float(peaks["bf16_tflops"])),
+                      "flops": f, "l2": "flushed between steps", "peak_source": src}), flush=True)
 
 
 def report_backward(args, dev):

@@ -1,5 +1,5 @@
-"""Exact, IO-aware attention for B200 (sm_100a): forward, backward, packed
-variable-length and split-KV decode.
+"""Exact, IO-aware attention for B200 (sm_100a): forward (bf16 and FP8),
+backward, packed variable-length and split-KV decode.
 
 The computation lives in hand-written CUDA kernels behind the C ABI of
 ``include/fa.h`` (``libfa_b200.so``); this package holds the ctypes binding
@@ -8,7 +8,7 @@ inputs (``workloads``).
 """
 from . import workloads  # noqa: F401
 
-_API = ("fwd", "bwd", "fwd_varlen", "fwd_decode", "decode_workspace_size", "bwd_workspace_size",
+_API = ("fwd", "bwd", "fwd_fp8", "fwd_varlen", "fwd_decode", "decode_workspace_size", "bwd_workspace_size",
         "check_status", "fwd_hostio")
 __all__ = list(_API) + ["workloads"]
 

@@ -1,5 +1,5 @@
 """Python entry points over the C ABI.  Argument marshalling only: every step
-of the attention forward runs in the CUDA kernels of libfa_b200.so.
+of the attention runs in the CUDA kernels of libfa_b200.so.
 
 PyTorch provides device memory and the current stream; nothing here computes.
 """
@@ -58,6 +58,48 @@ def fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *, causal: bool = Fal
                                dtype, _stream_handle(q.device),
                                None if status is None else status.data_ptr())
     _lib.check(rc, "fa_fwd_ex")
+    return out, lse
+
+
+def _codes(t: torch.Tensor, name: str) -> torch.Tensor:
+    if not t.is_cuda or t.dtype not in (torch.uint8, torch.float8_e4m3fn) or t.dim() != 4 \
+            or not t.is_contiguous():
+        raise ValueError(f"{name} must be a contiguous 4-D uint8 / float8_e4m3fn CUDA tensor")
+    return t
+
+
+def fwd_fp8(q: torch.Tensor, k: torch.Tensor, vt: torch.Tensor, *, descale_q: float,
+            descale_k: float, descale_v: float, causal: bool = False,
+            scale: float | None = None, seqlens: torch.Tensor | None = None,
+            out: torch.Tensor | None = None, lse: torch.Tensor | None = None,
+            status: torch.Tensor | None = None):
+    """Attention forward on FP8 E4M3 codes with per-tensor descales (value =
+    code * descale).  q: [B, Hq, N, 128], k: [B, Hkv, N, 128], vt: V
+    transposed [B, Hkv, 128, ldvt] (ldvt >= N, a multiple of 16); uint8 or
+    float8_e4m3fn, contiguous.  Returns (o bf16 [B, Hq, N, 128], lse fp32
+    [B, Hq, N])."""
+    q, k, vt = _codes(q, "q"), _codes(k, "k"), _codes(vt, "vt")
+    B, Hq, N, d = q.shape
+    Hkv = k.shape[1]
+    if k.shape != (B, Hkv, N, d) or vt.shape[:3] != (B, Hkv, d):
+        raise ValueError("k must be [B, Hkv, N, d] and vt [B, Hkv, d, ldvt]")
+    ldvt = vt.shape[3]
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    if out is None:
+        out = torch.empty((B, Hq, N, d), dtype=torch.bfloat16, device=q.device)
+    if lse is None:
+        lse = torch.empty((B, Hq, N), dtype=torch.float32, device=q.device)
+    sl_ptr = None
+    if seqlens is not None:
+        if seqlens.dtype != torch.int32 or seqlens.device != q.device or seqlens.numel() != B:
+            raise ValueError("seqlens must be int32 [B] on q's device")
+        sl_ptr = seqlens.data_ptr()
+    rc = _lib.load().fa_fwd_fp8(q.data_ptr(), k.data_ptr(), vt.data_ptr(), out.data_ptr(),
+                                lse.data_ptr(), B, Hq, Hkv, N, ldvt, d, scale, float(descale_q),
+                                float(descale_k), float(descale_v), int(bool(causal)), sl_ptr,
+                                _stream_handle(q.device),
+                                None if status is None else status.data_ptr())
+    _lib.check(rc, "fa_fwd_fp8")
     return out, lse
 
 

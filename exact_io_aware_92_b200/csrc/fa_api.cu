@@ -36,6 +36,7 @@ struct DeviceState {
   bool attr64 = false, attr128 = false;
   bool dec_attr64 = false, dec_attr128 = false;
   bool bwd_attr64 = false, bwd_attr128 = false;
+  bool fp8_attr = false;
 };
 DeviceState g_dev[kMaxDevices];
 std::mutex g_mu;
@@ -138,6 +139,71 @@ int make_map_packed(CUtensorMap *m, const void *ptr, int total, int H, int d) {
   return r == CUDA_SUCCESS ? FA_OK : FA_ERR_CUDA;
 }
 
+// 8-bit map over a [planes, rows, cols] tensor of E4M3 codes whose rows are
+// `pitch` bytes apart: box = 128 columns x 128 rows x 1 plane, 128-byte
+// swizzle; columns past `cols` and rows past `rows` read as zero.  Q and K:
+// rows = N, cols = pitch = d.  V^T: rows = d, cols = N keys, pitch = ldvt.
+int make_map_u8(CUtensorMap *m, const void *ptr, int planes, int rows, int cols, int pitch) {
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows),
+                        static_cast<cuuint64_t>(planes)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(pitch),
+                           static_cast<cuuint64_t>(rows) * static_cast<cuuint64_t>(pitch)};
+  cuuint32_t box[3] = {128, 128, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void *>(ptr), dims,
+                        strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? FA_OK : FA_ERR_CUDA;
+}
+
+int launch_fp8(DeviceState *ds, const void *q, const void *k, const void *vt, void *o, float *lse,
+               int B, int Hq, int Hkv, int N, int ldvt, float scale, float descale_q,
+               float descale_k, float descale_v, int causal, const int *seqlens,
+               cudaStream_t stream, int *status) {
+  using C = fa::Sm100Cfg<128, true>;
+  auto kernel = fa::fa_fwd_e4m3_sm100_kernel;
+  if (!ds->fp8_attr) {
+    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             C::SMEM_ALLOC) != cudaSuccess) {
+      cudaGetLastError();
+      return FA_ERR_LAUNCH;
+    }
+    ds->fp8_attr = true;
+  }
+  CUtensorMap tq, tk, tvt;
+  if (make_map_u8(&tq, q, B * Hq, N, 128, 128) != FA_OK ||
+      make_map_u8(&tk, k, B * Hkv, N, 128, 128) != FA_OK ||
+      make_map_u8(&tvt, vt, B * Hkv, 128, N, ldvt) != FA_OK)
+    return FA_ERR_CUDA;
+  fa::FwdParams p;
+  p.o = static_cast<uint16_t *>(o);
+  p.lse = lse;
+  p.seqlens = seqlens;
+  p.cu_seqlens = nullptr;
+  p.total = 0;
+  p.status = status;
+  p.B = B;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.N = N;
+  p.group = Hq / Hkv;
+  p.num_qpairs = (N + C::ROWS_PER_UNIT - 1) / C::ROWS_PER_UNIT;
+  p.causal = causal ? 1 : 0;
+  // scores of the codes times the two descales, in log2 units
+  p.scale_log2 = static_cast<float>(static_cast<double>(scale) * descale_q * descale_k *
+                                    1.4426950408889634);
+  p.out_scale = descale_v;
+  p.wait_limit_ns = kWaitLimitNs;
+  const long long units = static_cast<long long>(B) * Hq * p.num_qpairs;
+  if (units > 0x7fffffffll) return FA_ERR_SHAPE;
+  p.num_units = static_cast<int>(units);
+  const int grid = static_cast<int>(units < ds->num_sms ? units : ds->num_sms);
+  kernel<<<grid, C::THREADS, C::SMEM_ALLOC, stream>>>(tq, tk, tvt, p);
+  if (cudaGetLastError() != cudaSuccess) return FA_ERR_LAUNCH;
+  return FA_OK;
+}
+
 template <int D>
 int launch_bf16(DeviceState *ds, const void *q, const void *k, const void *v, void *o,
                 float *lse, int B, int Hq, int Hkv, int N, float scale, int causal,
@@ -179,6 +245,7 @@ int launch_bf16(DeviceState *ds, const void *q, const void *k, const void *v, vo
   p.num_qpairs = (N + C::ROWS_PER_UNIT - 1) / C::ROWS_PER_UNIT;
   p.causal = causal ? 1 : 0;
   p.scale_log2 = scale * kLog2e;
+  p.out_scale = 1.0f;
   p.wait_limit_ns = kWaitLimitNs;
   const long long units = static_cast<long long>(B) * Hq * p.num_qpairs;
   if (units > 0x7fffffffll) return FA_ERR_SHAPE;
@@ -525,6 +592,24 @@ int fa_fwd_varlen(const void *q, const void *k, const void *v, void *o, float *l
                                    nullptr, st, status, cu_seqlens, total)
                  : launch_bf16<128>(ds, q, k, v, o, lse, B, Hq, Hkv, max_seqlen, scale, causal,
                                     nullptr, st, status, cu_seqlens, total);
+}
+
+int fa_fwd_fp8(const void *q, const void *k, const void *vt, void *o, float *lse, int B, int Hq,
+               int Hkv, int N, int ldvt, int d, float scale, float descale_q, float descale_k,
+               float descale_v, int causal, const int *seqlens, void *stream, int *status_dev) {
+  int rc = check_args(q, k, vt, o, lse, B, Hq, Hkv, N, d, scale);
+  if (rc != FA_OK) return rc;
+  if (d != 128) return FA_ERR_HEADDIM;
+  for (float f : {descale_q, descale_k, descale_v})
+    if (!(std::isfinite(f) && f > 0.f)) return FA_ERR_SHAPE;
+  if (ldvt < N) return FA_ERR_SHAPE;
+  if (ldvt % 16 != 0) return FA_ERR_ALIGN;
+  DeviceState *ds = nullptr;
+  rc = current_device(&ds);
+  if (rc != FA_OK) return rc;
+  int *status = status_dev ? status_dev : ds->status_word;
+  return launch_fp8(ds, q, k, vt, o, lse, B, Hq, Hkv, N, ldvt, scale, descale_q, descale_k,
+                    descale_v, causal, seqlens, static_cast<cudaStream_t>(stream), status);
 }
 
 size_t fa_bwd_workspace_size(int B, int Hq, int N) {

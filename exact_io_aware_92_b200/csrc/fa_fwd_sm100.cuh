@@ -50,19 +50,28 @@ struct FwdParams {
   int num_qpairs;        // ceil(N / 256)
   int num_units;         // B * Hq * num_qpairs
   int causal;
-  float scale_log2;      // scale * log2(e)
+  float scale_log2;      // scale * log2(e) (times the Q and K descales for FP8 inputs)
+  float out_scale;       // FP8 inputs: the V descale, applied with 1/l; 1 otherwise
   unsigned long long wait_limit_ns;
 };
 
-template <int D>
+// F8: Q, K and V are FP8 E4M3 codes (head dim 128 only) and V arrives
+// transposed ([d, keys], keys contiguous), so both products read K-major
+// operands; otherwise bf16.
+template <int D, bool F8 = false>
 struct Sm100Cfg {
   static_assert(D == 64 || D == 128, "head dim 64 or 128");
+  static_assert(!F8 || D == 128, "FP8 inputs: head dim 128");
+  static constexpr int EB = F8 ? 1 : 2;           // bytes per input element
   static constexpr int BM = 128;                  // query rows per Q tile
   static constexpr int BN = 128;                  // keys per K/V tile
   static constexpr int ROWS_PER_UNIT = 2 * BM;
-  static constexpr int HALF_BYTES = 128 * 64 * 2; // one TMA box: 128 rows x 64 bf16
-  static constexpr int TILE_BYTES = 128 * D * 2;  // one Q, K or V tile
-  static constexpr int STAGES = (D == 128) ? 4 : 8;
+  static constexpr int BOX_BYTES = 128 * 128;     // one TMA box: 128 rows x 128 bytes
+  static constexpr int BOX_COLS = 128 / EB;       // elements in a box row
+  static constexpr int TILE_BYTES = 128 * D * EB; // one Q, K or V tile
+  static constexpr int NBOX = TILE_BYTES / BOX_BYTES;
+  static constexpr int KSTEPS = D * EB / 32;      // 32-byte K steps of the S product
+  static constexpr int STAGES = (TILE_BYTES == 32768) ? 4 : 8;
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_KV = OFF_Q + 2 * TILE_BYTES;
   static constexpr int OFF_BAR = OFF_KV + STAGES * TILE_BYTES;
@@ -87,7 +96,13 @@ struct Sm100Cfg {
   static constexpr uint32_t REGS_SOFTMAX = 224;
   static constexpr uint32_t TMEM_COLS = 512;
   static constexpr uint32_t COL_S0 = 0, COL_O0 = 256;
-  static constexpr float RESCALE_THRESHOLD = 8.0f;         // log2 units
+  // The reference max moves when the row max grows by more than this (log2
+  // units).  FP8: P is stored as E4M3 (largest finite 448) and carries a
+  // factor 2^P_SHIFT that keeps small probabilities out of the subnormal
+  // range, so P <= 2^(threshold + shift) = 256 must hold.
+  static constexpr float RESCALE_THRESHOLD = F8 ? 4.0f : 8.0f;
+  static constexpr float P_SHIFT = F8 ? 4.0f : 0.0f;
+  static constexpr int PK_WORDS = F8 ? 16 : 32;   // 32-bit words of P per 64 keys
   // Of every 8 consecutive pairs of probabilities, this many are computed on
   // the FMA pipe (exp2_poly_pair) instead of the MUFU pipe.  At d = 128 the
   // exponentials alone keep the MUFU pipe as busy as the MMAs keep the
@@ -115,9 +130,9 @@ struct Unit {
   size_t lse_base; // offset of row 0 in LSE
 };
 
-template <int D>
+template <int D, bool F8>
 __device__ __forceinline__ Unit unit_at(const FwdParams &p, int u) {
-  using C = Sm100Cfg<D>;
+  using C = Sm100Cfg<D, F8>;
   Unit x;
   const int BH = p.B * p.Hq;
   const int qp = p.num_qpairs - 1 - u / BH;
@@ -164,9 +179,9 @@ __device__ __forceinline__ int snake_unit(int k, int num_units) {
   return u < num_units ? u : -1;
 }
 
-template <int D>
+template <int D, bool F8>
 struct Sm100Ctx {
-  using C = Sm100Cfg<D>;
+  using C = Sm100Cfg<D, F8>;
   uint32_t smem;      // 1 KB aligned shared base (shared-window address)
   uint32_t tmem;      // tensor-memory base address
   volatile int *abort_flag;
@@ -177,20 +192,20 @@ struct Sm100Ctx {
 };
 
 // Ring position of K tile g (V tile g is the next one) in a CTA's stream.
-template <int D>
-__device__ __forceinline__ int ring_slot(int seq) { return seq % Sm100Cfg<D>::STAGES; }
-template <int D>
+template <int D, bool F8>
+__device__ __forceinline__ int ring_slot(int seq) { return seq % Sm100Cfg<D, F8>::STAGES; }
+template <int D, bool F8>
 __device__ __forceinline__ uint32_t ring_parity(int seq) {
-  return static_cast<uint32_t>((seq / Sm100Cfg<D>::STAGES) & 1);
+  return static_cast<uint32_t>((seq / Sm100Cfg<D, F8>::STAGES) & 1);
 }
 
 // --------------------------------------------------------------------------
 // TMA producer (one thread)
 // --------------------------------------------------------------------------
-template <int D>
-__device__ void role_producer(const Sm100Ctx<D> &x, const FwdParams &p, const CUtensorMap *tm_q,
+template <int D, bool F8>
+__device__ void role_producer(const Sm100Ctx<D, F8> &x, const FwdParams &p, const CUtensorMap *tm_q,
                               const CUtensorMap *tm_k, const CUtensorMap *tm_v) {
-  using C = Sm100Cfg<D>;
+  using C = Sm100Cfg<D, F8>;
   int seq = 0;  // K/V tiles put into the ring so far (K and V counted apart)
   int qi = 0;   // units with keys loaded so far
   const bool packed = p.cu_seqlens != nullptr;
@@ -199,7 +214,7 @@ __device__ void role_producer(const Sm100Ctx<D> &x, const FwdParams &p, const CU
     const int u = snake_unit(k, p.num_units);
     if (u == -2) break;
     if (u < 0) continue;
-    const Unit w = unit_at<D>(p, u);
+    const Unit w = unit_at<D, F8>(p, u);
     if (w.nkv == 0) continue;
     // Q tile t of this unit replaces the previous unit's once its last
     // S product has read it.
@@ -213,17 +228,17 @@ __device__ void role_producer(const Sm100Ctx<D> &x, const FwdParams &p, const CU
       // The padded layout's maps are (d, rows, plane); the packed layout's
       // are (d, head, token), which keeps their strides increasing.
       const int qrow = w.tok0 + w.row0 + t * C::BM;
-      for (int half = 0; half < D / 64; ++half)
-        tma_load_3d(x.q_tile(t) + half * C::HALF_BYTES, tm_q, x.bar(C::BAR_Q_FULL + t), half * 64,
-                    packed ? w.q_plane : qrow, packed ? qrow : w.q_plane);
+      for (int bx = 0; bx < C::NBOX; ++bx)
+        tma_load_3d(x.q_tile(t) + bx * C::BOX_BYTES, tm_q, x.bar(C::BAR_Q_FULL + t),
+                    bx * C::BOX_COLS, packed ? w.q_plane : qrow, packed ? qrow : w.q_plane);
     }
     if (!ok) break;
     ++qi;
     const int kv_plane = w.kv_plane;
     for (int j = 0; j < w.nkv && ok; ++j) {
       for (int kv = 0; kv < 2; ++kv, ++seq) {
-        const int slot = ring_slot<D>(seq);
-        if (!mbar_wait_bounded(x.bar(C::BAR_KV_EMPTY + slot), ring_parity<D>(seq) ^ 1,
+        const int slot = ring_slot<D, F8>(seq);
+        if (!mbar_wait_bounded(x.bar(C::BAR_KV_EMPTY + slot), ring_parity<D, F8>(seq) ^ 1,
                                x.abort_flag, p.status, p.wait_limit_ns, kErrTimeout)) {
           ok = false;
           break;
@@ -232,9 +247,14 @@ __device__ void role_producer(const Sm100Ctx<D> &x, const FwdParams &p, const CU
         mbar_arrive_expect_tx(full, C::TILE_BYTES);
         const CUtensorMap *m = kv ? tm_v : tm_k;
         const int krow = w.tok0 + j * C::BN;
-        for (int half = 0; half < D / 64; ++half)
-          tma_load_3d(x.kv_tile(slot) + half * C::HALF_BYTES, m, full, half * 64,
-                      packed ? kv_plane : krow, packed ? krow : kv_plane);
+        if (F8 && kv) {
+          // V^T tile: 128 keys (x, contiguous) by the d rows (y); one box.
+          tma_load_3d(x.kv_tile(slot), m, full, krow, 0, kv_plane);
+        } else {
+          for (int bx = 0; bx < C::NBOX; ++bx)
+            tma_load_3d(x.kv_tile(slot) + bx * C::BOX_BYTES, m, full, bx * C::BOX_COLS,
+                        packed ? kv_plane : krow, packed ? krow : kv_plane);
+        }
       }
     }
   }
@@ -246,7 +266,7 @@ __device__ void role_producer(const Sm100Ctx<D> &x, const FwdParams &p, const CU
                         p.wait_limit_ns, kErrTimeout);
   for (int s = 0; s < C::STAGES && s < seq; ++s) {
     const int last = s + C::STAGES * ((seq - 1 - s) / C::STAGES);
-    mbar_wait_bounded(x.bar(C::BAR_KV_FULL + s), ring_parity<D>(last), &never, p.status,
+    mbar_wait_bounded(x.bar(C::BAR_KV_FULL + s), ring_parity<D, F8>(last), &never, p.status,
                       p.wait_limit_ns, kErrTimeout);
   }
 }
@@ -256,11 +276,13 @@ __device__ void role_producer(const Sm100Ctx<D> &x, const FwdParams &p, const CU
 // descriptor arithmetic stays warp-uniform; one elected lane issues the
 // tcgen05 instructions and their commits)
 // --------------------------------------------------------------------------
-template <int D>
-__device__ void role_mma(const Sm100Ctx<D> &x, const FwdParams &p) {
-  using C = Sm100Cfg<D>;
-  constexpr uint32_t IDESC_S = idesc_bf16_f32(128, C::BN, 0, 0);  // Q, K both K-major
-  constexpr uint32_t IDESC_O = idesc_bf16_f32(128, D, 0, 1);      // P from TMEM, V MN-major
+template <int D, bool F8>
+__device__ void role_mma(const Sm100Ctx<D, F8> &x, const FwdParams &p) {
+  using C = Sm100Cfg<D, F8>;
+  // S: Q and K both K-major.  O: P from TMEM; V MN-major (bf16) or V^T
+  // K-major (FP8).
+  constexpr uint32_t IDESC_S = F8 ? idesc_e4m3_f32(128, C::BN) : idesc_bf16_f32(128, C::BN, 0, 0);
+  constexpr uint32_t IDESC_O = F8 ? idesc_e4m3_f32(128, D) : idesc_bf16_f32(128, D, 0, 1);
   const bool leader = elect_one();
   const uint32_t tS[2] = {x.tmem + C::COL_S0, x.tmem + C::COL_S0 + 128};
   const uint32_t tO[2] = {x.tmem + C::COL_O0, x.tmem + C::COL_O0 + 128};
@@ -270,7 +292,8 @@ __device__ void role_mma(const Sm100Ctx<D> &x, const FwdParams &p) {
   const uint64_t desc_q[2] = {smem_desc_sw128(x.q_tile(0), 16, 1024),
                               smem_desc_sw128(x.q_tile(1), 16, 1024)};
   const uint64_t desc_kv_k = smem_desc_sw128(x.kv_tile(0), 16, 1024);
-  const uint64_t desc_kv_v = smem_desc_sw128(x.kv_tile(0), C::HALF_BYTES, 1024);
+  const uint64_t desc_kv_v = F8 ? smem_desc_sw128(x.kv_tile(0), 16, 1024)
+                                : smem_desc_sw128(x.kv_tile(0), C::BOX_BYTES, 1024);
 
   auto wait = [&](int bar, uint32_t parity) {
     const bool ok = mbar_wait_bounded(x.bar(bar), parity, x.abort_flag, p.status,
@@ -281,29 +304,46 @@ __device__ void role_mma(const Sm100Ctx<D> &x, const FwdParams &p) {
     if (leader) tc_commit(x.bar(bar));
     __syncwarp();
   };
-  // S_t = Q_t K^T: K = d in steps of 16; a K step of 16 bf16 is 32 bytes inside
-  // a 128-byte swizzled row, and every 4 steps move to the next 64-column box.
+  // S_t = Q_t K^T: K = d in steps of 32 bytes (16 bf16 or 32 FP8 values)
+  // inside a 128-byte swizzled row; every 4 steps move to the next box.
   auto issue_s = [&](int t, int k_slot_idx) {
     const uint64_t kd = desc_kv_k + ((k_slot_idx * C::TILE_BYTES) >> 4);
 #pragma unroll
-    for (int kk = 0; kk < D / 16; ++kk) {
-      const uint32_t off = ((kk / 4) * C::HALF_BYTES + (kk % 4) * 32) >> 4;
-      if (leader) tc_mma_ss(tS[t], desc_q[t] + off, kd + off, IDESC_S, kk > 0 ? 1u : 0u);
+    for (int kk = 0; kk < C::KSTEPS; ++kk) {
+      const uint32_t off = ((kk / 4) * C::BOX_BYTES + (kk % 4) * 32) >> 4;
+      if (leader) {
+        if constexpr (F8)
+          tc_mma_ss_f8(tS[t], desc_q[t] + off, kd + off, IDESC_S, kk > 0 ? 1u : 0u);
+        else
+          tc_mma_ss(tS[t], desc_q[t] + off, kd + off, IDESC_S, kk > 0 ? 1u : 0u);
+      }
     }
     __syncwarp();
   };
   // O_t += P_t V for one half of the keys (64): K in steps of 16; P_t steps
   // 8 columns (16 bf16) in TMEM; V steps 16 key rows = 2048 bytes; its two
-  // 64-column boxes are HALF_BYTES apart (leading byte offset), 8-row groups
+  // 64-column boxes are BOX_BYTES apart (leading byte offset), 8-row groups
   // 1024 bytes apart.
+  // FP8: K in steps of 32 keys; P_t steps 8 columns (32 codes); V^T steps 32
+  // bytes along its 128-byte rows of keys.
   auto issue_pv_half = [&](int t, int v_slot_idx, int half, bool accumulate) {
     const uint64_t vd = desc_kv_v + ((v_slot_idx * C::TILE_BYTES) >> 4);
+    if constexpr (F8) {
 #pragma unroll
-    for (int k4 = 0; k4 < 4; ++k4) {
-      const int kk = 4 * half + k4;
-      if (leader)
-        tc_mma_ts(tO[t], tS[t] + kk * 8, vd + ((kk * 2048) >> 4), IDESC_O,
-                  (accumulate || kk > 0) ? 1u : 0u);
+      for (int k2 = 0; k2 < 2; ++k2) {
+        const int kk = 2 * half + k2;
+        if (leader)
+          tc_mma_ts_f8(tO[t], tS[t] + kk * 8, vd + ((kk * 32) >> 4), IDESC_O,
+                       (accumulate || kk > 0) ? 1u : 0u);
+      }
+    } else {
+#pragma unroll
+      for (int k4 = 0; k4 < 4; ++k4) {
+        const int kk = 4 * half + k4;
+        if (leader)
+          tc_mma_ts(tO[t], tS[t] + kk * 8, vd + ((kk * 2048) >> 4), IDESC_O,
+                    (accumulate || kk > 0) ? 1u : 0u);
+      }
     }
     __syncwarp();
   };
@@ -327,32 +367,32 @@ __device__ void role_mma(const Sm100Ctx<D> &x, const FwdParams &p) {
     const int u = snake_unit(k, p.num_units);
     if (u == -2) break;
     if (u < 0) continue;
-    const Unit w = unit_at<D>(p, u);
+    const Unit w = unit_at<D, F8>(p, u);
     const int nkv = w.nkv;
     if (nkv == 0) continue;
     const uint32_t qpar = static_cast<uint32_t>(qi & 1);
     if (!wait(C::BAR_Q_FULL + 0, qpar) || !wait(C::BAR_Q_FULL + 1, qpar) ||
-        !wait(C::BAR_KV_FULL + ring_slot<D>(2 * g), ring_parity<D>(2 * g))) {
+        !wait(C::BAR_KV_FULL + ring_slot<D, F8>(2 * g), ring_parity<D, F8>(2 * g))) {
       ok = false;
       break;
     }
     tc_fence_after();
     // Tile 0: S for both Q tiles.
-    issue_s(0, ring_slot<D>(2 * g));
+    issue_s(0, ring_slot<D, F8>(2 * g));
     commit(C::BAR_S_FULL + 0);
     if (nkv == 1) commit(C::BAR_Q_EMPTY + 0);
-    issue_s(1, ring_slot<D>(2 * g));
+    issue_s(1, ring_slot<D, F8>(2 * g));
     commit(C::BAR_S_FULL + 1);
-    commit(C::BAR_KV_EMPTY + ring_slot<D>(2 * g));
+    commit(C::BAR_KV_EMPTY + ring_slot<D, F8>(2 * g));
     if (nkv == 1) commit(C::BAR_Q_EMPTY + 1);
     // Steady state: PV of tile j-1, then S of tile j into the same columns
     // (the tensor pipe runs them in order, so P is read before S lands).
     for (int j = 1; j < nkv; ++j) {
       const int gp = g + j - 1, gc = g + j;
       const uint32_t pp = static_cast<uint32_t>(gp & 1);
-      const int vs = ring_slot<D>(2 * gp + 1), ks = ring_slot<D>(2 * gc);
-      if (!wait(C::BAR_KV_FULL + vs, ring_parity<D>(2 * gp + 1)) || !pv(0, vs, pp, j - 1 > 0) ||
-          !wait(C::BAR_KV_FULL + ks, ring_parity<D>(2 * gc))) {
+      const int vs = ring_slot<D, F8>(2 * gp + 1), ks = ring_slot<D, F8>(2 * gc);
+      if (!wait(C::BAR_KV_FULL + vs, ring_parity<D, F8>(2 * gp + 1)) || !pv(0, vs, pp, j - 1 > 0) ||
+          !wait(C::BAR_KV_FULL + ks, ring_parity<D, F8>(2 * gc))) {
         ok = false;
         break;
       }
@@ -373,9 +413,9 @@ __device__ void role_mma(const Sm100Ctx<D> &x, const FwdParams &p) {
     if (!ok) break;
     // Last tile's PV products, then the unit's output is complete.
     const int gl = g + nkv - 1;
-    const int vs = ring_slot<D>(2 * gl + 1);
+    const int vs = ring_slot<D, F8>(2 * gl + 1);
     const uint32_t pp = static_cast<uint32_t>(gl & 1);
-    if (!wait(C::BAR_KV_FULL + vs, ring_parity<D>(2 * gl + 1)) || !pv(0, vs, pp, nkv > 1)) {
+    if (!wait(C::BAR_KV_FULL + vs, ring_parity<D, F8>(2 * gl + 1)) || !pv(0, vs, pp, nkv > 1)) {
       ok = false;
       break;
     }
@@ -398,9 +438,9 @@ __device__ void role_mma(const Sm100Ctx<D> &x, const FwdParams &p) {
 // --------------------------------------------------------------------------
 // Softmax warpgroup t (128 threads, one query row each)
 // --------------------------------------------------------------------------
-template <int D>
-__device__ void role_softmax(const Sm100Ctx<D> &x, const FwdParams &p, int t) {
-  using C = Sm100Cfg<D>;
+template <int D, bool F8>
+__device__ void role_softmax(const Sm100Ctx<D, F8> &x, const FwdParams &p, int t) {
+  using C = Sm100Cfg<D, F8>;
   const int r = threadIdx.x & 127;
   const uint32_t lane_base = static_cast<uint32_t>((threadIdx.x >> 5) & 3) * 32u << 16;
   const uint32_t tS = x.tmem + lane_base + C::COL_S0 + 128 * t;
@@ -419,7 +459,7 @@ __device__ void role_softmax(const Sm100Ctx<D> &x, const FwdParams &p, int t) {
     const int u = snake_unit(k, p.num_units);
     if (u == -2) break;
     if (u < 0) continue;
-    const Unit w = unit_at<D>(p, u);
+    const Unit w = unit_at<D, F8>(p, u);
     const int tile_row0 = w.row0 + t * C::BM;
     const int i = tile_row0 + r;  // this thread's query row
     const bool valid = i < w.q_rows;
@@ -455,11 +495,12 @@ __device__ void role_softmax(const Sm100Ctx<D> &x, const FwdParams &p, int t) {
         for (int c = 0; c < 128; ++c)
           if (kbase + c >= limit) s[c] = __float_as_uint(-INFINITY);
       }
-      // p = 2^(s * scale * log2(e) - m_ref) for 64 keys: the row sum takes
-      // p in fp32 and the PV product its bf16 rounding.
+      // p = 2^(s * scale * log2(e) - m_ref + P_SHIFT) for 64 keys: the row
+      // sum takes p in fp32 and the PV product its bf16 (or E4M3) rounding.
       const uint64_t scale2 = f32x2(sl2, sl2);
-      auto exp_half = [&](int half, float m_use, uint32_t(&pk)[32], uint64_t &sum2) {
-        const uint64_t shift2 = f32x2(-m_use, -m_use);
+      auto exp_half = [&](int half, float m_use, uint32_t(&pk)[C::PK_WORDS], uint64_t &sum2) {
+        const float sh = F8 ? C::P_SHIFT - m_use : -m_use;
+        const uint64_t shift2 = f32x2(sh, sh);
 #pragma unroll
         for (int e = 0; e < 32; ++e) {
           const int c = half * 64 + 2 * e;
@@ -473,7 +514,15 @@ __device__ void role_softmax(const Sm100Ctx<D> &x, const FwdParams &p, int t) {
             p0 = ex2_approx(x0);
             p1 = ex2_approx(x1);
           }
-          pk[e] = pack_bf16x2(p0, p1);
+          if constexpr (F8) {
+            const uint32_t h = pack_e4m3x2(p0, p1);
+            if (e & 1)
+              pk[e >> 1] |= h << 16;
+            else
+              pk[e >> 1] = h;
+          } else {
+            pk[e] = pack_bf16x2(p0, p1);
+          }
           sum2 = add_f32x2(sum2, f32x2(p0, p1));
         }
       };
@@ -492,8 +541,15 @@ __device__ void role_softmax(const Sm100Ctx<D> &x, const FwdParams &p, int t) {
         return fmaxf(fmax3(mq[0], mq[1], mq[2]), fmax3(fmax3(mq[3], mq[4], mq[5]), mq[6], mq[7]));
       };
 
-      uint32_t pk[32];
+      uint32_t pk[C::PK_WORDS];
       uint64_t sum2 = f32x2(0.f, 0.f);
+      // P of one 64-key half over the first columns of S_t.
+      auto store_p = [&](int half) {
+        if constexpr (F8)
+          tmem_st16(tS + 16 * half, pk);
+        else
+          tmem_st32(tS + 32 * half, pk);
+      };
       bool need;
       float alpha = 1.0f;
       if (j > 0) {
@@ -522,7 +578,7 @@ __device__ void role_softmax(const Sm100Ctx<D> &x, const FwdParams &p, int t) {
         exp_half(0, (m_ref == -INFINITY) ? 0.0f : m_ref, pk, sum2);
       }
       const float m_use = (m_ref == -INFINITY) ? 0.0f : m_ref;
-      tmem_st32(tS, pk);
+      store_p(0);
       // O holds earlier tiles' sum only for j > 0; nothing writes it until
       // this warpgroup publishes P (the PV product of tile j-1 finished
       // before S_j did).  It is rescaled before the first half goes out.
@@ -542,7 +598,7 @@ __device__ void role_softmax(const Sm100Ctx<D> &x, const FwdParams &p, int t) {
       mbar_arrive(x.bar(C::BAR_P_HALF + 2 * t));
       // Second half of the keys.
       exp_half(1, m_use, pk, sum2);
-      tmem_st32(tS + 32, pk);
+      store_p(1);
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(x.bar(C::BAR_P_HALF + 2 * t + 1));
@@ -554,7 +610,8 @@ __device__ void role_softmax(const Sm100Ctx<D> &x, const FwdParams &p, int t) {
     // Epilogue: O = O~ / l in bf16, LSE = (m_ref + log2 l) * ln 2.
     if (!wait_all(C::BAR_O_FULL + t, static_cast<uint32_t>(qi & 1))) return;
     tc_fence_after();
-    const float inv_l = l > 0.f ? 1.0f / l : 0.0f;
+    float inv_l = l > 0.f ? 1.0f / l : 0.0f;
+    if constexpr (F8) inv_l *= p.out_scale;
     uint16_t *orow = p.o + w.o_base + (valid ? i : 0) * w.o_stride;
 #pragma unroll
     for (int c = 0; c < D / 32; ++c) {
@@ -573,20 +630,21 @@ __device__ void role_softmax(const Sm100Ctx<D> &x, const FwdParams &p, int t) {
           dst[v4] = make_uint4(wv[4 * v4], wv[4 * v4 + 1], wv[4 * v4 + 2], wv[4 * v4 + 3]);
       }
     }
-    if (valid)
+    if (valid) {
+      // l carries the factor 2^P_SHIFT of the stored probabilities.
+      const float m_lse = F8 ? m_ref - C::P_SHIFT : m_ref;
       p.lse[w.lse_base + i] =
-          l > 0.f ? (m_ref + __log2f(l)) * 0.69314718055994530942f : -INFINITY;
+          l > 0.f ? (m_lse + __log2f(l)) * 0.69314718055994530942f : -INFINITY;
+    }
     g += w.nkv;
     ++qi;
   }
 }
 
-template <int D>
-__global__ void __launch_bounds__(Sm100Cfg<D>::THREADS, 1)
-    fa_fwd_bf16_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
-                             const __grid_constant__ CUtensorMap tm_k,
-                             const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
-  using C = Sm100Cfg<D>;
+template <int D, bool F8>
+__device__ __forceinline__ void fwd_kernel_body(const CUtensorMap *tm_q, const CUtensorMap *tm_k,
+                                                const CUtensorMap *tm_v, const FwdParams &p) {
+  using C = Sm100Cfg<D, F8>;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
@@ -594,7 +652,7 @@ __global__ void __launch_bounds__(Sm100Cfg<D>::THREADS, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
-  Sm100Ctx<D> x;
+  Sm100Ctx<D, F8> x;
   x.smem = base;
   x.abort_flag = reinterpret_cast<volatile int *>(smem + C::OFF_MISC + 4);
 
@@ -620,9 +678,9 @@ __global__ void __launch_bounds__(Sm100Cfg<D>::THREADS, 1)
     tmem_relinquish();
   }
   if (warp == 8 && lane == 0) {
-    tma_prefetch_desc(&tm_q);
-    tma_prefetch_desc(&tm_k);
-    tma_prefetch_desc(&tm_v);
+    tma_prefetch_desc(tm_q);
+    tma_prefetch_desc(tm_k);
+    tma_prefetch_desc(tm_v);
   }
   tc_fence_before();
   __syncthreads();
@@ -634,13 +692,13 @@ __global__ void __launch_bounds__(Sm100Cfg<D>::THREADS, 1)
   if (warp >= 8) {
     regs_decrease<C::REGS_CONTROL>();
     if (warp == 8) {
-      if (lane == 0) role_producer<D>(x, p, &tm_q, &tm_k, &tm_v);
+      if (lane == 0) role_producer<D, F8>(x, p, tm_q, tm_k, tm_v);
     } else if (warp == 9) {
-      role_mma<D>(x, p);
+      role_mma<D, F8>(x, p);
     }
   } else {
     regs_increase<C::REGS_SOFTMAX>();
-    role_softmax<D>(x, p, warp >> 2);
+    role_softmax<D, F8>(x, p, warp >> 2);
   }
   __syncwarp();
   tc_fence_before();
@@ -649,6 +707,22 @@ __global__ void __launch_bounds__(Sm100Cfg<D>::THREADS, 1)
     tc_fence_after();
     tmem_dealloc(x.tmem, C::TMEM_COLS);
   }
+}
+
+template <int D>
+__global__ void __launch_bounds__(Sm100Cfg<D>::THREADS, 1)
+    fa_fwd_bf16_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
+                             const __grid_constant__ CUtensorMap tm_k,
+                             const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
+  fwd_kernel_body<D, false>(&tm_q, &tm_k, &tm_v, p);
+}
+
+// FP8 E4M3 inputs (head dim 128); tm_v maps V^T.
+__global__ void __launch_bounds__(Sm100Cfg<128, true>::THREADS, 1)
+    fa_fwd_e4m3_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
+                             const __grid_constant__ CUtensorMap tm_k,
+                             const __grid_constant__ CUtensorMap tm_vt, const FwdParams p) {
+  fwd_kernel_body<128, true>(&tm_q, &tm_k, &tm_vt, p);
 }
 
 }  // namespace fa

@@ -1,7 +1,8 @@
-"""Seeded synthetic inputs for the attention forward.
+"""Seeded synthetic inputs for the attention kernels.
 
-This module only draws numbers and rounds them to bf16; it holds none of the
-attention arithmetic.  Both the CUDA path (through the binding) and the CPU
+This module only draws numbers and rounds them to bf16 (or quantises them to
+FP8 E4M3 with one scale per tensor); it holds none of the attention
+arithmetic.  Both the CUDA path (through the binding) and the CPU
 oracle consume what it produces, so neither has to import the other.
 
 Recipe (the same for every workload):
@@ -15,7 +16,10 @@ Recipe (the same for every workload):
   * key-padded workloads then draw ``seqlens = rng.integers(lo, hi + 1, B)``
     from the same generator;
   * sampled-row checks draw their query rows from ``default_rng(seed + 100)``
-    without replacement, independently per (batch, head).
+    without replacement, independently per (batch, head);
+  * FP8 inputs take the same fp32 draws and quantise each tensor to E4M3
+    codes with descale = amax / 448 (round to nearest even, PyTorch's
+    float8_e4m3fn cast); V is also laid out transposed, keys contiguous.
 """
 from __future__ import annotations
 
@@ -63,7 +67,11 @@ DECODE = Workload("llama_gqa_decode_b8_hq32_hkv8_nq1_nk32768_d128", 8, 32, 8, 32
                   seed=6, seqlen_range=(16384, 32768), nq=1)
 
 ALL = (TINY, GPT2, BERT, LLAMA_GQA, LONG)
-BY_NAME = {w.name: w for w in ALL + (DECODE,)}
+# The GQA workload with FP8 E4M3 inputs (the same draws, quantised).
+LLAMA_GQA_FP8 = Workload("llama_gqa_causal_b2_hq32_hkv8_n8192_d128_e4m3", 2, 32, 8, 8192, 128,
+                         True, seed=4, k_scale=2.0, sample_rows=32)
+
+BY_NAME = {w.name: w for w in ALL + (DECODE, LLAMA_GQA_FP8)}
 
 
 def round_to_bf16_bits(x: np.ndarray) -> np.ndarray:
@@ -171,3 +179,73 @@ def flops(w: Workload, seqlens: np.ndarray | None = None) -> float:
         return 4.0 * w.Hq * w.d * w.N * float(np.sum(seqlens))
     f = 4.0 * w.B * w.Hq * w.N * w.N * w.d
     return f / 2 if w.causal else f
+
+
+# ---------------------------------------------------------------------------
+# FP8 E4M3 inputs
+# ---------------------------------------------------------------------------
+E4M3_MAX = 448.0
+
+
+def quantize_e4m3(x: np.ndarray) -> tuple[np.ndarray, float]:
+    """fp32 -> (E4M3 codes as uint8, descale): descale = amax / 448 in fp32,
+    codes = x / descale rounded to nearest even by PyTorch's float8_e4m3fn
+    cast (clamped to +-448 first), so code * descale approximates x."""
+    import torch
+    x = np.ascontiguousarray(x, dtype=np.float32)
+    amax = float(np.max(np.abs(x))) if x.size else 0.0
+    descale = np.float32(amax / E4M3_MAX) if amax > 0 else np.float32(1.0)
+    t = (torch.from_numpy(x) / torch.tensor(descale, dtype=torch.float32))
+    t = t.clamp(-E4M3_MAX, E4M3_MAX)
+    return t.to(torch.float8_e4m3fn).view(torch.uint8).numpy(), float(descale)
+
+
+def e4m3_transpose(v_codes: np.ndarray, ldvt: int | None = None) -> np.ndarray:
+    """[B, H, N, d] codes -> [B, H, d, ldvt] (keys contiguous), zero padded
+    past N; ldvt defaults to N rounded up to 16."""
+    B, H, N, d = v_codes.shape
+    ld = ldvt if ldvt is not None else (N + 15) // 16 * 16
+    if ld < N:
+        raise ValueError("ldvt must be >= N")
+    out = np.zeros((B, H, d, ld), dtype=np.uint8)
+    out[..., :N] = np.swapaxes(v_codes, 2, 3)
+    return out
+
+
+@dataclasses.dataclass
+class Fp8Inputs:
+    """One seeded draw quantised to E4M3: ``q``, ``k``, ``v`` are codes
+    [B, H, N, d]; element value = code * descale of its tensor."""
+    q: np.ndarray
+    k: np.ndarray
+    v: np.ndarray
+    descale_q: float
+    descale_k: float
+    descale_v: float
+    seqlens: np.ndarray | None
+
+    def vt(self, ldvt: int | None = None) -> np.ndarray:
+        return e4m3_transpose(self.v, ldvt)
+
+
+def draw_fp8(B: int, Hq: int, Hkv: int, N: int, d: int, seed: int, *, k_scale: float = 1.0,
+             seqlen_range: tuple[int, int] | None = None) -> Fp8Inputs:
+    """The fp32 draws of ``draw`` (same seed, same order), each tensor
+    quantised to E4M3 with its own scale."""
+    rng = np.random.default_rng(seed)
+    q = rng.standard_normal((B, Hq, N, d), dtype=np.float32)
+    k = rng.standard_normal((B, Hkv, N, d), dtype=np.float32)
+    v = rng.standard_normal((B, Hkv, N, d), dtype=np.float32)
+    if k_scale != 1.0:
+        k *= np.float32(k_scale)
+    seqlens = None
+    if seqlen_range is not None:
+        lo, hi = seqlen_range
+        seqlens = rng.integers(lo, hi + 1, B).astype(np.int32)
+    (qc, dq), (kc, dk), (vc, dv) = quantize_e4m3(q), quantize_e4m3(k), quantize_e4m3(v)
+    return Fp8Inputs(qc, kc, vc, dq, dk, dv, seqlens)
+
+
+def draw_fp8_workload(w: Workload) -> Fp8Inputs:
+    return draw_fp8(w.B, w.Hq, w.Hkv, w.N, w.d, w.seed, k_scale=w.k_scale,
+                    seqlen_range=w.seqlen_range)

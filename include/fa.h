@@ -151,6 +151,33 @@ FA_API int fa_bwd(const void *q, const void *k, const void *v, const void *o, co
                   size_t workspace_bytes, void *stream, int *status_dev);
 
 /*
+ * FP8 forward: the same operation as fa_fwd on inputs stored as FP8 E4M3
+ * codes with one scale per tensor (element value = code * descale).  The
+ * news explainer "FlashAttention" (saiita), section on the second and third
+ * generations, reports that the third generation reaches about 1.2 PFLOP/s
+ * on H100 with FP8; it gives no details, so the format choices here are
+ * this library's: E4M3 for Q, K, V and for the probabilities that enter
+ * the P.V product (3 mantissa bits), fp32 scores, row sums and LSE, bf16 O.
+ *  q  : [B, Hq, N, d] E4M3 codes      k : [B, Hkv, N, d] E4M3 codes
+ *  vt : V transposed, [B, Hkv, d, ldvt] E4M3 codes (keys contiguous);
+ *       ldvt >= N and a multiple of 16; columns N..ldvt-1 are never read
+ *  o  : [B, Hq, N, d] bf16            lse : [B, Hq, N] fp32, natural log of
+ *       the masked row sum of exp(scale * descale_q * descale_k * q.k)
+ *  d must be 128.  descale_q, descale_k, descale_v: finite and > 0.
+ *  seqlens, causal, GQA map: as fa_fwd.  All pointers DEVICE, 16-byte
+ *  aligned (lse 4-byte), owned by the caller; nothing is allocated.
+ * Returns FA_OK once launched on `stream` (NULL = legacy default stream);
+ * bounded-wait time-outs reach status_dev (or the library's own word).
+ * Errors: FA_ERR_NULL, FA_ERR_SHAPE (sizes, ldvt < N, a bad descale),
+ * FA_ERR_HEADS, FA_ERR_HEADDIM (d != 128), FA_ERR_ALIGN (a pointer, or ldvt
+ * not a multiple of 16), FA_ERR_ARCH, FA_ERR_CUDA, FA_ERR_LAUNCH.
+ */
+FA_API int fa_fwd_fp8(const void *q, const void *k, const void *vt, void *o, float *lse, int B,
+                      int Hq, int Hkv, int N, int ldvt, int d, float scale, float descale_q,
+                      float descale_k, float descale_v, int causal, const int *seqlens,
+                      void *stream, int *status_dev);
+
+/*
  * Packed variable-length forward: the tokens of B sequences are stored back
  * to back with no padding (the padding mask of the pages' statement, without
  * padded rows).  Same operation as fa_fwd per sequence, self-attention

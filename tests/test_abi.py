@@ -101,3 +101,18 @@ def test_without_a_b200_valid_calls_report_arch():
     lib = _lib.load()
     assert lib.fa_fwd(A, A, A, A, A, 1, 2, 1, 128, 64, 0.125, 0, None) == _lib.FA_ERR_ARCH
     assert lib.fa_check_status(None, None) == _lib.FA_ERR_ARCH
+
+
+def test_fp8_arguments_rejected_before_launch(lib):
+    # q, k, vt, o, lse, B, Hq, Hkv, N, ldvt, d, scale, descales, causal, seqlens, stream, status
+    def call(N=300, ldvt=304, d=128, dq=0.01, dk=0.01, dv=0.01, Hq=8, Hkv=2, q=A):
+        return lib.fa_fwd_fp8(q, A, A, A, A, 2, Hq, Hkv, N, ldvt, d, 0.088, dq, dk, dv, 1, None,
+                              None, None)
+    assert call(d=64) == _lib.FA_ERR_HEADDIM          # FP8 path: head dim 128 only
+    assert call(ldvt=296) == _lib.FA_ERR_SHAPE         # ldvt < N
+    assert call(ldvt=312 - 4) == _lib.FA_ERR_ALIGN     # not a multiple of 16
+    assert call(dq=0.0) == _lib.FA_ERR_SHAPE
+    assert call(dv=float("inf")) == _lib.FA_ERR_SHAPE
+    assert call(Hq=6, Hkv=4) == _lib.FA_ERR_HEADS
+    assert call(q=None) == _lib.FA_ERR_NULL
+    assert call(q=A + 8) == _lib.FA_ERR_ALIGN
