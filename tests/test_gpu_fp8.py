@@ -8,13 +8,13 @@ Tolerance (the pages give none for FP8; derived from the kernel's
 arithmetic).  The scores are exact products of 8-bit values summed in fp32,
 and the row sum l adds the fp32 probabilities, so LSE keeps the bf16 path's
 2e-3.  The probabilities enter the P.V product as E4M3 codes: the kernel
-stores p' = p * 2^c, with p = exp(s - max) and 4 <= c <= 8 (a factor 2^4
-plus the lag of at most 2^4 of its reference max).  A normal code is within
+stores p' = p * 2^c, with p = exp(s - max) and 2 <= c <= 8 (a factor 2^2
+plus the lag of at most 2^6 of its reference max).  A normal code is within
 a relative 2^-4 of p', and a subnormal one (p' < 2^-6) is within 2^-10
 absolute.  With w = p / sum(p), w_max = 1 / sum(p), and the exponential's
 own relative error (at most 7.5e-5), each output element of row i obeys
 
-  |O - O_ref| <= dv * sum_j |v_j| (max(2^-4 w_j, 2^-14 w_max) + 7.5e-5 w_j)
+  |O - O_ref| <= dv * sum_j |v_j| (max(2^-4 w_j, 2^-12 w_max) + 7.5e-5 w_j)
                  + 2^-9 |O_ref| + 1e-5
 
 where the sum runs over the keys the row sees (w_j > 0), v_j are V's codes
@@ -46,7 +46,7 @@ def _bounds(p, v_vals, o_ref, group):
         for h in range(Hq):
             w = p[b, h]
             wmax = w.max(axis=1, keepdims=True)
-            term = np.where(w > 0, np.maximum(2.0 ** -4 * w, 2.0 ** -14 * wmax) + 7.5e-5 * w, 0.0)
+            term = np.where(w > 0, np.maximum(2.0 ** -4 * w, 2.0 ** -12 * wmax) + 7.5e-5 * w, 0.0)
             out[b, h] = term @ np.abs(v_vals[b, h // group])
     return out + 2.0 ** -9 * np.abs(o_ref) + 1e-5
 
