@@ -46,14 +46,23 @@ def load_peaks():
 
 
 def kernel_source_hash() -> str:
-    import glob
+    """sha256[:16] of what defines the timed forward kernel and its launch:
+    the kernel header, the PTX helpers, and the host functions that build
+    its tensor maps and launch it (their text in fa_api.cu)."""
     import hashlib
-    files = sorted(glob.glob(os.path.join(ROOT, "exact_io_aware_92_b200", "csrc", "*")))
-    files.append(os.path.join(ROOT, "include", "fa.h"))
+    import re
+    csrc = os.path.join(ROOT, "exact_io_aware_92_b200", "csrc")
     h = hashlib.sha256()
-    for f in files:
-        with open(f, "rb") as fh:
+    for name in ("fa_fwd_sm100.cuh", "sm100_ptx.cuh"):
+        with open(os.path.join(csrc, name), "rb") as fh:
             h.update(fh.read())
+    with open(os.path.join(csrc, "fa_api.cu")) as fh:
+        api = fh.read()
+    for head in (r"\nint make_map\(", r"\ntemplate <int D>\nint launch_bf16\("):
+        m = re.search(head + r".*?\n}\n", api, re.S)
+        if m is None:
+            raise RuntimeError(f"kernel_source_hash: {head!r} not found in fa_api.cu")
+        h.update(m.group(0).encode())
     return h.hexdigest()[:16]
 
 
@@ -307,7 +316,9 @@ def run_mine(args, w: wl.Workload):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded, bf16-rounded N(0,1))",
         "config": dict(workload_config(w),
-                       l2=f"no flush: inputs {in_bytes / 2**20:.0f} MiB > L2 126 MiB",
+                       l2=(f"no flush: inputs {in_bytes / 2**20:.0f} MiB > L2 126 MiB"
+                           if in_bytes > L2_BYTES else
+                           f"not flushed: inputs {in_bytes / 2**20:.1f} MiB fit in L2"),
                        parallelism=f"replicas x{world}" if world > 1 else "single GPU"),
         "roofline": {"bound": "tensor", "achieved": kernel_tflops, "peak": peak,
                      "unit": "TFLOP/s", "frac": kernel_tflops / peak, "traffic": traffic,
@@ -324,13 +335,23 @@ def run_mine(args, w: wl.Workload):
 
 
 def report_all_workloads(args):
-    """Throughput of the forward on each of the five workloads (one GPU),
-    one JSON object per line; not the contract line."""
+    """Throughput of each path on its workloads (one GPU), one JSON object
+    per line; not the contract line.  --only picks one section."""
+    import torch
+    dev = torch.device("cuda", 0)
+    sections = {"forward": report_forward, "varlen": report_varlen, "decode": report_decode,
+                "backward": report_backward, "fp8": report_fp8}
+    for name, fn in sections.items():
+        if args.only in (None, name):
+            fn(args, dev)
+
+
+def report_forward(args, dev):
+    """The bf16 forward on each of the five workloads."""
     import torch
     from exact_io_aware_92_b200 import attention
     peaks, src = load_peaks()
     peak = float(peaks["bf16_tflops"])
-    dev = torch.device("cuda", 0)
     for w in wl.ALL:
         inp = wl.draw_workload(w)
         q, k, v = (torch.from_numpy(x).view(torch.bfloat16).to(dev)
@@ -361,10 +382,6 @@ def report_all_workloads(args):
                           "flops": f, "algorithmic_bytes": algo_bytes,
                           "l2": "flushed between steps" if in_bytes < L2_BYTES else "inputs > L2",
                           "peak_source": src}), flush=True)
-    report_varlen(args, dev)
-    report_decode(args, dev)
-    report_backward(args, dev)
-    report_fp8(args, dev)
 
 
 def report_fp8(args, dev):
@@ -529,12 +546,14 @@ def main():
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["mine", "reference"], default="mine")
-    ap.add_argument("--workload", default=wl.LLAMA_GQA.name, choices=sorted(wl.BY_NAME))
+    ap.add_argument("--workload", default=wl.LLAMA_GQA.name, choices=[w.name for w in wl.ALL])
     ap.add_argument("--cpu-budget", type=float, default=15.0,
                     help="seconds of CPU work for the oracle baseline sample")
     ap.add_argument("--ref-budget", type=float, default=8.0,
                     help="seconds of CPU work per reference-arm step")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--only", choices=["forward", "varlen", "decode", "backward", "fp8"],
+                    default=None, help="with --all-workloads: run one section")
     ap.add_argument("--all-workloads", action="store_true",
                     help="report per-workload throughput for the five workloads instead")
     ap.add_argument("--batch", type=int, default=None,
