@@ -17,8 +17,12 @@
 //                      the left operand read from TMEM.
 // fa_bwd_dq_kernel     one CTA per 128-row query tile; per key tile:
 //                      S = Q K^T, dP = dO V^T, dS in bf16 over S, dQ += dS K.
-// Both tcgen05 kernels use 192 threads: warps 0-3 elementwise work, warp 4
-// TMA producer, warp 5 MMA issuer (one elected lane).  Every wait is bounded.
+// Both tcgen05 kernels use 320 threads: warps 0-7 elementwise work in two
+// warpgroups (each takes 64 of the tile's 128 columns: thread = TMEM lane,
+// warp w reaches lanes 32*(w%4)), warp 8 TMA producer, warp 9 MMA issuer
+// (one elected lane).  A warpgroup writes its bf16 P or dS over the first 32
+// of its own 64 columns (columns 0-31 and 64-95), so neither overwrites
+// scores the other has not read yet.  Every wait is bounded.
 #pragma once
 
 #include <cstdint>
@@ -45,7 +49,11 @@ template <int D>
 struct BwdCfg {
   static constexpr int HALF_BYTES = 128 * 64 * 2;
   static constexpr int TILE_BYTES = 128 * D * 2;
-  static constexpr int THREADS = 192;
+  static constexpr int THREADS = 320;
+  // TMEM column of the bf16 left operand for K step kk (16 rows of the
+  // product's K dimension, 8 columns): the two warpgroups' halves sit at
+  // columns 0-31 and 64-95.
+  __host__ __device__ static constexpr uint32_t a_col(int kk) { return 8u * kk + (kk >= 4 ? 32u : 0u); }
   static constexpr uint32_t COL_A = 0, COL_B = 128, COL_C = 256, COL_D = 384;
   // dK/dV kernel: K, V resident; ring of (Q, dO, LSE2, D) stages.
   static constexpr int KV_STAGES = 2;
@@ -129,11 +137,11 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
   uint8_t *smem = smem_raw + (base - raw);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-  // Unit: (key tile, batch, kv head); causal units with the most query
-  // tiles (the first key tiles) run first.
-  const int BHkv = p.B * p.Hkv;
-  const int kt = static_cast<int>(blockIdx.x) / BHkv;
-  const int bkv = static_cast<int>(blockIdx.x) % BHkv;
+  // Unit: (batch, kv head, key tile), groups outermost so that the CTAs in
+  // flight share one group's Q and dO stream in L2; within a group, causal
+  // units with the most query tiles (the first key tiles) run first.
+  const int kt = static_cast<int>(blockIdx.x) % p.q_tiles;
+  const int bkv = static_cast<int>(blockIdx.x) / p.q_tiles;
   const int b = bkv / p.Hkv, hkv = bkv % p.Hkv;
   int L = p.N;
   if (p.seqlens) L = min(max(p.seqlens[b], 0), p.N);
@@ -158,7 +166,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
       mbar_init(bar_empty + 8 * s, 1);
     }
     mbar_init(bar_st, 1);
-    mbar_init(bar_pds, 128);
+    mbar_init(bar_pds, 256);
     mbar_init(bar_done, 1);
     *abort_flag = 0;
     fence_barrier_init();
@@ -175,7 +183,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
   auto step_head = [&](int s) { return hkv * p.group + s / nq_per_head; };
   auto step_qt = [&](int s) { return qt0 + s % nq_per_head; };
 
-  if (nsteps > 0 && warp == 4) {
+  if (nsteps > 0 && warp == 8) {
     if (lane == 0) {
       // --- producer ---
       mbar_arrive_expect_tx(bar_kv, 2 * C::TILE_BYTES);
@@ -205,7 +213,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
                           p.wait_limit_ns, kErrTimeout);
       }
     }
-  } else if (nsteps > 0 && warp == 5) {
+  } else if (nsteps > 0 && warp == 9) {
     // --- MMA issuer ---
     const bool leader = elect_one();
     constexpr uint32_t IDESC_SS = idesc_bf16_f32(128, 128, 0, 0);  // K-major A and B
@@ -251,9 +259,9 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
           if (leader) {
-            tc_mma_ts(tmem + C::COL_D, tmem + C::COL_A + kk * 8, dOm + ((kk * 2048) >> 4),
+            tc_mma_ts(tmem + C::COL_D, tmem + C::COL_A + C::a_col(kk), dOm + ((kk * 2048) >> 4),
                       IDESC_TS, (s > 0 || kk > 0) ? 1u : 0u);
-            tc_mma_ts(tmem + C::COL_C, tmem + C::COL_B + kk * 8, dQm + ((kk * 2048) >> 4),
+            tc_mma_ts(tmem + C::COL_C, tmem + C::COL_B + C::a_col(kk), dQm + ((kk * 2048) >> 4),
                       IDESC_TS, (s > 0 || kk > 0) ? 1u : 0u);
           }
         }
@@ -264,11 +272,14 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
     commit(bar_done);
     volatile int never = 0;
     mbar_wait_bounded(bar_done, 0, &never, p.status, p.wait_limit_ns, kErrTimeout);
-  } else if (warp < 4) {
-    // --- elementwise warpgroup: thread = key row ---
-    const int j = key0 + threadIdx.x;
-    const uint32_t lane_base = static_cast<uint32_t>(warp) * 32u << 16;
-    const uint32_t tA = tmem + lane_base + C::COL_A, tB = tmem + lane_base + C::COL_B;
+  } else if (warp < 8) {
+    // --- elementwise warpgroups: thread = key row, warpgroup e = query
+    // columns [64e, 64e + 64) ---
+    const int e = warp >> 2;
+    const int j = key0 + (threadIdx.x & 127);
+    const uint32_t lane_base = static_cast<uint32_t>(warp & 3) * 32u << 16;
+    const uint32_t tA = tmem + lane_base + C::COL_A + 64 * e;
+    const uint32_t tB = tmem + lane_base + C::COL_B + 64 * e;
     const bool key_ok = j < L;
     bool ok = true;
     for (int s = 0; s < nsteps && ok; ++s) {
@@ -293,41 +304,41 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
       const float *lse2 =
           reinterpret_cast<const float *>(smem + C::OFF_RING + st * C::STAGE_BYTES + 2 * C::TILE_BYTES);
       const float *delta = lse2 + 128;
-#pragma unroll
-      for (int half = 0; half < 2; ++half) {
+      {
         uint32_t sv[64], dp[64];
-        tmem_ld32(tA + 64 * half, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
-        tmem_ld32(tA + 64 * half + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
-        tmem_ld32(tB + 64 * half, *reinterpret_cast<uint32_t(*)[32]>(&dp[0]));
-        tmem_ld32(tB + 64 * half + 32, *reinterpret_cast<uint32_t(*)[32]>(&dp[32]));
+        tmem_ld32(tA, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
+        tmem_ld32(tA + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
+        tmem_ld32(tB, *reinterpret_cast<uint32_t(*)[32]>(&dp[0]));
+        tmem_ld32(tB + 32, *reinterpret_cast<uint32_t(*)[32]>(&dp[32]));
         tmem_wait_ld();
         uint32_t pk[32], dk[32];
 #pragma unroll
-        for (int e = 0; e < 32; ++e) {
+        for (int x = 0; x < 32; ++x) {
           float pv[2], dv[2];
 #pragma unroll
           for (int u = 0; u < 2; ++u) {
-            const int c = 64 * half + 2 * e + u;  // query column within the tile
+            const int c = 64 * e + 2 * x + u;  // query column within the tile
             const int i = q0 + c;
             const bool vis = key_ok && (!p.causal || i >= j);
-            const float pp = vis ? ex2_approx(fmaf(__uint_as_float(sv[2 * e + u]), p.scale_log2,
+            const float pp = vis ? ex2_approx(fmaf(__uint_as_float(sv[2 * x + u]), p.scale_log2,
                                                    -lse2[c]))
                                  : 0.f;
             pv[u] = pp;
-            dv[u] = pp * (__uint_as_float(dp[2 * e + u]) - delta[c]);
+            dv[u] = pp * (__uint_as_float(dp[2 * x + u]) - delta[c]);
           }
-          pk[e] = pack_bf16x2(pv[0], pv[1]);
-          dk[e] = pack_bf16x2(dv[0], dv[1]);
+          pk[x] = pack_bf16x2(pv[0], pv[1]);
+          dk[x] = pack_bf16x2(dv[0], dv[1]);
         }
-        // P^T over S^T's columns 32*half.., dS^T over dP^T's.
-        tmem_st32(tA + 32 * half, pk);
-        tmem_st32(tB + 32 * half, dk);
+        // P^T over the first 32 of this warpgroup's S^T columns, dS^T over dP^T's.
+        tmem_st32(tA, pk);
+        tmem_st32(tB, dk);
       }
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(bar_pds);
     }
-    // Epilogue: dK = scale * sum dS^T Q, dV = sum P^T dO, in bf16.
+    // Epilogue: dK = scale * sum dS^T Q (warpgroup 0), dV = sum P^T dO
+    // (warpgroup 1), in bf16.
     if (ok && nsteps > 0) {
       const bool got = mbar_wait_bounded(bar_done, 0, abort_flag, p.status, p.wait_limit_ns,
                                          kErrTimeout);
@@ -339,8 +350,8 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
       const bool row_ok = j < p.N;
       const size_t row = (static_cast<size_t>(bkv) * p.N + (row_ok ? j : 0)) * D;
       if (nsteps > 0) tc_fence_after();
-#pragma unroll
-      for (int which = 0; which < 2; ++which) {
+      {
+        const int which = e;
         uint16_t *dst = (which == 0 ? p.dk : p.dv) + row;
         const float mult = which == 0 ? p.scale : 1.0f;
         const uint32_t tcol = tmem + lane_base + (which == 0 ? C::COL_C : C::COL_D);
@@ -352,12 +363,12 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
             tmem_wait_ld();
           } else {
 #pragma unroll
-            for (int e = 0; e < 32; ++e) r[e] = 0u;  // keys past the length: no gradient
+            for (int x = 0; x < 32; ++x) r[x] = 0u;  // keys past the length: no gradient
           }
           uint32_t w[16];
 #pragma unroll
-          for (int e = 0; e < 16; ++e)
-            w[e] = pack_bf16x2(__uint_as_float(r[2 * e]) * mult, __uint_as_float(r[2 * e + 1]) * mult);
+          for (int x = 0; x < 16; ++x)
+            w[x] = pack_bf16x2(__uint_as_float(r[2 * x]) * mult, __uint_as_float(r[2 * x + 1]) * mult);
           uint4 *d4 = reinterpret_cast<uint4 *>(dst + 32 * c);
           if (row_ok) {
 #pragma unroll
@@ -393,11 +404,11 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
   uint8_t *smem = smem_raw + (base - raw);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-  // Unit: (query tile, batch, head); causal units with the most key tiles
-  // (the last query tiles) first.
-  const int BH = p.B * p.Hq;
-  const int qt = p.q_tiles - 1 - static_cast<int>(blockIdx.x) / BH;
-  const int bh = static_cast<int>(blockIdx.x) % BH;
+  // Unit: (batch, head, query tile), heads outermost so that the CTAs in
+  // flight share one group's K and V in L2; within a head, causal units
+  // with the most key tiles (the last query tiles) first.
+  const int qt = p.q_tiles - 1 - static_cast<int>(blockIdx.x) % p.q_tiles;
+  const int bh = static_cast<int>(blockIdx.x) / p.q_tiles;
   const int b = bh / p.Hq, h = bh % p.Hq, hkv = h / p.group;
   const int bkv = b * p.Hkv + hkv;
   int L = p.N;
@@ -422,7 +433,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
       mbar_init(bar_empty + 8 * s, 1);
     }
     mbar_init(bar_sd, 1);
-    mbar_init(bar_ds, 128);
+    mbar_init(bar_ds, 256);
     mbar_init(bar_done, 1);
     *abort_flag = 0;
     fence_barrier_init();
@@ -436,7 +447,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
   tc_fence_after();
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t *>(tmem_slot);
 
-  if (nkv > 0 && warp == 4) {
+  if (nkv > 0 && warp == 8) {
     if (lane == 0) {
       mbar_arrive_expect_tx(bar_q, 2 * C::TILE_BYTES);
       load_tile<D>(base + C::OFF_Q, &tm_q, bar_q, row0, bh);
@@ -460,7 +471,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
                           p.wait_limit_ns, kErrTimeout);
       }
     }
-  } else if (nkv > 0 && warp == 5) {
+  } else if (nkv > 0 && warp == 9) {
     const bool leader = elect_one();
     constexpr uint32_t IDESC_SS = idesc_bf16_f32(128, 128, 0, 0);
     constexpr uint32_t IDESC_TS = idesc_bf16_f32(128, D, 0, 1);
@@ -502,7 +513,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
           if (leader)
-            tc_mma_ts(tmem + C::COL_C, tmem + C::COL_A + kk * 8, dKm + ((kk * 2048) >> 4),
+            tc_mma_ts(tmem + C::COL_C, tmem + C::COL_A + C::a_col(kk), dKm + ((kk * 2048) >> 4),
                       IDESC_TS, (j > 0 || kk > 0) ? 1u : 0u);
         __syncwarp();
         commit(bar_empty + 8 * st);
@@ -511,10 +522,13 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
     commit(bar_done);
     volatile int never = 0;
     mbar_wait_bounded(bar_done, 0, &never, p.status, p.wait_limit_ns, kErrTimeout);
-  } else if (warp < 4) {
-    const int i = row0 + threadIdx.x;
-    const uint32_t lane_base = static_cast<uint32_t>(warp) * 32u << 16;
-    const uint32_t tA = tmem + lane_base + C::COL_A, tB = tmem + lane_base + C::COL_B;
+  } else if (warp < 8) {
+    // thread = query row; warpgroup e = key columns [64e, 64e + 64)
+    const int e = warp >> 2;
+    const int i = row0 + (threadIdx.x & 127);
+    const uint32_t lane_base = static_cast<uint32_t>(warp & 3) * 32u << 16;
+    const uint32_t tA = tmem + lane_base + C::COL_A + 64 * e;
+    const uint32_t tB = tmem + lane_base + C::COL_B + 64 * e;
     const size_t vrow = static_cast<size_t>(bh) * p.Npad + i;
     const float lse2 = p.ws_lse2[vrow];
     const float delta = p.ws_delta[vrow];
@@ -528,29 +542,29 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
         break;
       }
       tc_fence_after();
-#pragma unroll
-      for (int half = 0; half < 2; ++half) {
+      {
         uint32_t sv[64], dp[64];
-        tmem_ld32(tA + 64 * half, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
-        tmem_ld32(tA + 64 * half + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
-        tmem_ld32(tB + 64 * half, *reinterpret_cast<uint32_t(*)[32]>(&dp[0]));
-        tmem_ld32(tB + 64 * half + 32, *reinterpret_cast<uint32_t(*)[32]>(&dp[32]));
+        tmem_ld32(tA, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
+        tmem_ld32(tA + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
+        tmem_ld32(tB, *reinterpret_cast<uint32_t(*)[32]>(&dp[0]));
+        tmem_ld32(tB + 32, *reinterpret_cast<uint32_t(*)[32]>(&dp[32]));
         tmem_wait_ld();
         uint32_t dk[32];
 #pragma unroll
-        for (int e = 0; e < 32; ++e) {
+        for (int x = 0; x < 32; ++x) {
           float dv[2];
 #pragma unroll
           for (int u = 0; u < 2; ++u) {
-            const int key = j * 128 + 64 * half + 2 * e + u;
-            const float pp = key < limit ? ex2_approx(fmaf(__uint_as_float(sv[2 * e + u]),
+            const int key = j * 128 + 64 * e + 2 * x + u;
+            const float pp = key < limit ? ex2_approx(fmaf(__uint_as_float(sv[2 * x + u]),
                                                            p.scale_log2, -lse2))
                                          : 0.f;
-            dv[u] = pp * (__uint_as_float(dp[2 * e + u]) - delta);
+            dv[u] = pp * (__uint_as_float(dp[2 * x + u]) - delta);
           }
-          dk[e] = pack_bf16x2(dv[0], dv[1]);
+          dk[x] = pack_bf16x2(dv[0], dv[1]);
         }
-        tmem_st32(tA + 32 * half, dk);
+        // dS over the first 32 of this warpgroup's S columns
+        tmem_st32(tA, dk);
       }
       tmem_wait_st();
       tc_fence_before();
@@ -566,21 +580,23 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
       const bool row_ok = i < p.N;
       uint16_t *dst = p.dq + (static_cast<size_t>(bh) * p.N + (row_ok ? i : 0)) * D;
       if (nkv > 0) tc_fence_after();
+      // warpgroup e writes columns [e D/2, (e + 1) D/2) of the row
 #pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
+      for (int c0 = 0; c0 < D / 64; ++c0) {
+        const int c = e * (D / 64) + c0;
         uint32_t r[32];
         if (nkv > 0) {
           tmem_ld32(tmem + lane_base + C::COL_C + 32 * c, r);
           tmem_wait_ld();
         } else {
 #pragma unroll
-          for (int e = 0; e < 32; ++e) r[e] = 0u;
+          for (int x = 0; x < 32; ++x) r[x] = 0u;
         }
         uint32_t w[16];
 #pragma unroll
-        for (int e = 0; e < 16; ++e)
-          w[e] = pack_bf16x2(__uint_as_float(r[2 * e]) * p.scale,
-                             __uint_as_float(r[2 * e + 1]) * p.scale);
+        for (int x = 0; x < 16; ++x)
+          w[x] = pack_bf16x2(__uint_as_float(r[2 * x]) * p.scale,
+                             __uint_as_float(r[2 * x + 1]) * p.scale);
         uint4 *d4 = reinterpret_cast<uint4 *>(dst + 32 * c);
         if (row_ok) {
 #pragma unroll
