@@ -42,17 +42,21 @@ struct DecodeParams {
 
 template <int D>
 struct DecodeCfg {
-  static constexpr int THREADS = 128;
+  static constexpr int WARPS = 8;   // two CTAs per SM (shared memory): 16 warps hide
+                                    // the latency of the shuffle reductions
+  static constexpr int THREADS = 32 * WARPS;
   static constexpr int ROWS = 4;                      // query rows per CTA
   static constexpr int CHUNK_BYTES = 16384;           // one K (or V) chunk
   static constexpr int KEYS = CHUNK_BYTES / (D * 2);  // keys per chunk: 64 (d=128), 128 (d=64)
   static constexpr int LPK = D / 8;                   // lanes per key (16 bytes each)
   static constexpr int KPW = 32 / LPK;                // keys per warp step
-  static constexpr int KPS = 4 * KPW;                 // keys per CTA step
-  static constexpr int STEPS = KEYS / KPS;            // steps per chunk (8)
+  static constexpr int KPS = WARPS * KPW;             // keys per CTA step
+  static constexpr int STEPS = KEYS / KPS;            // steps per chunk (4)
   static constexpr int STAGES = 3;
   static constexpr int SMEM = STAGES * 2 * CHUNK_BYTES + 64;
-  static_assert(STEPS == 8, "8 keys per lane group per chunk");
+  static_assert(STEPS * KPS == KEYS, "whole steps per chunk");
+  static_assert(WARPS * 4 * D * 4 + WARPS * 4 * 8 <= STAGES * 2 * CHUNK_BYTES,
+                "the cross-warp merge fits in the ring");
 };
 
 __device__ __forceinline__ void bulk_load(uint32_t dst, const void *src, uint32_t bytes,
@@ -229,7 +233,7 @@ __global__ void __launch_bounds__(DecodeCfg<D>::THREADS)
   }
 
   // Merge the lane groups of each warp (same columns, different keys), then
-  // the four warps through shared memory, then write the CTA's partial.
+  // the warps through shared memory, then write the CTA's partial.
 #pragma unroll
   for (int r = 0; r < R; ++r) {
 #pragma unroll
@@ -249,8 +253,8 @@ __global__ void __launch_bounds__(DecodeCfg<D>::THREADS)
     }
   }
   __syncthreads();  // the ring is free; reuse it for the cross-warp merge
-  float *red_o = reinterpret_cast<float *>(smem);          // [4 warps][R][D]
-  float *red_ml = red_o + 4 * R * D;                        // [4 warps][R][2]
+  float *red_o = reinterpret_cast<float *>(smem);          // [WARPS][R][D]
+  float *red_ml = red_o + C::WARPS * R * D;                 // [WARPS][R][2]
   if (lane < C::LPK) {
 #pragma unroll
     for (int r = 0; r < R; ++r) {
@@ -271,11 +275,11 @@ __global__ void __launch_bounds__(DecodeCfg<D>::THREADS)
     if (rr >= rows_total) continue;
     float mm = -INFINITY;
 #pragma unroll
-    for (int w = 0; w < 4; ++w) mm = fmaxf(mm, red_ml[(w * R + r) * 2]);
+    for (int w = 0; w < C::WARPS; ++w) mm = fmaxf(mm, red_ml[(w * R + r) * 2]);
     const float mu = (mm == -INFINITY) ? 0.f : mm;
     float acc = 0.f, ll = 0.f;
 #pragma unroll
-    for (int w = 0; w < 4; ++w) {
+    for (int w = 0; w < C::WARPS; ++w) {
       const float wgt = ex2_approx(red_ml[(w * R + r) * 2] - mu);
       acc += wgt * red_o[(w * R + r) * D + col];
       ll += wgt * red_ml[(w * R + r) * 2 + 1];
