@@ -19,9 +19,7 @@ import json
 import math
 import os
 import statistics
-import subprocess
 import sys
-import tempfile
 import time
 
 import numpy as np
@@ -72,60 +70,85 @@ def dist_env():
 
 
 class ClockSampler:
-    """nvidia-smi clocks and throttle reasons, sampled every 200 ms while the
-    timed region runs."""
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    """SM clock, power and clock-event reasons of the GPU the timed region runs
+    on, sampled every 10 ms through NVML in a background thread.  The device is
+    found by the UUID torch reports (CUDA_VISIBLE_DEVICES renumbers devices,
+    NVML does not).  Only samples taken between region_start() and
+    region_stop() are reported; without NVML the record says so.  Reading
+    only: nothing here changes a setting of the GPU."""
+    REASONS = (("hw_slowdown", "nvmlClocksEventReasonHwSlowdown"),
+               ("hw_thermal_slowdown", "nvmlClocksEventReasonHwThermalSlowdown"),
+               ("sw_thermal_slowdown", "nvmlClocksEventReasonSwThermalSlowdown"),
+               ("sw_power_cap", "nvmlClocksEventReasonSwPowerCap"))
 
-    def __init__(self, gpu_index: int):
-        self.gpu = gpu_index
-        self.proc = None
-        self.out = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+    def __init__(self, torch_index: int):
+        import threading
+        self.samples = []  # (t, sm_mhz, power_w, reasons bitmask)
+        self.t0 = self.t1 = None
+        self.stop_evt = threading.Event()
+        self.thread = None
+        self.nvml = None
+        self.handle = None
+        self.max_mhz = None
+        try:
+            import pynvml
+            import torch
+            pynvml.nvmlInit()
+            uuid = str(torch.cuda.get_device_properties(torch_index).uuid)
+            if not uuid.startswith("GPU-"):
+                uuid = "GPU-" + uuid
+            self.handle = pynvml.nvmlDeviceGetHandleByUUID(uuid)
+            self.max_mhz = float(pynvml.nvmlDeviceGetMaxClockInfo(self.handle,
+                                                                  pynvml.NVML_CLOCK_SM))
+            self.nvml = pynvml
+        except Exception:
+            self.nvml = None
+
+    def _run(self):
+        nv = self.nvml
+        while not self.stop_evt.is_set():
+            try:
+                t = time.monotonic()
+                sm = nv.nvmlDeviceGetClockInfo(self.handle, nv.NVML_CLOCK_SM)
+                pw = nv.nvmlDeviceGetPowerUsage(self.handle) / 1000.0
+                rs = nv.nvmlDeviceGetCurrentClocksEventReasons(self.handle)
+                self.samples.append((t, float(sm), pw, int(rs)))
+            except Exception:
+                pass
+            self.stop_evt.wait(0.01)
 
     def start(self):
-        try:
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "200"],
-                stdout=self.out, stderr=subprocess.DEVNULL)
-        except OSError:
-            self.proc = None
+        import threading
+        if self.nvml is not None:
+            self.thread = threading.Thread(target=self._run, daemon=True)
+            self.thread.start()
+
+    def region_start(self):
+        self.t0 = time.monotonic()
+
+    def region_stop(self):
+        self.t1 = time.monotonic()
 
     def stop(self):
-        if self.proc is None:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
-        time.sleep(0.25)
-        self.proc.terminate()
-        try:
-            self.proc.wait(timeout=5)
-        except subprocess.TimeoutExpired:
-            self.proc.kill()
-        self.out.flush()
-        self.out.seek(0)
-        sm, smax, power, reasons = [], [], [], set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for line in self.out.read().splitlines():
-            parts = [p.strip() for p in line.split(",")]
-            if len(parts) < 9:
-                continue
-            try:
-                sm.append(float(parts[1]))
-                smax.append(float(parts[2]))
-                power.append(float(parts[3]))
-            except ValueError:
-                continue
-            for name, flag in zip(names, parts[5:9]):
-                if flag.lower().startswith("active"):
+        if self.nvml is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvml unavailable"]}
+        self.stop_evt.set()
+        self.thread.join(timeout=5)
+        inside = [x for x in self.samples
+                  if self.t0 is not None and self.t1 is not None and self.t0 <= x[0] <= self.t1]
+        if not inside:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["no samples"]}
+        reasons = set()
+        for _, _, _, rs in inside:
+            for name, const in self.REASONS:
+                if rs & getattr(self.nvml, const):
                     reasons.add(name)
-        os.unlink(self.out.name)
-        if not sm:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
-        loaded = [s for s in sm if s > 0.5 * max(sm)] or sm
-        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": max(smax),
-                "reasons": sorted(reasons), "samples": len(sm),
-                "power_w_median": statistics.median(power) if power else None,
-                "power_w_max": max(power) if power else None}
+        sm = [x[1] for x in inside]
+        pw = [x[2] for x in inside]
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": self.max_mhz,
+                "sm_mhz_min": min(sm), "reasons": sorted(reasons), "samples": len(inside),
+                "power_w_median": statistics.median(pw), "power_w_max": max(pw),
+                "source": "NVML, 10 ms, timed region only"}
 
 
 def oracle_sample_rows(w: wl.Workload, rows_per_head: int, seed: int = 1234) -> np.ndarray:
@@ -245,12 +268,14 @@ def run_mine(args, w: wl.Workload):
     barrier()
     torch.cuda.synchronize(dev)
     sampler.start()
-    time.sleep(0.3)
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     start.record(stream)
     for _ in range(args.steps):
         step()
     end.record(stream)
+    sampler.region_start()  # launches are queued; the GPU runs them from here
+    end.synchronize()
+    sampler.region_stop()
     torch.cuda.synchronize(dev)
     barrier()
     clocks = sampler.stop()

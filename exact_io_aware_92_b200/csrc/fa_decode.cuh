@@ -68,6 +68,13 @@ __device__ __forceinline__ void bulk_load(uint32_t dst, const void *src, uint32_
       : "memory");
 }
 
+// Packed fp32 multiply of two pairs.
+__device__ __forceinline__ uint64_t mul_f32x2(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+
 // Eight bf16 values (16 bytes) to fp32.
 __device__ __forceinline__ void bf16x8_to_f32(const uint4 &u, float (&f)[8]) {
   const uint32_t w[4] = {u.x, u.y, u.z, u.w};
@@ -146,13 +153,42 @@ __global__ void __launch_bounds__(DecodeCfg<D>::THREADS)
   if (threadIdx.x == 0)
     for (; issued < C::STAGES - 1 && issued < nchunks; ++issued) issue(issued);
 
-  float m[R], l[R], o[R][8];
+  // q as packed pairs (columns 2k, 2k + 1 of this lane's 8).
+  uint64_t q2[R][4];
+#pragma unroll
+  for (int r = 0; r < R; ++r)
+#pragma unroll
+    for (int k = 0; k < 4; ++k) q2[r][k] = f32x2(q[r][2 * k], q[r][2 * k + 1]);
+
+  // Online-softmax state, the same on every lane of a key group: row max
+  // (log2 units), row sum, and this lane's 8 output columns as 4 pairs.
+  float m[R], l[R];
+  uint64_t o2[R][4];
 #pragma unroll
   for (int r = 0; r < R; ++r) {
     m[r] = -INFINITY;
     l[r] = 0.f;
 #pragma unroll
-    for (int c = 0; c < 8; ++c) o[r][c] = 0.f;
+    for (int k = 0; k < 4; ++k) o2[r][k] = f32x2(0.f, 0.f);
+  }
+
+  // A chunk gives each key group NV = STEPS * R partial dot products (index
+  // i = step * R + row).  They are summed over the group's LPK lanes by a
+  // reduce-scatter, after which lane c of the group holds the scores of
+  // indices c * VPL .. c * VPL + VPL - 1: one step, VPL consecutive rows.
+  constexpr int NV = C::STEPS * R;
+  constexpr int VPL = NV / C::LPK;       // 1 (d = 128) or 2 (d = 64)
+  constexpr int RPL = R / VPL;           // lanes per step in a group
+  static_assert(NV % C::LPK == 0 && R % VPL == 0 && RPL * C::STEPS == C::LPK, "lane map");
+  const int gbase = lane - col8;                       // first lane of this key group
+  const int own_step = col8 / RPL;
+  const int own_row0 = (col8 % RPL) * VPL;
+  int own_limit[VPL];
+#pragma unroll
+  for (int v = 0; v < VPL; ++v) {
+    const int rr = blockIdx.z * R + own_row0 + v;
+    const int iqv = rr < rows_total ? rr % p.Nq : 0;
+    own_limit[v] = p.causal ? min(L, L - p.Nq + iqv + 1) : L;
   }
 
   bool ok = true;
@@ -168,45 +204,87 @@ __global__ void __launch_bounds__(DecodeCfg<D>::THREADS)
     const uint8_t *ks = smem + s * 2 * C::CHUNK_BYTES;
     const uint8_t *vs = ks + C::CHUNK_BYTES;
     const int n_here = min(C::KEYS, nkeys - c * C::KEYS);  // keys copied into this stage
-    // Scores of this lane group's 8 keys (log2 units), masked to -inf.
-    float sc[C::STEPS][R];
+    // Partial dot products over this lane's 8 columns (packed FMA pairs).
+    float red[NV];
 #pragma unroll
     for (int st = 0; st < C::STEPS; ++st) {
       const int kl = st * C::KPS + warp * C::KPW + key_in_warp;  // key within the chunk
-      const int key = k0 + c * C::KEYS + kl;
       float kf[8];
       bf16x8_to_f32(*reinterpret_cast<const uint4 *>(ks + (kl * D + col8 * 8) * 2), kf);
+      uint64_t k2[4];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) k2[k] = f32x2(kf[2 * k], kf[2 * k + 1]);
 #pragma unroll
       for (int r = 0; r < R; ++r) {
-        float acc = 0.f;
+        uint64_t acc = fma_f32x2(q2[r][0], k2[0], f32x2(0.f, 0.f));
 #pragma unroll
-        for (int e = 0; e < 8; ++e) acc = fmaf(q[r][e], kf[e], acc);
-#pragma unroll
-        for (int off = C::LPK / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-        sc[st][r] = (key < k1 && key < limit[r]) ? acc * p.scale_log2 : -INFINITY;
+        for (int k = 1; k < 4; ++k) acc = fma_f32x2(q2[r][k], k2[k], acc);
+        float a0, a1;
+        f32x2_split(acc, a0, a1);
+        red[st * R + r] = a0 + a1;
       }
     }
-    // Online softmax over this block of 8 keys, then O += P V.
-    float pr[C::STEPS][R];
+    // Reduce-scatter over the key group: each level halves the values a lane
+    // keeps and adds its partner's matching half.
+#pragma unroll
+    for (int lev = 1; lev < C::LPK; lev <<= 1) {
+      const int mask = C::LPK / (2 * lev);
+      const int h = NV / (2 * lev);
+      const bool up = (col8 & mask) != 0;
+#pragma unroll
+      for (int i = 0; i < h; ++i) {
+        const float send = up ? red[i] : red[h + i];
+        const float keep = up ? red[h + i] : red[i];
+        red[i] = keep + __shfl_xor_sync(0xffffffffu, send, mask);
+      }
+    }
+    // This lane's scores (log2 units), masked to -inf past the range, the
+    // sequence or the causal limit of their row.
+    const int own_key = k0 + c * C::KEYS + own_step * C::KPS + warp * C::KPW + key_in_warp;
+    float sc[VPL], bm[VPL];
+#pragma unroll
+    for (int v = 0; v < VPL; ++v) {
+      sc[v] = (own_key < k1 && own_key < own_limit[v]) ? red[v] * p.scale_log2 : -INFINITY;
+      bm[v] = sc[v];
+    }
+    // Block max of each row over the group's steps, then on every lane.
+#pragma unroll
+    for (int sm = RPL; sm < C::LPK; sm <<= 1)
+#pragma unroll
+      for (int v = 0; v < VPL; ++v) bm[v] = fmaxf(bm[v], __shfl_xor_sync(0xffffffffu, bm[v], sm));
+    float m_use[R], alpha[R];
 #pragma unroll
     for (int r = 0; r < R; ++r) {
-      float mb = sc[0][r];
-#pragma unroll
-      for (int st = 1; st < C::STEPS; ++st) mb = fmaxf(mb, sc[st][r]);
-      const float m_new = fmaxf(m[r], mb);
-      const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
-      const float alpha = ex2_approx(m[r] - m_use);
-      float sum = 0.f;
-#pragma unroll
-      for (int st = 0; st < C::STEPS; ++st) {
-        pr[st][r] = ex2_approx(sc[st][r] - m_use);
-        sum += pr[st][r];
-      }
-      l[r] = l[r] * alpha + sum;
+      const float bmax = __shfl_sync(0xffffffffu, bm[r % VPL], gbase + r / VPL);
+      const float m_new = fmaxf(m[r], bmax);
+      m_use[r] = (m_new == -INFINITY) ? 0.f : m_new;
+      alpha[r] = ex2_approx(m[r] - m_use[r]);
       m[r] = m_new;
-#pragma unroll
-      for (int e = 0; e < 8; ++e) o[r][e] *= alpha;
     }
+    // Probabilities of this lane's scores; row sums over the steps.
+    float pw[VPL], ps[VPL];
+#pragma unroll
+    for (int v = 0; v < VPL; ++v) {
+      const int r = own_row0 + v;
+      const float mu = r == 0 ? m_use[0] : r == 1 ? m_use[1] : r == 2 ? m_use[2] : m_use[3];
+      pw[v] = ex2_approx(sc[v] - mu);
+      ps[v] = pw[v];
+    }
+#pragma unroll
+    for (int sm = RPL; sm < C::LPK; sm <<= 1)
+#pragma unroll
+      for (int v = 0; v < VPL; ++v) ps[v] += __shfl_xor_sync(0xffffffffu, ps[v], sm);
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+      const float psum = __shfl_sync(0xffffffffu, ps[r % VPL], gbase + r / VPL);
+      l[r] = l[r] * alpha[r] + psum;
+#pragma unroll
+      for (int k = 0; k < 4; ++k) o2[r][k] = mul_f32x2(o2[r][k], f32x2(alpha[r], alpha[r]));
+    }
+    // Every lane needs every probability of its group for O += P V.
+    float pa[NV];
+#pragma unroll
+    for (int i = 0; i < NV; ++i) pa[i] = __shfl_sync(0xffffffffu, pw[i % VPL], gbase + i / VPL);
 #pragma unroll
     for (int st = 0; st < C::STEPS; ++st) {
       const int kl = st * C::KPS + warp * C::KPW + key_in_warp;
@@ -216,10 +294,15 @@ __global__ void __launch_bounds__(DecodeCfg<D>::THREADS)
 #pragma unroll
         for (int e = 0; e < 8; ++e) vf[e] = 0.f;
       }
+      uint64_t v2[4];
 #pragma unroll
-      for (int r = 0; r < R; ++r)
+      for (int k = 0; k < 4; ++k) v2[k] = f32x2(vf[2 * k], vf[2 * k + 1]);
 #pragma unroll
-        for (int e = 0; e < 8; ++e) o[r][e] = fmaf(pr[st][r], vf[e], o[r][e]);
+      for (int r = 0; r < R; ++r) {
+        const uint64_t p2 = f32x2(pa[st * R + r], pa[st * R + r]);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) o2[r][k] = fma_f32x2(p2, v2[k], o2[r][k]);
+      }
     }
     __syncthreads();  // every thread is done with this stage before it is refilled
     if (threadIdx.x == 0 && issued < nchunks) issue(issued++);
@@ -232,6 +315,11 @@ __global__ void __launch_bounds__(DecodeCfg<D>::THREADS)
                         &never, nullptr, p.wait_limit_ns, 0);
   }
 
+  float o[R][8];
+#pragma unroll
+  for (int r = 0; r < R; ++r)
+#pragma unroll
+    for (int k = 0; k < 4; ++k) f32x2_split(o2[r][k], o[r][2 * k], o[r][2 * k + 1]);
   // Merge the lane groups of each warp (same columns, different keys), then
   // the warps through shared memory, then write the CTA's partial.
 #pragma unroll
