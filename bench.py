@@ -76,10 +76,11 @@ class ClockSampler:
     NVML does not).  Only samples taken between region_start() and
     region_stop() are reported; without NVML the record says so.  Reading
     only: nothing here changes a setting of the GPU."""
-    REASONS = (("hw_slowdown", "nvmlClocksEventReasonHwSlowdown"),
-               ("hw_thermal_slowdown", "nvmlClocksEventReasonHwThermalSlowdown"),
-               ("sw_thermal_slowdown", "nvmlClocksEventReasonSwThermalSlowdown"),
-               ("sw_power_cap", "nvmlClocksEventReasonSwPowerCap"))
+    # every clock-event reason bit NVML defines, by the name the report uses
+    REASONS = (("gpu_idle", 0x1), ("applications_clocks_setting", 0x2), ("sw_power_cap", 0x4),
+               ("hw_slowdown", 0x8), ("sync_boost", 0x10), ("sw_thermal_slowdown", 0x20),
+               ("hw_thermal_slowdown", 0x40), ("hw_power_brake_slowdown", 0x80),
+               ("display_clock_setting", 0x100))
 
     def __init__(self, torch_index: int):
         import threading
@@ -90,6 +91,7 @@ class ClockSampler:
         self.nvml = None
         self.handle = None
         self.max_mhz = None
+        self.instant_field = None
         try:
             import pynvml
             import torch
@@ -100,9 +102,23 @@ class ClockSampler:
             self.handle = pynvml.nvmlDeviceGetHandleByUUID(uuid)
             self.max_mhz = float(pynvml.nvmlDeviceGetMaxClockInfo(self.handle,
                                                                   pynvml.NVML_CLOCK_SM))
+            self.instant_field = getattr(pynvml, "NVML_FI_DEV_POWER_INSTANT", None)
             self.nvml = pynvml
         except Exception:
             self.nvml = None
+
+    def _power_w(self):
+        """Instantaneous board power where NVML offers it (the plain power
+        reading is averaged over about a second), else the averaged one."""
+        nv = self.nvml
+        if self.instant_field is not None:
+            try:
+                v = nv.nvmlDeviceGetFieldValues(self.handle, [self.instant_field])[0]
+                if v.nvmlReturn == nv.NVML_SUCCESS:
+                    return float(v.value.uiVal) / 1000.0
+            except Exception:
+                pass
+        return nv.nvmlDeviceGetPowerUsage(self.handle) / 1000.0
 
     def _run(self):
         nv = self.nvml
@@ -110,7 +126,7 @@ class ClockSampler:
             try:
                 t = time.monotonic()
                 sm = nv.nvmlDeviceGetClockInfo(self.handle, nv.NVML_CLOCK_SM)
-                pw = nv.nvmlDeviceGetPowerUsage(self.handle) / 1000.0
+                pw = self._power_w()
                 rs = nv.nvmlDeviceGetCurrentClocksEventReasons(self.handle)
                 self.samples.append((t, float(sm), pw, int(rs)))
             except Exception:
@@ -140,8 +156,8 @@ class ClockSampler:
             return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["no samples"]}
         reasons = set()
         for _, _, _, rs in inside:
-            for name, const in self.REASONS:
-                if rs & getattr(self.nvml, const):
+            for name, bit in self.REASONS:
+                if rs & bit:
                     reasons.add(name)
         sm = [x[1] for x in inside]
         pw = [x[2] for x in inside]
