@@ -65,8 +65,32 @@ def kernel_source_hash() -> str:
 
 
 def dist_env():
+    """(rank, world size, local rank) from the launcher's environment."""
     return (int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")),
             int(os.environ.get("LOCAL_RANK", "0")))
+
+
+def replica_seed(w: wl.Workload, rank: int) -> int:
+    """Each rank times its own replica of the workload, drawn from its own seed."""
+    return w.seed + 1000 * rank
+
+
+def reduce_max(x: float, device) -> float:
+    """Max of x over the ranks of the default process group (x itself
+    without one): the slowest rank sets the job's time."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(flops_per_step: float, steps: int, ms_max: float, world: int) -> float:
+    """Whole-job TFLOP/s: `world` replicas each ran `steps` steps in at most
+    ms_max milliseconds."""
+    return world * flops_per_step * steps / (ms_max * 1e-3) / 1e12
 
 
 class ClockSampler:
@@ -254,7 +278,7 @@ def run_mine(args, w: wl.Workload):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=dev)
     # Each rank: its own replica of the workload (seed offset by rank).
-    inp = wl.draw(w.B, w.Hq, w.Hkv, w.N, w.d, w.seed + 1000 * rank, k_scale=w.k_scale,
+    inp = wl.draw(w.B, w.Hq, w.Hkv, w.N, w.d, replica_seed(w, rank), k_scale=w.k_scale,
                   seqlen_range=w.seqlen_range)
     q, k, v = (torch.from_numpy(x).view(torch.bfloat16).to(dev)
                for x in (inp.q_bits, inp.k_bits, inp.v_bits))
@@ -298,13 +322,9 @@ def run_mine(args, w: wl.Workload):
     ms_total = start.elapsed_time(end)
     if attention.check_status(status) != 0:
         raise RuntimeError("kernel reported a time-out in the timed region")
-    ms_max = ms_total
-    if world > 1:
-        t = torch.tensor([ms_total], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_max = float(t.item())
+    ms_max = reduce_max(ms_total, dev)
     ms_per_step = ms_max / args.steps
-    value = world * flops * args.steps / (ms_max * 1e-3) / 1e12
+    value = job_throughput(flops, args.steps, ms_max, world)
     kernel_tflops = flops / (ms_total / args.steps * 1e-3) / 1e12
 
     # End to end through the C ABI on host buffers: pinned host inputs are
@@ -325,12 +345,8 @@ def run_mine(args, w: wl.Workload):
                              scale=w.scale, seqlens_h=sl_h, seqlens_d=sl)
     e1.record(stream)
     torch.cuda.synchronize(dev)
-    e2e_ms = e0.elapsed_time(e1)
-    if world > 1:
-        t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
-    e2e_value = world * flops * e2e_steps / (e2e_ms * 1e-3) / 1e12
+    e2e_ms = reduce_max(e0.elapsed_time(e1), dev)
+    e2e_value = job_throughput(flops, e2e_steps, e2e_ms, world)
     h2d = in_bytes + (0 if sl is None else sl.numel() * 4)
     d2h = o.numel() * 2 + lse.numel() * 4
 
