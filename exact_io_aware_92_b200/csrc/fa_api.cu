@@ -37,6 +37,11 @@ struct DeviceState {
   bool dec_attr64 = false, dec_attr128 = false;
   bool bwd_attr64 = false, bwd_attr128 = false;
   bool fp8_attr = false;
+  // fa_fwd_hostio's copy streams and per-slice events, created on first use
+  // and kept for the process's lifetime.
+  bool io_ready = false;
+  cudaStream_t io_in = nullptr, io_out = nullptr;
+  cudaEvent_t io_ev_in[16] = {}, io_ev_done[16] = {}, io_ev_end = nullptr;
 };
 DeviceState g_dev[kMaxDevices];
 std::mutex g_mu;
@@ -553,26 +558,92 @@ int fa_fwd_hostio(const void *q_h, const void *k_h, const void *v_h, void *o_h, 
   if (seqlens_h && !seqlens_d) return FA_ERR_NULL;
   int rc = check_args(q_d, k_d, v_d, o_d, lse_d, B, Hq, Hkv, N, d, scale);
   if (rc != FA_OK) return rc;
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  const size_t qn = static_cast<size_t>(B) * Hq * N * d * 2;
-  const size_t kn = static_cast<size_t>(B) * Hkv * N * d * 2;
-  const size_t ln = static_cast<size_t>(B) * Hq * N * sizeof(float);
-  if (cudaMemcpyAsync(q_d, q_h, qn, cudaMemcpyHostToDevice, st) != cudaSuccess ||
-      cudaMemcpyAsync(k_d, k_h, kn, cudaMemcpyHostToDevice, st) != cudaSuccess ||
-      cudaMemcpyAsync(v_d, v_h, kn, cudaMemcpyHostToDevice, st) != cudaSuccess ||
-      (seqlens_h && cudaMemcpyAsync(seqlens_d, seqlens_h, sizeof(int) * B,
-                                    cudaMemcpyHostToDevice, st) != cudaSuccess)) {
-    cudaGetLastError();
-    return FA_ERR_CUDA;
-  }
-  rc = fa_fwd_ex(q_d, k_d, v_d, o_d, lse_d, B, Hq, Hkv, N, d, scale, causal,
-                 seqlens_h ? seqlens_d : nullptr, FA_DTYPE_BF16, stream, nullptr);
+  DeviceState *ds = nullptr;
+  rc = current_device(&ds);
   if (rc != FA_OK) return rc;
-  if (cudaMemcpyAsync(o_h, o_d, qn, cudaMemcpyDeviceToHost, st) != cudaSuccess ||
-      cudaMemcpyAsync(lse_h, lse_d, ln, cudaMemcpyDeviceToHost, st) != cudaSuccess) {
+  {
+    std::lock_guard<std::mutex> lock(g_mu);
+    if (!ds->io_ready) {
+      bool ok = cudaStreamCreateWithFlags(&ds->io_in, cudaStreamNonBlocking) == cudaSuccess &&
+                cudaStreamCreateWithFlags(&ds->io_out, cudaStreamNonBlocking) == cudaSuccess &&
+                cudaEventCreateWithFlags(&ds->io_ev_end, cudaEventDisableTiming) == cudaSuccess;
+      for (int i = 0; ok && i < 16; ++i)
+        ok = cudaEventCreateWithFlags(&ds->io_ev_in[i], cudaEventDisableTiming) == cudaSuccess &&
+             cudaEventCreateWithFlags(&ds->io_ev_done[i], cudaEventDisableTiming) == cudaSuccess;
+      if (!ok) {
+        cudaGetLastError();
+        return FA_ERR_CUDA;
+      }
+      ds->io_ready = true;
+    }
+  }
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  // Slices run as problems of their own, so slice s's copies in and s-1's
+  // copies out overlap the forward of slice s.  Without key lengths a slice
+  // is a run of consecutive (batch, kv head) pairs -- contiguous in q, k, v,
+  // o and lse, and an attention problem of its own with batch = its kv heads
+  // and Hkv = 1; with key lengths it is a run of whole batches.
+  const int G = Hq / Hkv;
+  const int units = seqlens_h ? B : B * Hkv;            // indivisible pieces
+  const int nslices = units < 16 ? units : 16;
+  const size_t q_unit = static_cast<size_t>(seqlens_h ? Hq : G) * N * d;   // elements
+  const size_t k_unit = static_cast<size_t>(seqlens_h ? Hkv : 1) * N * d;
+  const size_t l_unit = static_cast<size_t>(seqlens_h ? Hq : G) * N;
+  auto bytes16 = [](const void *p, size_t off) {
+    return static_cast<const uint8_t *>(p) + off * 2;
+  };
+  auto fail = [&]() {
+    cudaGetLastError();
+    cudaStreamSynchronize(ds->io_in);
+    cudaStreamSynchronize(ds->io_out);
+    cudaStreamSynchronize(st);
     cudaGetLastError();
     return FA_ERR_CUDA;
+  };
+  // the slices' inputs must not be overwritten before earlier work on the
+  // caller's stream has finished with the device buffers
+  if (cudaEventRecord(ds->io_ev_end, st) != cudaSuccess ||
+      cudaStreamWaitEvent(ds->io_in, ds->io_ev_end, 0) != cudaSuccess)
+    return fail();
+  if (seqlens_h && cudaMemcpyAsync(seqlens_d, seqlens_h, sizeof(int) * B, cudaMemcpyHostToDevice,
+                                   ds->io_in) != cudaSuccess)
+    return fail();
+  for (int s = 0; s < nslices; ++s) {
+    const int u0 = static_cast<int>(static_cast<long long>(units) * s / nslices);
+    const int u1 = static_cast<int>(static_cast<long long>(units) * (s + 1) / nslices);
+    const int nu = u1 - u0;
+    const size_t qo = q_unit * u0, ko = k_unit * u0, lo = l_unit * u0;
+    if (cudaMemcpyAsync(const_cast<uint8_t *>(bytes16(q_d, qo)), bytes16(q_h, qo),
+                        q_unit * nu * 2, cudaMemcpyHostToDevice, ds->io_in) != cudaSuccess ||
+        cudaMemcpyAsync(const_cast<uint8_t *>(bytes16(k_d, ko)), bytes16(k_h, ko),
+                        k_unit * nu * 2, cudaMemcpyHostToDevice, ds->io_in) != cudaSuccess ||
+        cudaMemcpyAsync(const_cast<uint8_t *>(bytes16(v_d, ko)), bytes16(v_h, ko),
+                        k_unit * nu * 2, cudaMemcpyHostToDevice, ds->io_in) != cudaSuccess ||
+        cudaEventRecord(ds->io_ev_in[s], ds->io_in) != cudaSuccess ||
+        cudaStreamWaitEvent(st, ds->io_ev_in[s], 0) != cudaSuccess)
+      return fail();
+    rc = seqlens_h
+             ? fa_fwd_ex(bytes16(q_d, qo), bytes16(k_d, ko), bytes16(v_d, ko),
+                         const_cast<uint8_t *>(bytes16(o_d, qo)), lse_d + lo, nu, Hq, Hkv, N, d,
+                         scale, causal, seqlens_d + u0, FA_DTYPE_BF16, stream, nullptr)
+             : fa_fwd_ex(bytes16(q_d, qo), bytes16(k_d, ko), bytes16(v_d, ko),
+                         const_cast<uint8_t *>(bytes16(o_d, qo)), lse_d + lo, nu, G, 1, N, d,
+                         scale, causal, nullptr, FA_DTYPE_BF16, stream, nullptr);
+    if (rc != FA_OK) {
+      fail();
+      return rc;
+    }
+    if (cudaEventRecord(ds->io_ev_done[s], st) != cudaSuccess ||
+        cudaStreamWaitEvent(ds->io_out, ds->io_ev_done[s], 0) != cudaSuccess ||
+        cudaMemcpyAsync(const_cast<uint8_t *>(bytes16(o_h, qo)), bytes16(o_d, qo),
+                        q_unit * nu * 2, cudaMemcpyDeviceToHost, ds->io_out) != cudaSuccess ||
+        cudaMemcpyAsync(lse_h + lo, lse_d + lo, l_unit * nu * sizeof(float),
+                        cudaMemcpyDeviceToHost, ds->io_out) != cudaSuccess)
+      return fail();
   }
+  if (cudaEventRecord(ds->io_ev_end, ds->io_out) != cudaSuccess ||
+      cudaStreamWaitEvent(st, ds->io_ev_end, 0) != cudaSuccess)
+    return fail();
   return fa_check_status(nullptr, stream);
 }
 

@@ -116,7 +116,12 @@ FA_API int fa_fwd_f32(const float *q, const float *k, const float *v, float *o, 
 /*
  * End-to-end call on HOST buffers: copies q, k, v (and seqlens) from host to
  * the caller's device buffers, runs the bf16 forward and copies o and lse
- * back, all on `stream`, then waits for the stream.
+ * back, then waits.  The work runs in up to 16 slices so that copies overlap
+ * the forward: runs of consecutive (batch, kv head) pairs, or of whole
+ * batches when seqlens is given.  The copies go on two streams the library
+ * creates once per device; the forward runs on `stream`, which first waits
+ * for them.  Before the first copy the copy stream waits for work already
+ * queued on `stream`.
  *  q_h, k_h, v_h, o_h, lse_h, seqlens_h: host buffers (pinned memory gives
  *  asynchronous copies; seqlens_h may be NULL).
  *  q_d, k_d, v_d, o_d, lse_d, seqlens_d: device buffers of the same sizes
