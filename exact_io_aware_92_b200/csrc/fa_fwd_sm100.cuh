@@ -124,6 +124,8 @@ struct Sm100Cfg {
 // packed layout (0 otherwise).
 struct Unit {
   int b, h, hkv, bh, row0, L, nkv;
+  int nkv0;        // key tiles Q tile 0 needs: causal units skip a last tile
+                   // that lies wholly above tile 0's rows
   int q_rows;      // query rows that exist (N, or the sequence length when packed)
   int tok0;        // first token of the sequence (packed layout)
   int q_plane;     // TMA plane of Q: b*Hq+h, or h when packed
@@ -168,6 +170,7 @@ __device__ __forceinline__ Unit unit_at(const FwdParams &p, int u) {
   const int kv_end = p.causal ? min(L, x.row0 + C::ROWS_PER_UNIT) : L;
   // A unit past the end of its sequence (packed layout) has no rows at all.
   x.nkv = x.row0 < x.q_rows ? (kv_end + C::BN - 1) / C::BN : 0;
+  x.nkv0 = (p.causal && x.nkv > 1 && (x.nkv - 1) * C::BN >= x.row0 + C::BM) ? x.nkv - 1 : x.nkv;
   return x;
 }
 
@@ -363,16 +366,17 @@ __device__ void role_mma(const Sm100Ctx<D, F8> &x, const FwdParams &p) {
     return true;
   };
 
-  int g = 0;   // K/V tiles consumed by this CTA so far (ring and phase position)
-  int qi = 0;  // units with keys processed so far
+  int g = 0;             // K/V tiles consumed by this CTA so far (ring position)
+  int gs[2] = {0, 0};    // key tiles each Q tile has processed (its S/P phases)
+  int qi = 0;            // units with keys processed so far
   bool ok = true;
   for (int k = 0; ok; ++k) {
     const int u = snake_unit(k, p.num_units);
     if (u == -2) break;
     if (u < 0) continue;
     const Unit w = unit_at<D, F8>(p, u);
-    const int nkv = w.nkv;
-    if (nkv == 0) continue;
+    const int n1 = w.nkv, n0 = w.nkv0;  // n0 is n1 or n1 - 1
+    if (n1 == 0) continue;
     const uint32_t qpar = static_cast<uint32_t>(qi & 1);
     if (!wait(C::BAR_Q_FULL + 0, qpar) || !wait(C::BAR_Q_FULL + 1, qpar) ||
         !wait(C::BAR_KV_FULL + ring_slot<D, F8>(2 * g), ring_parity<D, F8>(2 * g))) {
@@ -383,27 +387,32 @@ __device__ void role_mma(const Sm100Ctx<D, F8> &x, const FwdParams &p) {
     // Tile 0: S for both Q tiles.
     issue_s(0, ring_slot<D, F8>(2 * g));
     commit(C::BAR_S_FULL + 0);
-    if (nkv == 1) commit(C::BAR_Q_EMPTY + 0);
+    if (n0 == 1) commit(C::BAR_Q_EMPTY + 0);
     issue_s(1, ring_slot<D, F8>(2 * g));
     commit(C::BAR_S_FULL + 1);
     commit(C::BAR_KV_EMPTY + ring_slot<D, F8>(2 * g));
-    if (nkv == 1) commit(C::BAR_Q_EMPTY + 1);
+    if (n1 == 1) commit(C::BAR_Q_EMPTY + 1);
     // Steady state: PV of tile j-1, then S of tile j into the same columns
     // (the tensor pipe runs them in order, so P is read before S lands).
-    for (int j = 1; j < nkv; ++j) {
+    // Q tile 0 stops after its n0 tiles.
+    for (int j = 1; j < n1; ++j) {
       const int gp = g + j - 1, gc = g + j;
-      const uint32_t pp = static_cast<uint32_t>(gp & 1);
       const int vs = ring_slot<D, F8>(2 * gp + 1), ks = ring_slot<D, F8>(2 * gc);
-      if (!wait(C::BAR_KV_FULL + vs, ring_parity<D, F8>(2 * gp + 1)) || !pv(0, vs, pp, j - 1 > 0) ||
+      if (!wait(C::BAR_KV_FULL + vs, ring_parity<D, F8>(2 * gp + 1)) ||
+          !pv(0, vs, static_cast<uint32_t>((gs[0] + j - 1) & 1), j - 1 > 0) ||
           !wait(C::BAR_KV_FULL + ks, ring_parity<D, F8>(2 * gc))) {
         ok = false;
         break;
       }
       tc_fence_after();
-      issue_s(0, ks);
-      commit(C::BAR_S_FULL + 0);
-      if (j == nkv - 1) commit(C::BAR_Q_EMPTY + 0);
-      if (!pv(1, vs, pp, j - 1 > 0)) {
+      if (j < n0) {
+        issue_s(0, ks);
+        commit(C::BAR_S_FULL + 0);
+        if (j == n0 - 1) commit(C::BAR_Q_EMPTY + 0);
+      } else {
+        commit(C::BAR_O_FULL + 0);  // Q tile 0's last PV was issued just above
+      }
+      if (!pv(1, vs, static_cast<uint32_t>((gs[1] + j - 1) & 1), j - 1 > 0)) {
         ok = false;
         break;
       }
@@ -411,25 +420,32 @@ __device__ void role_mma(const Sm100Ctx<D, F8> &x, const FwdParams &p) {
       issue_s(1, ks);
       commit(C::BAR_S_FULL + 1);
       commit(C::BAR_KV_EMPTY + ks);
-      if (j == nkv - 1) commit(C::BAR_Q_EMPTY + 1);
+      if (j == n1 - 1) commit(C::BAR_Q_EMPTY + 1);
     }
     if (!ok) break;
     // Last tile's PV products, then the unit's output is complete.
-    const int gl = g + nkv - 1;
+    const int gl = g + n1 - 1;
     const int vs = ring_slot<D, F8>(2 * gl + 1);
-    const uint32_t pp = static_cast<uint32_t>(gl & 1);
-    if (!wait(C::BAR_KV_FULL + vs, ring_parity<D, F8>(2 * gl + 1)) || !pv(0, vs, pp, nkv > 1)) {
+    if (!wait(C::BAR_KV_FULL + vs, ring_parity<D, F8>(2 * gl + 1))) {
       ok = false;
       break;
     }
-    commit(C::BAR_O_FULL + 0);
-    if (!pv(1, vs, pp, nkv > 1)) {
+    if (n0 == n1) {
+      if (!pv(0, vs, static_cast<uint32_t>((gs[0] + n1 - 1) & 1), n1 > 1)) {
+        ok = false;
+        break;
+      }
+      commit(C::BAR_O_FULL + 0);
+    }
+    if (!pv(1, vs, static_cast<uint32_t>((gs[1] + n1 - 1) & 1), n1 > 1)) {
       ok = false;
       break;
     }
     commit(C::BAR_O_FULL + 1);
     commit(C::BAR_KV_EMPTY + vs);
-    g += nkv;
+    g += n1;
+    gs[0] += n0;
+    gs[1] += n1;
     ++qi;
   }
   // Every MMA issued above must finish before tensor memory is released.
@@ -477,10 +493,11 @@ __device__ void role_softmax(const Sm100Ctx<D, F8> &x, const FwdParams &p, int t
       continue;
     }
     const int limit = p.causal ? min(w.L, i + 1) : w.L;  // visible keys are [0, limit)
+    const int nkv_t = t == 0 ? w.nkv0 : w.nkv;            // key tiles this Q tile needs
 
     float m_ref = -INFINITY;  // reference max (log2 units) the exponentials use
     float l = 0.f;            // row sum of the fp32 probabilities relative to m_ref
-    for (int j = 0; j < w.nkv; ++j) {
+    for (int j = 0; j < nkv_t; ++j) {
       if (!wait_all(C::BAR_S_FULL + t, static_cast<uint32_t>((g + j) & 1))) return;
       tc_fence_after();
       uint32_t s[128];
@@ -639,7 +656,7 @@ __device__ void role_softmax(const Sm100Ctx<D, F8> &x, const FwdParams &p, int t
       p.lse[w.lse_base + i] =
           l > 0.f ? (m_lse + __log2f(l)) * 0.69314718055994530942f : -INFINITY;
     }
-    g += w.nkv;
+    g += nkv_t;
     ++qi;
   }
 }
