@@ -1,0 +1,61 @@
+"""bench.ClockSampler against a fake NVML (no GPU, nothing real is queried).
+
+The sampler must look the device up by the UUID torch reports, keep only
+the samples taken inside the timed region, decode every clock-event reason
+bit, and prefer the instantaneous power field."""
+import sys
+import time
+import types
+
+import bench
+
+
+class _Field:
+    def __init__(self, value):
+        self.nvmlReturn = 0
+        self.value = types.SimpleNamespace(uiVal=value)
+
+
+def _fake_nvml(state):
+    nv = types.ModuleType("pynvml")
+    nv.NVML_CLOCK_SM = 1
+    nv.NVML_SUCCESS = 0
+    nv.NVML_FI_DEV_POWER_INSTANT = 186
+    nv.nvmlInit = lambda: None
+    nv.nvmlDeviceGetHandleByUUID = lambda uuid: state.setdefault("uuid", uuid) and "handle"
+    nv.nvmlDeviceGetMaxClockInfo = lambda h, c: 1965
+    nv.nvmlDeviceGetClockInfo = lambda h, c: 1500 if state["busy"] else 600
+    nv.nvmlDeviceGetPowerUsage = lambda h: 123000
+    nv.nvmlDeviceGetFieldValues = lambda h, ids: [_Field(990000 if state["busy"] else 90000)]
+    nv.nvmlDeviceGetCurrentClocksEventReasons = lambda h: (0x4 | 0x8) if state["busy"] else 0x1
+    return nv
+
+
+def test_sampler_keeps_the_timed_region_and_decodes_reasons(monkeypatch):
+    import torch
+    state = {"busy": False}
+    monkeypatch.setitem(sys.modules, "pynvml", _fake_nvml(state))
+    monkeypatch.setattr(torch.cuda, "get_device_properties",
+                        lambda i: types.SimpleNamespace(uuid="1234-abcd"))
+    s = bench.ClockSampler(0)
+    assert s.nvml is not None and state["uuid"] == "GPU-1234-abcd"
+    s.start()
+    time.sleep(0.06)                 # idle samples before the region
+    state["busy"] = True
+    s.region_start()
+    time.sleep(0.12)
+    s.region_stop()
+    state["busy"] = False
+    time.sleep(0.06)                 # idle samples after it
+    rec = s.stop()
+    assert rec["samples"] >= 3
+    assert rec["sm_mhz"] == 1500.0 and rec["sm_mhz_min"] == 1500.0
+    assert rec["sm_max_mhz"] == 1965.0
+    assert rec["reasons"] == ["hw_slowdown", "sw_power_cap"]   # gpu_idle stays outside
+    assert rec["power_w_median"] == 990.0 and rec["power_w_max"] == 990.0
+
+
+def test_sampler_without_nvml_says_so(monkeypatch):
+    monkeypatch.setitem(sys.modules, "pynvml", None)  # import fails
+    rec = bench.ClockSampler(0).stop()
+    assert rec["sm_mhz"] is None and rec["reasons"] == ["nvml unavailable"]
