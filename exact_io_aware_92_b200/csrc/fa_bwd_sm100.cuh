@@ -486,37 +486,69 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
       if (leader) tc_commit(bar);
       __syncwarp();
     };
-    if (wait(bar_q, 0)) {
-      for (int j = 0; j < nkv; ++j) {
-        const int st = j % C::Q_STAGES;
-        if (!wait(bar_full + 8 * st, (j / C::Q_STAGES) & 1)) break;
-        tc_fence_after();
-        const uint32_t stage = base + C::OFF_KVRING + st * C::KVSTAGE_BYTES;
-        const uint64_t dKk = smem_desc_sw128(stage, 16, 1024);
-        const uint64_t dVk = smem_desc_sw128(stage + C::TILE_BYTES, 16, 1024);
+    // S(j) goes to columns COL_A (even j) or COL_D (odd j), so S(j + 2) is
+    // issued right behind dQ(j) and only dP(j + 1) stands between one
+    // elementwise step and the next.
+    auto sbuf = [&](int jj) { return (jj & 1) ? C::COL_D : C::COL_A; };
+    auto stage_of = [&](int jj) {
+      return base + C::OFF_KVRING + (jj % C::Q_STAGES) * C::KVSTAGE_BYTES;
+    };
+    auto wait_full = [&](int jj) {
+      return wait(bar_full + 8 * (jj % C::Q_STAGES), (jj / C::Q_STAGES) & 1);
+    };
+    auto issue_s = [&](int jj) {  // S = Q K^T
+      const uint64_t dKk = smem_desc_sw128(stage_of(jj), 16, 1024);
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = ((kk / 4) * C::HALF_BYTES + (kk % 4) * 32) >> 4;
-          if (leader) tc_mma_ss(tmem + C::COL_A, dQk + off, dKk + off, IDESC_SS, kk > 0);
-        }
+      for (int kk = 0; kk < D / 16; ++kk) {
+        const uint32_t off = ((kk / 4) * C::HALF_BYTES + (kk % 4) * 32) >> 4;
+        if (leader) tc_mma_ss(tmem + sbuf(jj), dQk + off, dKk + off, IDESC_SS, kk > 0);
+      }
+      __syncwarp();
+    };
+    auto issue_dp = [&](int jj) {  // dP = dO V^T
+      const uint64_t dVk = smem_desc_sw128(stage_of(jj) + C::TILE_BYTES, 16, 1024);
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = ((kk / 4) * C::HALF_BYTES + (kk % 4) * 32) >> 4;
-          if (leader) tc_mma_ss(tmem + C::COL_B, dOk + off, dVk + off, IDESC_SS, kk > 0);
+      for (int kk = 0; kk < D / 16; ++kk) {
+        const uint32_t off = ((kk / 4) * C::HALF_BYTES + (kk % 4) * 32) >> 4;
+        if (leader) tc_mma_ss(tmem + C::COL_B, dOk + off, dVk + off, IDESC_SS, kk > 0);
+      }
+      __syncwarp();
+    };
+    bool ok = wait(bar_q, 0) && wait_full(0);
+    if (ok) {
+      tc_fence_after();
+      issue_s(0);
+      issue_dp(0);
+      commit(bar_sd);
+      if (nkv > 1) {
+        ok = wait_full(1);
+        if (ok) {
+          tc_fence_after();
+          issue_s(1);
         }
-        __syncwarp();
+      }
+    }
+    for (int j = 0; ok && j < nkv; ++j) {
+      if (!wait(bar_ds, j & 1)) break;
+      tc_fence_after();
+      // dP's columns are free again; stage j + 1 is full (waited for S(j + 1)).
+      if (j + 1 < nkv) {
+        issue_dp(j + 1);
         commit(bar_sd);
-        if (!wait(bar_ds, j & 1)) break;
-        tc_fence_after();
-        // dQ += dS K: K = 128 keys in steps of 16, K read MN-major.
-        const uint64_t dKm = smem_desc_sw128(stage, C::HALF_BYTES, 1024);
+      }
+      // dQ += dS K: K = 128 keys in steps of 16, K read MN-major.
+      const uint64_t dKm = smem_desc_sw128(stage_of(j), C::HALF_BYTES, 1024);
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          if (leader)
-            tc_mma_ts(tmem + C::COL_C, tmem + C::COL_A + C::a_col(kk), dKm + ((kk * 2048) >> 4),
-                      IDESC_TS, (j > 0 || kk > 0) ? 1u : 0u);
-        __syncwarp();
-        commit(bar_empty + 8 * st);
+      for (int kk = 0; kk < 8; ++kk)
+        if (leader)
+          tc_mma_ts(tmem + C::COL_C, tmem + sbuf(j) + C::a_col(kk), dKm + ((kk * 2048) >> 4),
+                    IDESC_TS, (j > 0 || kk > 0) ? 1u : 0u);
+      __syncwarp();
+      commit(bar_empty + 8 * (j % C::Q_STAGES));
+      if (j + 2 < nkv) {
+        if (!wait_full(j + 2)) break;
+        tc_fence_after();
+        issue_s(j + 2);  // behind dQ(j), which reads dS(j) in the same columns
       }
     }
     commit(bar_done);
@@ -527,7 +559,6 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
     const int e = warp >> 2;
     const int i = row0 + (threadIdx.x & 127);
     const uint32_t lane_base = static_cast<uint32_t>(warp & 3) * 32u << 16;
-    const uint32_t tA = tmem + lane_base + C::COL_A + 64 * e;
     const uint32_t tB = tmem + lane_base + C::COL_B + 64 * e;
     const size_t vrow = static_cast<size_t>(bh) * p.Npad + i;
     const float lse2 = p.ws_lse2[vrow];
@@ -542,6 +573,8 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
         break;
       }
       tc_fence_after();
+      // S(j) sits in the columns of its parity (COL_A or COL_D)
+      const uint32_t tA = tmem + lane_base + ((j & 1) ? C::COL_D : C::COL_A) + 64 * e;
       {
         uint32_t sv[64], dp[64];
         tmem_ld32(tA, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
