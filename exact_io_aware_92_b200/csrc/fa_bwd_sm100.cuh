@@ -153,9 +153,13 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
   const uint32_t bar_kv = base + C::OFF_BAR_KV;         // K, V loaded
   const uint32_t bar_full = bar_kv + 8;                  // [KV_STAGES]
   const uint32_t bar_empty = bar_full + 8 * C::KV_STAGES;  // [KV_STAGES]
-  const uint32_t bar_st = bar_empty + 8 * C::KV_STAGES;  // S^T and dP^T in TMEM
-  const uint32_t bar_pds = bar_st + 8;                   // P^T and dS^T in TMEM
-  const uint32_t bar_done = bar_pds + 8;                 // all products finished
+  // Each 128-query step runs as two halves of 64 queries; half gh uses
+  // tensor-memory buffer gh & 1 (S^T at columns 128b, dP^T at 128b + 64) and
+  // that buffer's own pair of barriers, so a barrier's next phase needs
+  // products issued only after its previous one was consumed.
+  const uint32_t bar_st = bar_empty + 8 * C::KV_STAGES;  // [2]: S^T and dP^T of a half in TMEM
+  const uint32_t bar_pds = bar_st + 16;                  // [2]: P^T and dS^T of a half in TMEM
+  const uint32_t bar_done = bar_pds + 16;                // all products finished
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + C::OFF_BAR_KV + 120);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + C::OFF_BAR_KV + 124);
 
@@ -165,8 +169,10 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
       mbar_init(bar_full + 8 * s, 1);
       mbar_init(bar_empty + 8 * s, 1);
     }
-    mbar_init(bar_st, 1);
-    mbar_init(bar_pds, 256);
+    for (int b2 = 0; b2 < 2; ++b2) {
+      mbar_init(bar_st + 8 * b2, 1);
+      mbar_init(bar_pds + 8 * b2, 256);
+    }
     mbar_init(bar_done, 1);
     *abort_flag = 0;
     fence_barrier_init();
@@ -216,7 +222,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
   } else if (nsteps > 0 && warp == 9) {
     // --- MMA issuer ---
     const bool leader = elect_one();
-    constexpr uint32_t IDESC_SS = idesc_bf16_f32(128, 128, 0, 0);  // K-major A and B
+    constexpr uint32_t IDESC_SS = idesc_bf16_f32(128, 64, 0, 0);   // K-major A and B, 64 queries
     constexpr uint32_t IDESC_TS = idesc_bf16_f32(128, D, 0, 1);    // A in TMEM, B MN-major
     const uint64_t dK = smem_desc_sw128(base + C::OFF_K, 16, 1024);
     const uint64_t dV = smem_desc_sw128(base + C::OFF_V, 16, 1024);
@@ -229,70 +235,99 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
       if (leader) tc_commit(bar);
       __syncwarp();
     };
-    if (wait(bar_kv, 0)) {
-      for (int s = 0; s < nsteps; ++s) {
-        const int st = s % C::KV_STAGES;
-        if (!wait(bar_full + 8 * st, (s / C::KV_STAGES) & 1)) break;
-        tc_fence_after();
-        const uint32_t stage = base + C::OFF_RING + st * C::STAGE_BYTES;
-        const uint64_t dQk = smem_desc_sw128(stage, 16, 1024);
-        const uint64_t dOk = smem_desc_sw128(stage + C::TILE_BYTES, 16, 1024);
-        // S^T = K Q^T and dP^T = V dO^T (K = d in steps of 16).
+    auto stage_addr = [&](int st_step) {
+      return base + C::OFF_RING + (st_step % C::KV_STAGES) * C::STAGE_BYTES;
+    };
+    auto wait_full = [&](int st_step) {
+      return wait(bar_full + 8 * (st_step % C::KV_STAGES), (st_step / C::KV_STAGES) & 1);
+    };
+    // S^T = K Q_h^T and dP^T = V dO_h^T for half gh (64 queries; query row 64
+    // starts 8 swizzle atoms into each box), K = d in steps of 16.
+    auto issue_sdp = [&](int gh) {
+      const uint32_t stage = stage_addr(gh >> 1), rows = (gh & 1) * 8192u;
+      const uint64_t dQk = smem_desc_sw128(stage + rows, 16, 1024);
+      const uint64_t dOk = smem_desc_sw128(stage + C::TILE_BYTES + rows, 16, 1024);
+      const uint32_t colS = (gh & 1) * 128u;
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = ((kk / 4) * C::HALF_BYTES + (kk % 4) * 32) >> 4;
-          if (leader) tc_mma_ss(tmem + C::COL_A, dK + off, dQk + off, IDESC_SS, kk > 0);
-        }
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = ((kk / 4) * C::HALF_BYTES + (kk % 4) * 32) >> 4;
-          if (leader) tc_mma_ss(tmem + C::COL_B, dV + off, dOk + off, IDESC_SS, kk > 0);
-        }
-        __syncwarp();
-        commit(bar_st);
-        if (!wait(bar_pds, s & 1)) break;
-        tc_fence_after();
-        // dV += P^T dO, dK += dS^T Q: K = 128 queries in steps of 16; the
-        // right operand is the tile read MN-major (queries as rows).
-        const uint64_t dOm = smem_desc_sw128(stage + C::TILE_BYTES, C::HALF_BYTES, 1024);
-        const uint64_t dQm = smem_desc_sw128(stage, C::HALF_BYTES, 1024);
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          if (leader) {
-            tc_mma_ts(tmem + C::COL_D, tmem + C::COL_A + C::a_col(kk), dOm + ((kk * 2048) >> 4),
-                      IDESC_TS, (s > 0 || kk > 0) ? 1u : 0u);
-            tc_mma_ts(tmem + C::COL_C, tmem + C::COL_B + C::a_col(kk), dQm + ((kk * 2048) >> 4),
-                      IDESC_TS, (s > 0 || kk > 0) ? 1u : 0u);
-          }
-        }
-        __syncwarp();
-        commit(bar_empty + 8 * st);
+      for (int kk = 0; kk < D / 16; ++kk) {
+        const uint32_t off = ((kk / 4) * C::HALF_BYTES + (kk % 4) * 32) >> 4;
+        if (leader) tc_mma_ss(tmem + colS, dK + off, dQk + off, IDESC_SS, kk > 0);
       }
+#pragma unroll
+      for (int kk = 0; kk < D / 16; ++kk) {
+        const uint32_t off = ((kk / 4) * C::HALF_BYTES + (kk % 4) * 32) >> 4;
+        if (leader) tc_mma_ss(tmem + colS + 64, dV + off, dOk + off, IDESC_SS, kk > 0);
+      }
+      __syncwarp();
+    };
+    // dV += P^T dO_h, dK += dS^T Q_h: K = 64 queries in steps of 16; the right
+    // operand is the tile read MN-major (queries as rows).  The warpgroups'
+    // bf16 halves sit at columns 0-15 and 32-47 of S^T (and of dP^T).
+    auto issue_ts = [&](int gh) {
+      const uint32_t stage = stage_addr(gh >> 1), rows = (gh & 1) * 8192u;
+      const uint64_t dOm = smem_desc_sw128(stage + C::TILE_BYTES + rows, C::HALF_BYTES, 1024);
+      const uint64_t dQm = smem_desc_sw128(stage + rows, C::HALF_BYTES, 1024);
+      const uint32_t colS = (gh & 1) * 128u;
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk) {
+        const uint32_t a = 8u * kk + (kk >= 2 ? 16u : 0u);
+        if (leader) {
+          tc_mma_ts(tmem + C::COL_D, tmem + colS + a, dOm + ((kk * 2048) >> 4), IDESC_TS,
+                    (gh > 0 || kk > 0) ? 1u : 0u);
+          tc_mma_ts(tmem + C::COL_C, tmem + colS + 64 + a, dQm + ((kk * 2048) >> 4), IDESC_TS,
+                    (gh > 0 || kk > 0) ? 1u : 0u);
+        }
+      }
+      __syncwarp();
+    };
+    const int nhalves = 2 * nsteps;
+    bool ok = wait(bar_kv, 0) && wait_full(0);
+    if (ok) {
+      tc_fence_after();
+      issue_sdp(0);
+      commit(bar_st);
+    }
+    for (int gh = 0; ok && gh < nhalves; ++gh) {
+      // The next half's products go into the other buffer while this half's
+      // P^T and dS^T are formed (that buffer's last readers, half gh - 1's
+      // products, were issued before).
+      const int nx = gh + 1;
+      if (nx < nhalves) {
+        if ((nx & 1) == 0) {
+          if (!wait_full(nx >> 1)) break;
+          tc_fence_after();
+        }
+        issue_sdp(nx);
+        commit(bar_st + 8 * (nx & 1));
+      }
+      if (!wait(bar_pds + 8 * (gh & 1), (gh >> 1) & 1)) break;
+      tc_fence_after();
+      issue_ts(gh);
+      if (gh & 1) commit(bar_empty + 8 * ((gh >> 1) % C::KV_STAGES));
     }
     commit(bar_done);
     volatile int never = 0;
     mbar_wait_bounded(bar_done, 0, &never, p.status, p.wait_limit_ns, kErrTimeout);
   } else if (warp < 8) {
-    // --- elementwise warpgroups: thread = key row, warpgroup e = query
-    // columns [64e, 64e + 64) ---
+    // --- elementwise warpgroups: thread = key row; in each 64-query half,
+    // warpgroup e takes queries [32e, 32e + 32) ---
     const int e = warp >> 2;
     const int j = key0 + (threadIdx.x & 127);
     const uint32_t lane_base = static_cast<uint32_t>(warp & 3) * 32u << 16;
-    const uint32_t tA = tmem + lane_base + C::COL_A + 64 * e;
-    const uint32_t tB = tmem + lane_base + C::COL_B + 64 * e;
     const bool key_ok = j < L;
     bool ok = true;
-    for (int s = 0; s < nsteps && ok; ++s) {
+    for (int gh = 0; gh < 2 * nsteps && ok; ++gh) {
+      const int s = gh >> 1, hq = gh & 1;
       const int st = s % C::KV_STAGES;
-      const bool got = mbar_wait_bounded(bar_st, s & 1, abort_flag, p.status, p.wait_limit_ns,
-                                         kErrTimeout);
+      const bool got = mbar_wait_bounded(bar_st + 8 * hq, (gh >> 1) & 1, abort_flag, p.status,
+                                         p.wait_limit_ns, kErrTimeout);
       if (!__all_sync(0xffffffffu, got)) {
         ok = false;
         break;
       }
       // The per-row vectors came with the stage's bulk copies: observe that
-      // stage's fill directly (it is refilled only after this step's P^T and
-      // dS^T are published, so the phase cannot have moved on).
+      // stage's fill directly (it is refilled only after this step's second
+      // half is consumed, so the phase cannot have moved on).
       const bool filled = mbar_wait_bounded(bar_full + 8 * st, (s / C::KV_STAGES) & 1, abort_flag,
                                             p.status, p.wait_limit_ns, kErrTimeout);
       if (!__all_sync(0xffffffffu, filled)) {
@@ -300,24 +335,24 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
         break;
       }
       tc_fence_after();
+      const int c0 = 64 * hq + 32 * e;  // first query column of this thread's block
       const int q0 = step_qt(s) * 128;
       const float *lse2 =
           reinterpret_cast<const float *>(smem + C::OFF_RING + st * C::STAGE_BYTES + 2 * C::TILE_BYTES);
       const float *delta = lse2 + 128;
+      const uint32_t tS = tmem + lane_base + hq * 128 + 32 * e;
       {
-        uint32_t sv[64], dp[64];
-        tmem_ld32(tA, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
-        tmem_ld32(tA + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
-        tmem_ld32(tB, *reinterpret_cast<uint32_t(*)[32]>(&dp[0]));
-        tmem_ld32(tB + 32, *reinterpret_cast<uint32_t(*)[32]>(&dp[32]));
+        uint32_t sv[32], dp[32];
+        tmem_ld32(tS, sv);
+        tmem_ld32(tS + 64, dp);
         tmem_wait_ld();
-        uint32_t pk[32], dk[32];
+        uint32_t pk[16], dk[16];
 #pragma unroll
-        for (int x = 0; x < 32; ++x) {
+        for (int x = 0; x < 16; ++x) {
           float pv[2], dv[2];
 #pragma unroll
           for (int u = 0; u < 2; ++u) {
-            const int c = 64 * e + 2 * x + u;  // query column within the tile
+            const int c = c0 + 2 * x + u;  // query column within the tile
             const int i = q0 + c;
             const bool vis = key_ok && (!p.causal || i >= j);
             const float pp = vis ? ex2_approx(fmaf(__uint_as_float(sv[2 * x + u]), p.scale_log2,
@@ -329,13 +364,13 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
           pk[x] = pack_bf16x2(pv[0], pv[1]);
           dk[x] = pack_bf16x2(dv[0], dv[1]);
         }
-        // P^T over the first 32 of this warpgroup's S^T columns, dS^T over dP^T's.
-        tmem_st32(tA, pk);
-        tmem_st32(tB, dk);
+        // P^T over the first 16 of this block's 32 S^T columns, dS^T over dP^T's.
+        tmem_st16(tS, pk);
+        tmem_st16(tS + 64, dk);
       }
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(bar_pds);
+      mbar_arrive(bar_pds + 8 * hq);
     }
     // Epilogue: dK = scale * sum dS^T Q (warpgroup 0), dV = sum P^T dO
     // (warpgroup 1), in bf16.
