@@ -10,19 +10,24 @@
 //                      to whole 128-row tiles (padding: D = 0, LSE = +inf).
 // fa_bwd_dkdv_kernel   one CTA per 128-key tile of one (batch, kv head); it
 //                      walks the query tiles of every query head of the
-//                      group.  Per query tile:  S^T = K Q^T, dP^T = V dO^T
-//                      (tcgen05, TMEM); the softmax warpgroup (thread = key
-//                      row = TMEM lane) forms P^T and dS^T in bf16 over those
-//                      TMEM columns; then dV += P^T dO and dK += dS^T Q with
-//                      the left operand read from TMEM.
-// fa_bwd_dq_kernel     one CTA per 128-row query tile; per key tile:
-//                      S = Q K^T, dP = dO V^T, dS in bf16 over S, dQ += dS K.
+//                      group, each as two halves of 64 queries.  Per half:
+//                      S^T = K Q_h^T, dP^T = V dO_h^T (tcgen05, TMEM); the
+//                      elementwise warpgroups (thread = key row = TMEM lane)
+//                      form P^T and dS^T in bf16 over those TMEM columns; then
+//                      dV += P^T dO_h and dK += dS^T Q_h with the left operand
+//                      read from TMEM.
+// fa_bwd_dq_kernel     one CTA per 128-row query tile; per key tile, as two
+//                      halves of 64 keys: S = Q K_h^T, dP = dO V_h^T, dS in
+//                      bf16 over S, dQ += dS K_h.
+// Halves alternate between two tensor-memory buffers (S or S^T at columns
+// 128b, dP or dP^T at 128b + 64), each with its own pair of barriers, so the
+// next half's products run while the elementwise warps work on this one.
 // Both tcgen05 kernels use 320 threads: warps 0-7 elementwise work in two
-// warpgroups (each takes 64 of the tile's 128 columns: thread = TMEM lane,
+// warpgroups (each takes 32 of a half's 64 columns: thread = TMEM lane,
 // warp w reaches lanes 32*(w%4)), warp 8 TMA producer, warp 9 MMA issuer
-// (one elected lane).  A warpgroup writes its bf16 P or dS over the first 32
-// of its own 64 columns (columns 0-31 and 64-95), so neither overwrites
-// scores the other has not read yet.  Every wait is bounded.
+// (one elected lane).  A warpgroup writes its bf16 P or dS over the first 16
+// of its own 32 columns (columns 0-15 and 32-47 of the buffer), so neither
+// overwrites scores the other has not read yet.  Every wait is bounded.
 #pragma once
 
 #include <cstdint>
@@ -50,10 +55,6 @@ struct BwdCfg {
   static constexpr int HALF_BYTES = 128 * 64 * 2;
   static constexpr int TILE_BYTES = 128 * D * 2;
   static constexpr int THREADS = 320;
-  // TMEM column of the bf16 left operand for K step kk (16 rows of the
-  // product's K dimension, 8 columns): the two warpgroups' halves sit at
-  // columns 0-31 and 64-95.
-  __host__ __device__ static constexpr uint32_t a_col(int kk) { return 8u * kk + (kk >= 4 ? 32u : 0u); }
   static constexpr uint32_t COL_A = 0, COL_B = 128, COL_C = 256, COL_D = 384;
   // dK/dV kernel: K, V resident; ring of (Q, dO, LSE2, D) stages.
   static constexpr int KV_STAGES = 2;
@@ -455,9 +456,12 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
   const uint32_t bar_q = base + C::OFF_BAR_Q;
   const uint32_t bar_full = bar_q + 8;
   const uint32_t bar_empty = bar_full + 8 * C::Q_STAGES;
-  const uint32_t bar_sd = bar_empty + 8 * C::Q_STAGES;  // S and dP in TMEM
-  const uint32_t bar_ds = bar_sd + 8;                    // dS in TMEM
-  const uint32_t bar_done = bar_ds + 8;
+  // Each 128-key tile runs as two halves of 64 keys; half gh uses
+  // tensor-memory buffer gh & 1 (S at columns 128b, dP at 128b + 64; dQ at
+  // 256) and that buffer's own pair of barriers.
+  const uint32_t bar_sd = bar_empty + 8 * C::Q_STAGES;  // [2]: S and dP of a half in TMEM
+  const uint32_t bar_ds = bar_sd + 16;                   // [2]: dS of a half in TMEM
+  const uint32_t bar_done = bar_ds + 16;
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + C::OFF_BAR_Q + 120);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + C::OFF_BAR_Q + 124);
 
@@ -467,8 +471,10 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
       mbar_init(bar_full + 8 * s, 1);
       mbar_init(bar_empty + 8 * s, 1);
     }
-    mbar_init(bar_sd, 1);
-    mbar_init(bar_ds, 256);
+    for (int b2 = 0; b2 < 2; ++b2) {
+      mbar_init(bar_sd + 8 * b2, 1);
+      mbar_init(bar_ds + 8 * b2, 256);
+    }
     mbar_init(bar_done, 1);
     *abort_flag = 0;
     fence_barrier_init();
@@ -508,7 +514,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
     }
   } else if (nkv > 0 && warp == 9) {
     const bool leader = elect_one();
-    constexpr uint32_t IDESC_SS = idesc_bf16_f32(128, 128, 0, 0);
+    constexpr uint32_t IDESC_SS = idesc_bf16_f32(128, 64, 0, 0);  // 64 keys per half
     constexpr uint32_t IDESC_TS = idesc_bf16_f32(128, D, 0, 1);
     const uint64_t dQk = smem_desc_sw128(base + C::OFF_Q, 16, 1024);
     const uint64_t dOk = smem_desc_sw128(base + C::OFF_DO, 16, 1024);
@@ -521,109 +527,107 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
       if (leader) tc_commit(bar);
       __syncwarp();
     };
-    // S(j) goes to columns COL_A (even j) or COL_D (odd j), so S(j + 2) is
-    // issued right behind dQ(j) and only dP(j + 1) stands between one
-    // elementwise step and the next.
-    auto sbuf = [&](int jj) { return (jj & 1) ? C::COL_D : C::COL_A; };
     auto stage_of = [&](int jj) {
       return base + C::OFF_KVRING + (jj % C::Q_STAGES) * C::KVSTAGE_BYTES;
     };
     auto wait_full = [&](int jj) {
       return wait(bar_full + 8 * (jj % C::Q_STAGES), (jj / C::Q_STAGES) & 1);
     };
-    auto issue_s = [&](int jj) {  // S = Q K^T
-      const uint64_t dKk = smem_desc_sw128(stage_of(jj), 16, 1024);
+    // S = Q K_h^T and dP = dO V_h^T for half gh (64 keys; key row 64 starts
+    // 8 swizzle atoms into each box), K = d in steps of 16.
+    auto issue_sdp = [&](int gh) {
+      const uint32_t stage = stage_of(gh >> 1), rows = (gh & 1) * 8192u;
+      const uint64_t dKk = smem_desc_sw128(stage + rows, 16, 1024);
+      const uint64_t dVk = smem_desc_sw128(stage + C::TILE_BYTES + rows, 16, 1024);
+      const uint32_t colS = (gh & 1) * 128u;
 #pragma unroll
       for (int kk = 0; kk < D / 16; ++kk) {
         const uint32_t off = ((kk / 4) * C::HALF_BYTES + (kk % 4) * 32) >> 4;
-        if (leader) tc_mma_ss(tmem + sbuf(jj), dQk + off, dKk + off, IDESC_SS, kk > 0);
+        if (leader) tc_mma_ss(tmem + colS, dQk + off, dKk + off, IDESC_SS, kk > 0);
       }
-      __syncwarp();
-    };
-    auto issue_dp = [&](int jj) {  // dP = dO V^T
-      const uint64_t dVk = smem_desc_sw128(stage_of(jj) + C::TILE_BYTES, 16, 1024);
 #pragma unroll
       for (int kk = 0; kk < D / 16; ++kk) {
         const uint32_t off = ((kk / 4) * C::HALF_BYTES + (kk % 4) * 32) >> 4;
-        if (leader) tc_mma_ss(tmem + C::COL_B, dOk + off, dVk + off, IDESC_SS, kk > 0);
+        if (leader) tc_mma_ss(tmem + colS + 64, dOk + off, dVk + off, IDESC_SS, kk > 0);
       }
       __syncwarp();
     };
+    // dQ += dS_h K_h: K = 64 keys in steps of 16, K read MN-major; the
+    // warpgroups' bf16 halves sit at columns 0-15 and 32-47 of S.
+    auto issue_ts = [&](int gh) {
+      const uint32_t stage = stage_of(gh >> 1), rows = (gh & 1) * 8192u;
+      const uint64_t dKm = smem_desc_sw128(stage + rows, C::HALF_BYTES, 1024);
+      const uint32_t colS = (gh & 1) * 128u;
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk) {
+        const uint32_t a = 8u * kk + (kk >= 2 ? 16u : 0u);
+        if (leader)
+          tc_mma_ts(tmem + C::COL_C, tmem + colS + a, dKm + ((kk * 2048) >> 4), IDESC_TS,
+                    (gh > 0 || kk > 0) ? 1u : 0u);
+      }
+      __syncwarp();
+    };
+    const int nhalves = 2 * nkv;
     bool ok = wait(bar_q, 0) && wait_full(0);
     if (ok) {
       tc_fence_after();
-      issue_s(0);
-      issue_dp(0);
+      issue_sdp(0);
       commit(bar_sd);
-      if (nkv > 1) {
-        ok = wait_full(1);
-        if (ok) {
-          tc_fence_after();
-          issue_s(1);
-        }
-      }
     }
-    for (int j = 0; ok && j < nkv; ++j) {
-      if (!wait(bar_ds, j & 1)) break;
+    for (int gh = 0; ok && gh < nhalves; ++gh) {
+      // The next half's products go into the other buffer while this half's
+      // dS is formed (that buffer's last reader, half gh - 1's dQ product,
+      // was issued before).
+      const int nx = gh + 1;
+      if (nx < nhalves) {
+        if ((nx & 1) == 0) {
+          if (!wait_full(nx >> 1)) break;
+          tc_fence_after();
+        }
+        issue_sdp(nx);
+        commit(bar_sd + 8 * (nx & 1));
+      }
+      if (!wait(bar_ds + 8 * (gh & 1), (gh >> 1) & 1)) break;
       tc_fence_after();
-      // dP's columns are free again; stage j + 1 is full (waited for S(j + 1)).
-      if (j + 1 < nkv) {
-        issue_dp(j + 1);
-        commit(bar_sd);
-      }
-      // dQ += dS K: K = 128 keys in steps of 16, K read MN-major.
-      const uint64_t dKm = smem_desc_sw128(stage_of(j), C::HALF_BYTES, 1024);
-#pragma unroll
-      for (int kk = 0; kk < 8; ++kk)
-        if (leader)
-          tc_mma_ts(tmem + C::COL_C, tmem + sbuf(j) + C::a_col(kk), dKm + ((kk * 2048) >> 4),
-                    IDESC_TS, (j > 0 || kk > 0) ? 1u : 0u);
-      __syncwarp();
-      commit(bar_empty + 8 * (j % C::Q_STAGES));
-      if (j + 2 < nkv) {
-        if (!wait_full(j + 2)) break;
-        tc_fence_after();
-        issue_s(j + 2);  // behind dQ(j), which reads dS(j) in the same columns
-      }
+      issue_ts(gh);
+      if (gh & 1) commit(bar_empty + 8 * ((gh >> 1) % C::Q_STAGES));
     }
     commit(bar_done);
     volatile int never = 0;
     mbar_wait_bounded(bar_done, 0, &never, p.status, p.wait_limit_ns, kErrTimeout);
   } else if (warp < 8) {
-    // thread = query row; warpgroup e = key columns [64e, 64e + 64)
+    // thread = query row; in each 64-key half, warpgroup e takes keys
+    // [32e, 32e + 32)
     const int e = warp >> 2;
     const int i = row0 + (threadIdx.x & 127);
     const uint32_t lane_base = static_cast<uint32_t>(warp & 3) * 32u << 16;
-    const uint32_t tB = tmem + lane_base + C::COL_B + 64 * e;
     const size_t vrow = static_cast<size_t>(bh) * p.Npad + i;
     const float lse2 = p.ws_lse2[vrow];
     const float delta = p.ws_delta[vrow];
     const int limit = p.causal ? min(L, i + 1) : L;
     bool ok = true;
-    for (int j = 0; j < nkv && ok; ++j) {
-      const bool got = mbar_wait_bounded(bar_sd, j & 1, abort_flag, p.status, p.wait_limit_ns,
-                                         kErrTimeout);
+    for (int gh = 0; gh < 2 * nkv && ok; ++gh) {
+      const int jt = gh >> 1, hk = gh & 1;  // key tile, key half
+      const bool got = mbar_wait_bounded(bar_sd + 8 * hk, (gh >> 1) & 1, abort_flag, p.status,
+                                         p.wait_limit_ns, kErrTimeout);
       if (!__all_sync(0xffffffffu, got)) {
         ok = false;
         break;
       }
       tc_fence_after();
-      // S(j) sits in the columns of its parity (COL_A or COL_D)
-      const uint32_t tA = tmem + lane_base + ((j & 1) ? C::COL_D : C::COL_A) + 64 * e;
+      const uint32_t tS = tmem + lane_base + hk * 128 + 32 * e;
       {
-        uint32_t sv[64], dp[64];
-        tmem_ld32(tA, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
-        tmem_ld32(tA + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
-        tmem_ld32(tB, *reinterpret_cast<uint32_t(*)[32]>(&dp[0]));
-        tmem_ld32(tB + 32, *reinterpret_cast<uint32_t(*)[32]>(&dp[32]));
+        uint32_t sv[32], dp[32];
+        tmem_ld32(tS, sv);
+        tmem_ld32(tS + 64, dp);
         tmem_wait_ld();
-        uint32_t dk[32];
+        uint32_t dk[16];
 #pragma unroll
-        for (int x = 0; x < 32; ++x) {
+        for (int x = 0; x < 16; ++x) {
           float dv[2];
 #pragma unroll
           for (int u = 0; u < 2; ++u) {
-            const int key = j * 128 + 64 * e + 2 * x + u;
+            const int key = jt * 128 + 64 * hk + 32 * e + 2 * x + u;
             const float pp = key < limit ? ex2_approx(fmaf(__uint_as_float(sv[2 * x + u]),
                                                            p.scale_log2, -lse2))
                                          : 0.f;
@@ -631,12 +635,12 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
           }
           dk[x] = pack_bf16x2(dv[0], dv[1]);
         }
-        // dS over the first 32 of this warpgroup's S columns
-        tmem_st32(tA, dk);
+        // dS over the first 16 of this block's 32 S columns
+        tmem_st16(tS, dk);
       }
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(bar_ds);
+      mbar_arrive(bar_ds + 8 * hk);
     }
     if (ok && nkv > 0) {
       const bool got = mbar_wait_bounded(bar_done, 0, abort_flag, p.status, p.wait_limit_ns,
