@@ -207,44 +207,76 @@ def sample_flops(w: wl.Workload, rows: np.ndarray, seqlens) -> float:
     return total / 2 if w.causal else total
 
 
-def time_oracle(w: wl.Workload, inp: wl.Inputs, budget_s: float):
-    """The CPU oracle on a bounded sample of query rows of the same workload."""
+def oracle_sample(w: wl.Workload, inp: wl.Inputs, target_s: float):
+    """A seeded sample of query rows per (batch, head) on which one oracle run
+    takes about target_s on this host (at least 4 rows per head, at most all
+    rows): the sample doubles, or jumps to the estimated size, until a run
+    reaches a quarter of the target."""
     import oracle
     threads = oracle.num_threads()
-    rows_per_head = 4
     scale = float(np.float32(w.scale))
+    rows_per_head = 4
     while True:
         rows = oracle_sample_rows(w, rows_per_head)
         t0 = time.perf_counter()
         oracle.attention_forward(inp.q_bits, inp.k_bits, inp.v_bits, causal=w.causal, scale=scale,
                                  seqlens=inp.seqlens, rows=rows, threads=threads)
         dt = time.perf_counter() - t0
-        if dt > budget_s / 4 or rows_per_head >= w.N:
-            break
-        rows_per_head = min(w.N, rows_per_head * max(2, int(budget_s / 4 / max(dt, 1e-3))))
+        if dt > target_s / 4 or rows_per_head >= w.N:
+            return rows, rows_per_head, dt, threads
+        rows_per_head = min(w.N, rows_per_head * max(2, int(target_s / 4 / max(dt, 1e-3))))
+
+
+def run_oracle_rows(w: wl.Workload, inp: wl.Inputs, rows, threads) -> float:
+    """Seconds for one oracle run on the given query rows."""
+    import oracle
+    t0 = time.perf_counter()
+    oracle.attention_forward(inp.q_bits, inp.k_bits, inp.v_bits, causal=w.causal,
+                             scale=float(np.float32(w.scale)), seqlens=inp.seqlens, rows=rows,
+                             threads=threads)
+    return time.perf_counter() - t0
+
+
+def time_oracle(w: wl.Workload, inp: wl.Inputs, budget_s: float):
+    """The CPU oracle on a bounded sample of query rows of the same workload."""
+    rows, rows_per_head, dt, threads = oracle_sample(w, inp, budget_s)
     f = sample_flops(w, rows, inp.seqlens)
     return {"value": f / dt / 1e12, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
             "sample": f"{rows_per_head} seeded query rows per (batch, head) of {w.name} "
                       f"({rows.size} rows, every visible key), {dt:.1f} s wall"}, dt
 
 
+# The reference arm's whole warm-up + timed run stays within about this many
+# seconds, whatever --steps and --warmup are.
+REF_TOTAL_S = 150.0
+
+
 def run_reference(args, w: wl.Workload):
+    """The oracle as the reference arm: one run on a fixed row sample per step,
+    the sample sized so that all warm-up and timed steps fit REF_TOTAL_S."""
     rank, world, _ = dist_env()
     if rank != 0:
         return 0
     inp = wl.draw_workload(w)
+    total = args.warmup + args.steps
+    target = max(0.05, min(args.ref_budget, REF_TOTAL_S / max(total, 1)))
+    rows, rows_per_head, _, threads = oracle_sample(w, inp, target)
+    f = sample_flops(w, rows, inp.seqlens)
     per_step = []
-    cpu = None
-    for s in range(args.warmup + args.steps):
-        cpu, dt = time_oracle(w, inp, budget_s=args.ref_budget)
+    for s in range(total):
+        dt = run_oracle_rows(w, inp, rows, threads)
         if s >= args.warmup:
-            per_step.append(cpu["value"])
-    value = statistics.median(per_step)
-    cpu["value"] = value
+            per_step.append(dt)
+    ms = statistics.median(per_step) * 1e3
+    value = f / (ms * 1e-3) / 1e12
+    cpu = {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+           "sample": f"{rows_per_head} seeded query rows per (batch, head) of {w.name} "
+                     f"({rows.size} rows, every visible key) per step; median of "
+                     f"{len(per_step)} timed steps of {ms / 1e3:.2f} s"}
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
-        "ms_per_step": None, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "f64", "data": "synthetic (seeded, bf16-rounded N(0,1))",
         "config": workload_config(w),
         "cpu_baseline": cpu,
