@@ -132,17 +132,21 @@ class ClockSampler:
             self.nvml = None
 
     def _power_w(self):
-        """Instantaneous board power where NVML offers it (the plain power
-        reading is averaged over about a second), else the averaged one."""
+        """(board power as nvidia-smi's power.draw reports it, averaged by the
+        driver over about a second; NVML's instantaneous power field where it
+        exists, else None).  The instantaneous field updates far more slowly
+        than the 10 ms sampling, so only its maximum is reported."""
         nv = self.nvml
+        avg = nv.nvmlDeviceGetPowerUsage(self.handle) / 1000.0
+        inst = None
         if self.instant_field is not None:
             try:
                 v = nv.nvmlDeviceGetFieldValues(self.handle, [self.instant_field])[0]
                 if v.nvmlReturn == nv.NVML_SUCCESS:
-                    return float(v.value.uiVal) / 1000.0
+                    inst = float(v.value.uiVal) / 1000.0
             except Exception:
-                pass
-        return nv.nvmlDeviceGetPowerUsage(self.handle) / 1000.0
+                inst = None
+        return avg, inst
 
     def _run(self):
         nv = self.nvml
@@ -184,10 +188,12 @@ class ClockSampler:
                 if rs & bit:
                     reasons.add(name)
         sm = [x[1] for x in inside]
-        pw = [x[2] for x in inside]
+        pw = [x[2][0] for x in inside]
+        inst = [x[2][1] for x in inside if x[2][1] is not None]
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": self.max_mhz,
                 "sm_mhz_min": min(sm), "reasons": sorted(reasons), "samples": len(inside),
                 "power_w_median": statistics.median(pw), "power_w_max": max(pw),
+                "power_w_instant_max": max(inst) if inst else None,
                 "source": "NVML, 10 ms, timed region only"}
 
 

@@ -22,14 +22,20 @@
 // O1 [384,384+d).  P_t (bf16, packed two per column) overwrites the first 64
 // columns of S_t and feeds the PV product straight from tensor memory; it is
 // published in two halves of 64 keys so the PV product starts on the first
-// half while the second is computed.
+// half while the second is computed.  In a causal unit, Q tile 0 skips the last
+// key tile when it lies wholly above its rows (Q tile 1 still needs it).
+//
+// The same body serves FP8 E4M3 inputs (F8 = true, head dim 128): 8-bit
+// tiles, kind::f8f6f4 products, V given transposed so both products read
+// K-major operands, and P stored as E4M3 with a factor 2^2 and a rescale
+// threshold of 6 (log2 units) so it never saturates.
 //
 // Differences from the pages' statement of the recurrence, all algebraically
 // equivalent: O is kept unnormalised (O~ = l * O) and divided by l once at the
 // end; exponentials are base 2 on log2(e)-scaled scores; the max used for the
 // exponentials (m_ref) is only moved when the row max grows by more than
-// 2^8, so most tiles skip the O rescale (values stay below 2^8, far from fp32
-// overflow).
+// 2^8 (bf16; 2^6 for FP8), so most tiles skip the O rescale (values stay
+// below 2^8, far from fp32 overflow).
 #pragma once
 
 #include <cstdint>

@@ -2,7 +2,8 @@
 
 The sampler must look the device up by the UUID torch reports, keep only
 the samples taken inside the timed region, decode every clock-event reason
-bit, and prefer the instantaneous power field."""
+bit, and report the averaged board power with the instantaneous field's
+maximum beside it."""
 import sys
 import time
 import types
@@ -25,7 +26,7 @@ def _fake_nvml(state):
     nv.nvmlDeviceGetHandleByUUID = lambda uuid: state.setdefault("uuid", uuid) and "handle"
     nv.nvmlDeviceGetMaxClockInfo = lambda h, c: 1965
     nv.nvmlDeviceGetClockInfo = lambda h, c: 1500 if state["busy"] else 600
-    nv.nvmlDeviceGetPowerUsage = lambda h: 123000
+    nv.nvmlDeviceGetPowerUsage = lambda h: 950000 if state["busy"] else 123000
     nv.nvmlDeviceGetFieldValues = lambda h, ids: [_Field(990000 if state["busy"] else 90000)]
     nv.nvmlDeviceGetCurrentClocksEventReasons = lambda h: (0x4 | 0x8) if state["busy"] else 0x1
     return nv
@@ -52,7 +53,8 @@ def test_sampler_keeps_the_timed_region_and_decodes_reasons(monkeypatch):
     assert rec["sm_mhz"] == 1500.0 and rec["sm_mhz_min"] == 1500.0
     assert rec["sm_max_mhz"] == 1965.0
     assert rec["reasons"] == ["hw_slowdown", "sw_power_cap"]   # gpu_idle stays outside
-    assert rec["power_w_median"] == 990.0 and rec["power_w_max"] == 990.0
+    assert rec["power_w_median"] == 950.0 and rec["power_w_max"] == 950.0
+    assert rec["power_w_instant_max"] == 990.0
 
 
 def test_sampler_without_nvml_says_so(monkeypatch):
