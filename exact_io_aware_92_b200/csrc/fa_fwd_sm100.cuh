@@ -86,11 +86,18 @@ struct Sm100Cfg {
   static constexpr int BAR_Q_EMPTY = 2;                 // [2 tiles]
   static constexpr int BAR_KV_FULL = 4;                 // [STAGES]
   static constexpr int BAR_KV_EMPTY = 4 + STAGES;       // [STAGES]
-  static constexpr int BAR_S_FULL = 4 + 2 * STAGES;     // [2 tiles]
-  static constexpr int BAR_P_HALF = BAR_S_FULL + 2;     // [2 tiles][2 halves of the keys]
-  static constexpr int BAR_O_FULL = BAR_P_HALF + 4;     // [2 tiles]
+  // D = 64 (bf16): tensor memory has room for a third S buffer.  Three
+  // buffers rotate over the CTA's sequence of S products (both Q tiles
+  // interleaved), so a Q tile's next S is computed while it still works on
+  // the current one.
+  static constexpr bool TRIPLE = (D == 64) && !F8;
+  static constexpr int NSBUF = TRIPLE ? 3 : 2;
+  static constexpr int BAR_S_FULL = 4 + 2 * STAGES;     // [NSBUF]
+  static constexpr int BAR_P_HALF = BAR_S_FULL + NSBUF; // [NSBUF][2 halves of the keys]
+  static constexpr int BAR_O_FULL = BAR_P_HALF + 2 * NSBUF;  // [2 tiles]
   static constexpr int BAR_MMA_DONE = BAR_O_FULL + 2;   // 1
-  static constexpr int NUM_BARS = BAR_MMA_DONE + 1;
+  static constexpr int BAR_PV_DONE = BAR_MMA_DONE + 1;  // [2 tiles] (TRIPLE): a PV product landed
+  static constexpr int NUM_BARS = BAR_PV_DONE + (TRIPLE ? 2 : 0);
   static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;  // tmem base, abort flag
   static constexpr int SMEM_BYTES = OFF_MISC + 16;
   static constexpr int SMEM_ALLOC = SMEM_BYTES + 1024;     // room to align the base to 1 KB
@@ -101,7 +108,9 @@ struct Sm100Cfg {
   static constexpr uint32_t REGS_CONTROL = 56;
   static constexpr uint32_t REGS_SOFTMAX = 224;
   static constexpr uint32_t TMEM_COLS = 512;
-  static constexpr uint32_t COL_S0 = 0, COL_O0 = 256;
+  static constexpr uint32_t COL_S0 = 0;
+  static constexpr uint32_t COL_O0 = TRIPLE ? 384 : 256;  // O0; O1 is O_STRIDE further
+  static constexpr uint32_t O_STRIDE = TRIPLE ? 64 : 128;
   // The reference max moves when the row max grows by more than this (log2
   // units).  FP8: P is stored as E4M3 (largest finite 448) and carries a
   // factor 2^P_SHIFT that keeps small probabilities out of the subnormal
@@ -176,7 +185,9 @@ __device__ __forceinline__ Unit unit_at(const FwdParams &p, int u) {
   const int kv_end = p.causal ? min(L, x.row0 + C::ROWS_PER_UNIT) : L;
   // A unit past the end of its sequence (packed layout) has no rows at all.
   x.nkv = x.row0 < x.q_rows ? (kv_end + C::BN - 1) / C::BN : 0;
-  x.nkv0 = (p.causal && x.nkv > 1 && (x.nkv - 1) * C::BN >= x.row0 + C::BM) ? x.nkv - 1 : x.nkv;
+  x.nkv0 = (!C::TRIPLE && p.causal && x.nkv > 1 && (x.nkv - 1) * C::BN >= x.row0 + C::BM)
+               ? x.nkv - 1
+               : x.nkv;
   return x;
 }
 
@@ -297,7 +308,7 @@ __device__ void role_mma(const Sm100Ctx<D, F8> &x, const FwdParams &p) {
   constexpr uint32_t IDESC_O = F8 ? idesc_e4m3_f32(128, D) : idesc_bf16_f32(128, D, 0, 1);
   const bool leader = elect_one();
   const uint32_t tS[2] = {x.tmem + C::COL_S0, x.tmem + C::COL_S0 + 128};
-  const uint32_t tO[2] = {x.tmem + C::COL_O0, x.tmem + C::COL_O0 + 128};
+  const uint32_t tO[2] = {x.tmem + C::COL_O0, x.tmem + C::COL_O0 + C::O_STRIDE};
 
   // Descriptors are linear in the start address (16-byte units in the low
   // bits), so they are built once and offset per operand.
@@ -461,6 +472,121 @@ __device__ void role_mma(const Sm100Ctx<D, F8> &x, const FwdParams &p) {
 }
 
 // --------------------------------------------------------------------------
+// MMA issuer with three S buffers (D = 64).  The CTA's S products form one
+// sequence, index T = 2 * (key tiles so far) + Q tile, and S(T) goes to
+// buffer T % 3.  S(T) is issued right after PV(T - 3), the last reader of
+// that buffer's P, so a Q tile's next S is usually complete before its
+// softmax finishes the current tile.  Barriers: S full and P halves per
+// buffer (phase T / 3), PV done per Q tile (one phase per tile), O full per
+// Q tile and unit.
+// --------------------------------------------------------------------------
+template <int D, bool F8>
+__device__ void role_mma_triple(const Sm100Ctx<D, F8> &x, const FwdParams &p) {
+  using C = Sm100Cfg<D, F8>;
+  static_assert(C::TRIPLE, "three S buffers: bf16, head dim 64");
+  constexpr uint32_t IDESC_S = idesc_bf16_f32(128, C::BN, 0, 0);  // Q, K both K-major
+  constexpr uint32_t IDESC_O = idesc_bf16_f32(128, D, 0, 1);      // P from TMEM, V MN-major
+  const bool leader = elect_one();
+  const uint64_t desc_q0 = smem_desc_sw128(x.q_tile(0), 16, 1024);
+  const uint64_t desc_q1 = smem_desc_sw128(x.q_tile(1), 16, 1024);
+  const uint64_t desc_kv_k = smem_desc_sw128(x.kv_tile(0), 16, 1024);
+  const uint64_t desc_kv_v = smem_desc_sw128(x.kv_tile(0), C::BOX_BYTES, 1024);
+  auto wait = [&](int bar, uint32_t parity) {
+    const bool ok = mbar_wait_bounded(x.bar(bar), parity, x.abort_flag, p.status,
+                                      p.wait_limit_ns, kErrTimeout);
+    return __all_sync(0xffffffffu, ok);
+  };
+  auto commit = [&](int bar) {
+    if (leader) tc_commit(x.bar(bar));
+    __syncwarp();
+  };
+  auto sbuf = [&](int tt) { return x.tmem + C::COL_S0 + 128u * static_cast<uint32_t>(tt % 3); };
+
+  int T = 0;   // S products issued by this CTA so far
+  int g = 0;   // K/V tiles consumed (ring position)
+  int qi = 0;  // units with keys processed so far
+  bool ok = true;
+  for (int k = 0; ok; ++k) {
+    const int u = snake_unit(k, p.num_units);
+    if (u == -2) break;
+    if (u < 0) continue;
+    const Unit w = unit_at<D, F8>(p, u);
+    const int n = w.nkv;
+    if (n == 0) continue;
+    const uint32_t qpar = static_cast<uint32_t>(qi & 1);
+    if (!wait(C::BAR_Q_FULL + 0, qpar) || !wait(C::BAR_Q_FULL + 1, qpar)) break;
+    const int t0 = T, tend = T + 2 * n;
+    // S of sequence index tt (key tile j, Q tile q); K tile j is waited for
+    // by Q tile 0's product and released after Q tile 1's.
+    auto issue_s = [&](int tt) {
+      const int j = (tt - t0) >> 1, q = (tt - t0) & 1;
+      const int ks = ring_slot<D, F8>(2 * (g + j));
+      if (q == 0) {
+        if (!wait(C::BAR_KV_FULL + ks, ring_parity<D, F8>(2 * (g + j)))) return false;
+        tc_fence_after();
+      }
+      const uint64_t kd = desc_kv_k + ((ks * C::TILE_BYTES) >> 4);
+#pragma unroll
+      for (int kk = 0; kk < C::KSTEPS; ++kk) {
+        const uint32_t off = ((kk / 4) * C::BOX_BYTES + (kk % 4) * 32) >> 4;
+        if (leader)
+          tc_mma_ss(sbuf(tt), (q ? desc_q1 : desc_q0) + off, kd + off, IDESC_S, kk > 0 ? 1u : 0u);
+      }
+      __syncwarp();
+      commit(C::BAR_S_FULL + tt % 3);
+      if (q == 1) commit(C::BAR_KV_EMPTY + ks);
+      if (j == n - 1) commit(C::BAR_Q_EMPTY + q);
+      return true;
+    };
+    for (int tt = t0; ok && tt < t0 + 3 && tt < tend; ++tt) ok = issue_s(tt);
+    for (int tp = t0; ok && tp < tend; ++tp) {
+      const int j = (tp - t0) >> 1, q = (tp - t0) & 1;
+      const int vs = ring_slot<D, F8>(2 * (g + j) + 1);
+      if (q == 0 && !wait(C::BAR_KV_FULL + vs, ring_parity<D, F8>(2 * (g + j) + 1))) {
+        ok = false;
+        break;
+      }
+      const uint32_t par = static_cast<uint32_t>((tp / 3) & 1);
+      const uint64_t vd = desc_kv_v + ((vs * C::TILE_BYTES) >> 4);
+      const uint32_t tO = x.tmem + C::COL_O0 + C::O_STRIDE * q;
+      // O_q += P V for each 64-key half as the softmax publishes it.
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+        if (!wait(C::BAR_P_HALF + 2 * (tp % 3) + half, par)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+#pragma unroll
+        for (int k4 = 0; k4 < 4; ++k4) {
+          const int kk = 4 * half + k4;
+          if (leader)
+            tc_mma_ts(tO, sbuf(tp) + kk * 8, vd + ((kk * 2048) >> 4), IDESC_O,
+                      (j > 0 || kk > 0) ? 1u : 0u);
+        }
+        __syncwarp();
+      }
+      if (!ok) break;
+      commit(C::BAR_PV_DONE + q);
+      if (q == 1) commit(C::BAR_KV_EMPTY + vs);
+      if (j == n - 1) commit(C::BAR_O_FULL + q);
+      // the buffer tp's P sat in is free once this PV has read it
+      if (tp + 3 < tend && !issue_s(tp + 3)) {
+        ok = false;
+        break;
+      }
+    }
+    if (!ok) break;
+    T = tend;
+    g += n;
+    ++qi;
+  }
+  commit(C::BAR_MMA_DONE);
+  volatile int never = 0;
+  mbar_wait_bounded(x.bar(C::BAR_MMA_DONE), 0, &never, p.status, p.wait_limit_ns, kErrTimeout);
+}
+
+// --------------------------------------------------------------------------
 // Softmax warpgroup t (128 threads, one query row each)
 // --------------------------------------------------------------------------
 template <int D, bool F8>
@@ -469,7 +595,7 @@ __device__ void role_softmax(const Sm100Ctx<D, F8> &x, const FwdParams &p, int t
   const int r = threadIdx.x & 127;
   const uint32_t lane_base = static_cast<uint32_t>((threadIdx.x >> 5) & 3) * 32u << 16;
   const uint32_t tS = x.tmem + lane_base + C::COL_S0 + 128 * t;
-  const uint32_t tO = x.tmem + lane_base + C::COL_O0 + 128 * t;
+  const uint32_t tO = x.tmem + lane_base + C::COL_O0 + C::O_STRIDE * t;
   const float sl2 = p.scale_log2;
 
   auto wait_all = [&](int bar, uint32_t parity) {
@@ -504,13 +630,20 @@ __device__ void role_softmax(const Sm100Ctx<D, F8> &x, const FwdParams &p, int t
     float m_ref = -INFINITY;  // reference max (log2 units) the exponentials use
     float l = 0.f;            // row sum of the fp32 probabilities relative to m_ref
     for (int j = 0; j < nkv_t; ++j) {
-      if (!wait_all(C::BAR_S_FULL + t, static_cast<uint32_t>((g + j) & 1))) return;
+      // This tile's S buffer and barriers: fixed per Q tile, or (three
+      // buffers) sequence index tt = 2 (g + j) + t, buffer tt % 3.
+      const int tt = 2 * (g + j) + t;
+      const int sb = C::TRIPLE ? tt % 3 : t;
+      const uint32_t spar =
+          static_cast<uint32_t>(C::TRIPLE ? (tt / 3) & 1 : (g + j) & 1);
+      const uint32_t tSj = C::TRIPLE ? x.tmem + lane_base + C::COL_S0 + 128u * sb : tS;
+      if (!wait_all(C::BAR_S_FULL + sb, spar)) return;
       tc_fence_after();
       uint32_t s[128];
-      tmem_ld32(tS + 0, *reinterpret_cast<uint32_t(*)[32]>(&s[0]));
-      tmem_ld32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&s[32]));
-      tmem_ld32(tS + 64, *reinterpret_cast<uint32_t(*)[32]>(&s[64]));
-      tmem_ld32(tS + 96, *reinterpret_cast<uint32_t(*)[32]>(&s[96]));
+      tmem_ld32(tSj + 0, *reinterpret_cast<uint32_t(*)[32]>(&s[0]));
+      tmem_ld32(tSj + 32, *reinterpret_cast<uint32_t(*)[32]>(&s[32]));
+      tmem_ld32(tSj + 64, *reinterpret_cast<uint32_t(*)[32]>(&s[64]));
+      tmem_ld32(tSj + 96, *reinterpret_cast<uint32_t(*)[32]>(&s[96]));
       tmem_wait_ld();
 
       const int kbase = j * C::BN;
@@ -572,9 +705,9 @@ __device__ void role_softmax(const Sm100Ctx<D, F8> &x, const FwdParams &p, int t
       // P of one 64-key half over the first columns of S_t.
       auto store_p = [&](int half) {
         if constexpr (F8)
-          tmem_st16(tS + 16 * half, pk);
+          tmem_st16(tSj + 16 * half, pk);
         else
-          tmem_st32(tS + 32 * half, pk);
+          tmem_st32(tSj + 32 * half, pk);
       };
       bool need;
       float alpha = 1.0f;
@@ -606,9 +739,15 @@ __device__ void role_softmax(const Sm100Ctx<D, F8> &x, const FwdParams &p, int t
       const float m_use = (m_ref == -INFINITY) ? 0.0f : m_ref;
       store_p(0);
       // O holds earlier tiles' sum only for j > 0; nothing writes it until
-      // this warpgroup publishes P (the PV product of tile j-1 finished
-      // before S_j did).  It is rescaled before the first half goes out.
+      // this warpgroup publishes P.  With two S buffers the PV product of
+      // tile j-1 finished before S_j did; with three it may still be running,
+      // so its completion is awaited first.  O is rescaled before the first
+      // half goes out.
       if (j > 0 && __any_sync(0xffffffffu, need)) {
+        if constexpr (C::TRIPLE) {
+          if (!wait_all(C::BAR_PV_DONE + t, static_cast<uint32_t>((g + j - 1) & 1))) return;
+          tc_fence_after();
+        }
 #pragma unroll
         for (int c = 0; c < D / 32; ++c) {
           uint32_t o[32];
@@ -621,13 +760,13 @@ __device__ void role_softmax(const Sm100Ctx<D, F8> &x, const FwdParams &p, int t
       }
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(x.bar(C::BAR_P_HALF + 2 * t));
+      mbar_arrive(x.bar(C::BAR_P_HALF + 2 * sb));
       // Second half of the keys.
       exp_half(1, m_use, pk, sum2);
       store_p(1);
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(x.bar(C::BAR_P_HALF + 2 * t + 1));
+      mbar_arrive(x.bar(C::BAR_P_HALF + 2 * sb + 1));
       float a0, a1;
       f32x2_split(sum2, a0, a1);
       l += a0 + a1;
@@ -686,10 +825,13 @@ __device__ __forceinline__ void fwd_kernel_body(const CUtensorMap *tm_q, const C
     for (int t = 0; t < 2; ++t) {
       mbar_init(x.bar(C::BAR_Q_FULL + t), 1);
       mbar_init(x.bar(C::BAR_Q_EMPTY + t), 1);
-      mbar_init(x.bar(C::BAR_S_FULL + t), 1);
-      mbar_init(x.bar(C::BAR_P_HALF + 2 * t), 128);
-      mbar_init(x.bar(C::BAR_P_HALF + 2 * t + 1), 128);
       mbar_init(x.bar(C::BAR_O_FULL + t), 1);
+      if (C::TRIPLE) mbar_init(x.bar(C::BAR_PV_DONE + t), 1);
+    }
+    for (int b = 0; b < C::NSBUF; ++b) {
+      mbar_init(x.bar(C::BAR_S_FULL + b), 1);
+      mbar_init(x.bar(C::BAR_P_HALF + 2 * b), 128);
+      mbar_init(x.bar(C::BAR_P_HALF + 2 * b + 1), 128);
     }
     for (int s = 0; s < C::STAGES; ++s) {
       mbar_init(x.bar(C::BAR_KV_FULL + s), 1);
@@ -720,7 +862,10 @@ __device__ __forceinline__ void fwd_kernel_body(const CUtensorMap *tm_q, const C
     if (warp == 8) {
       if (lane == 0) role_producer<D, F8>(x, p, tm_q, tm_k, tm_v);
     } else if (warp == 9) {
-      role_mma<D, F8>(x, p);
+      if constexpr (C::TRIPLE)
+        role_mma_triple<D, F8>(x, p);
+      else
+        role_mma<D, F8>(x, p);
     }
   } else {
     regs_increase<C::REGS_SOFTMAX>();
