@@ -192,7 +192,8 @@ class ClockSampler:
         inst = [x[2][1] for x in inside if x[2][1] is not None]
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": self.max_mhz,
                 "sm_mhz_min": min(sm), "reasons": sorted(reasons), "samples": len(inside),
-                "power_w_median": statistics.median(pw), "power_w_max": max(pw),
+                "power_w_1s_avg_median": statistics.median(pw),
+                "power_w_1s_avg_max": max(pw),
                 "power_w_instant_max": max(inst) if inst else None,
                 "source": "NVML, 10 ms, timed region only"}
 

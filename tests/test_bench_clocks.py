@@ -53,7 +53,7 @@ def test_sampler_keeps_the_timed_region_and_decodes_reasons(monkeypatch):
     assert rec["sm_mhz"] == 1500.0 and rec["sm_mhz_min"] == 1500.0
     assert rec["sm_max_mhz"] == 1965.0
     assert rec["reasons"] == ["hw_slowdown", "sw_power_cap"]   # gpu_idle stays outside
-    assert rec["power_w_median"] == 950.0 and rec["power_w_max"] == 950.0
+    assert rec["power_w_1s_avg_median"] == 950.0 and rec["power_w_1s_avg_max"] == 950.0
     assert rec["power_w_instant_max"] == 990.0
 
 

@@ -106,6 +106,27 @@ def test_full_workload_sampled_rows(w):
     compare(og, lg, o_ref, lse_ref, o_tol=O_TOL_BF16, lse_tol=LSE_TOL_BF16, what=w.name)
 
 
+@pytest.mark.parametrize("causal,lens", [(True, None), (False, [4096, 2500, 1, 3333])])
+def test_long_d64_sampled_rows(causal, lens):
+    # d = 64 rotates three S buffers over both Q tiles' products: units of up
+    # to 32 key tiles, many units per CTA, K x 2 for more rescales.
+    B = 4
+    inp = wl.draw(B, 8, 2, 4096, 64, seed=1900 + int(causal), k_scale=2.0)
+    if lens is not None:
+        inp.seqlens = np.asarray(lens, dtype=np.int32)
+    o, lse = run_bf16(inp, causal=causal, scale=0.125)
+    assert np.all(np.isfinite(o))
+    w = wl.Workload("long_d64", B, 8, 2, 4096, 64, causal, seed=1900)
+    rows = wl.sample_rows(w, 64)
+    rows[:, 0] = 0
+    rows[:, -1] = 4095
+    rows.sort(axis=1)
+    o_ref, lse_ref = reference(inp, causal=causal, scale=0.125, rows=rows)
+    og, lg = gather_rows(o, lse, rows)
+    compare(og, lg, o_ref, lse_ref, o_tol=O_TOL_BF16, lse_tol=LSE_TOL_BF16,
+            what=f"long d64 causal={causal}")
+
+
 def test_deterministic():
     inp = wl.draw(2, 8, 2, 1000, 128, seed=55)
     a = run_bf16(inp, causal=True, scale=0.088)
