@@ -1,9 +1,12 @@
-// C ABI of the attention-forward library (declared in include/fa.h).
+// C ABI of the attention library (declared in include/fa.h).
 //
 // Host side only: argument checks, TMA tensor maps (cuTensorMapEncodeTiled,
 // reached through the runtime's driver entry point so the library does not
-// link libcuda), launch configuration, and the status word.  All attention
-// arithmetic runs in the kernels of fa_fwd_sm100.cuh and fa_fwd_f32.cuh.
+// link libcuda), launch configuration, the status word, and the copy
+// streams of the host-buffer call.  All attention arithmetic runs in the
+// kernels: fa_fwd_sm100.cuh (bf16 and FP8 forward, packed layout),
+// fa_fwd_f32.cuh (fp32 check mode), fa_bwd_sm100.cuh (backward) and
+// fa_decode.cuh (split-KV decode).
 #include <cmath>
 #include <cstdint>
 #include <algorithm>
@@ -38,7 +41,9 @@ struct DeviceState {
   bool bwd_attr64 = false, bwd_attr128 = false;
   bool fp8_attr = false;
   // fa_fwd_hostio's copy streams and per-slice events, created on first use
-  // and kept for the process's lifetime.
+  // and kept for the process's lifetime.  io_mu is held for a whole call, so
+  // host threads that call it on one device take turns.
+  std::mutex io_mu;
   bool io_ready = false;
   cudaStream_t io_in = nullptr, io_out = nullptr;
   cudaEvent_t io_ev_in[16] = {}, io_ev_done[16] = {}, io_ev_end = nullptr;
@@ -561,21 +566,19 @@ int fa_fwd_hostio(const void *q_h, const void *k_h, const void *v_h, void *o_h, 
   DeviceState *ds = nullptr;
   rc = current_device(&ds);
   if (rc != FA_OK) return rc;
-  {
-    std::lock_guard<std::mutex> lock(g_mu);
-    if (!ds->io_ready) {
-      bool ok = cudaStreamCreateWithFlags(&ds->io_in, cudaStreamNonBlocking) == cudaSuccess &&
-                cudaStreamCreateWithFlags(&ds->io_out, cudaStreamNonBlocking) == cudaSuccess &&
-                cudaEventCreateWithFlags(&ds->io_ev_end, cudaEventDisableTiming) == cudaSuccess;
-      for (int i = 0; ok && i < 16; ++i)
-        ok = cudaEventCreateWithFlags(&ds->io_ev_in[i], cudaEventDisableTiming) == cudaSuccess &&
-             cudaEventCreateWithFlags(&ds->io_ev_done[i], cudaEventDisableTiming) == cudaSuccess;
-      if (!ok) {
-        cudaGetLastError();
-        return FA_ERR_CUDA;
-      }
-      ds->io_ready = true;
+  std::lock_guard<std::mutex> io_lock(ds->io_mu);
+  if (!ds->io_ready) {
+    bool ok = cudaStreamCreateWithFlags(&ds->io_in, cudaStreamNonBlocking) == cudaSuccess &&
+              cudaStreamCreateWithFlags(&ds->io_out, cudaStreamNonBlocking) == cudaSuccess &&
+              cudaEventCreateWithFlags(&ds->io_ev_end, cudaEventDisableTiming) == cudaSuccess;
+    for (int i = 0; ok && i < 16; ++i)
+      ok = cudaEventCreateWithFlags(&ds->io_ev_in[i], cudaEventDisableTiming) == cudaSuccess &&
+           cudaEventCreateWithFlags(&ds->io_ev_done[i], cudaEventDisableTiming) == cudaSuccess;
+    if (!ok) {
+      cudaGetLastError();
+      return FA_ERR_CUDA;
     }
+    ds->io_ready = true;
   }
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   // Slices run as problems of their own, so slice s's copies in and s-1's

@@ -1,7 +1,10 @@
 /*
- * fa.h - exact, IO-aware attention forward for NVIDIA B200 (sm_100a).
+ * fa.h - exact, IO-aware attention for NVIDIA B200 (sm_100a).
  *
- * One operation: for every batch b, query head h and query row i,
+ * The forward operation, which every fa_fwd* call computes (fa_bwd
+ * differentiates it, fa_fwd_decode evaluates it for a few query rows
+ * against a long key range): for every batch b, query head h and query
+ * row i,
  *
  *     O[b,h,i,:] = softmax_j( scale * Q[b,h,i,:] . K[b,g,j,:] + mask(i,j) ) V[b,g,j,:]
  *     LSE[b,h,i] = log sum_j exp( scale * Q[b,h,i,:] . K[b,g,j,:] + mask(i,j) )
@@ -121,7 +124,8 @@ FA_API int fa_fwd_f32(const float *q, const float *k, const float *v, float *o, 
  * batches when seqlens is given.  The copies go on two streams the library
  * creates once per device; the forward runs on `stream`, which first waits
  * for them.  Before the first copy the copy stream waits for work already
- * queued on `stream`.
+ * queued on `stream`.  Calls from several host threads on one device are
+ * served one at a time.
  *  q_h, k_h, v_h, o_h, lse_h, seqlens_h: host buffers (pinned memory gives
  *  asynchronous copies; seqlens_h may be NULL).
  *  q_d, k_d, v_d, o_d, lse_d, seqlens_d: device buffers of the same sizes
