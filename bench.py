@@ -33,6 +33,28 @@ L2_BYTES = 126 * 1024 * 1024
 FALLBACK_PEAKS = {"bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "hbm_gbs": 6650.0}
 
 
+# Cycles of the spin kernel queued before each single-call start event (about
+# 0.5 ms at B200 clocks).  The GPU is still busy with it while the host
+# queues the timed call, so the events measure device time only and not the
+# host's call overhead.
+LAUNCH_COVER_CYCLES = 1_000_000
+
+
+def flush_l2(buf):
+    """Evict the L2 between timed calls: write `buf` (256 MiB, twice the L2),
+    then read it back, so that the write-backs of its dirty lines happen here
+    and not inside the next timed call."""
+    buf.zero_()
+    buf.sum()
+
+
+def record_start(ev):
+    """Record a start event behind a spin kernel (LAUNCH_COVER_CYCLES)."""
+    import torch
+    torch.cuda._sleep(LAUNCH_COVER_CYCLES)
+    ev.record()
+
+
 def load_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -467,9 +489,9 @@ def report_forward(args, dev):
         times = []
         for _ in range(args.steps):
             if in_bytes < L2_BYTES:
-                flush.zero_()  # inputs smaller than L2: evict them between steps
+                flush_l2(flush)  # inputs smaller than L2: evict them between steps
             e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            e0.record()
+            record_start(e0)
             attention.fwd(q, k, v, causal=w.causal, scale=w.scale, seqlens=sl, out=o, lse=lse)
             e1.record()
             e1.synchronize()
@@ -513,9 +535,9 @@ def report_fp8(args, dev):
     torch.cuda.synchronize(dev)
     times = []
     for _ in range(args.steps):
-        flush.zero_()
+        flush_l2(flush)
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record()
+        record_start(e0)
         attention.fwd_fp8(q, k, vt, **kw)
         e1.record()
         e1.synchronize()
@@ -552,9 +574,9 @@ def report_backward(args, dev):
         torch.cuda.synchronize(dev)
         times = []
         for _ in range(args.steps):
-            flush.zero_()
+            flush_l2(flush)
             e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            e0.record()
+            record_start(e0)
             attention.bwd(q, k, v, o, do, lse, causal=w.causal, scale=w.scale, workspace=ws)
             e1.record()
             e1.synchronize()
@@ -589,9 +611,9 @@ def report_varlen(args, dev):
     torch.cuda.synchronize(dev)
     times = []
     for _ in range(args.steps):
-        flush.zero_()
+        flush_l2(flush)
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record()
+        record_start(e0)
         attention.fwd_varlen(q, k, v, cu, max(lengths), causal=False, scale=w.scale, out=o,
                              lse=lse)
         e1.record()
@@ -627,9 +649,9 @@ def report_decode(args, dev):
     torch.cuda.synchronize(dev)
     times = []
     for _ in range(args.steps):
-        flush.zero_()
+        flush_l2(flush)
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record()
+        record_start(e0)
         attention.fwd_decode(q, k, v, causal=w.causal, scale=w.scale, seqlens=sl, workspace=ws,
                              out=o, lse=lse)
         e1.record()

@@ -19,6 +19,7 @@
 #include "fa.h"
 #include "fa_bwd_sm100.cuh"
 #include "fa_decode.cuh"
+#include "fa_decode_tc.cuh"
 #include "fa_fwd_f32.cuh"
 #include "fa_fwd_sm100.cuh"
 
@@ -38,6 +39,7 @@ struct DeviceState {
   int *status_word = nullptr;  // device address of g_status_word
   bool attr64 = false, attr128 = false;
   bool dec_attr64 = false, dec_attr128 = false;
+  bool dec_tc_attr[2][3] = {};  // [d = 64, 128][4, 8, 16 row slots]
   bool bwd_attr64 = false, bwd_attr128 = false;
   bool fp8_attr = false;
   // fa_fwd_hostio's copy streams and per-slice events, created on first use
@@ -141,6 +143,21 @@ int make_map_packed(CUtensorMap *m, const void *ptr, int total, int H, int d) {
   cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2,
                            static_cast<cuuint64_t>(H) * static_cast<cuuint64_t>(d) * 2};
   cuuint32_t box[3] = {64, 1, 128};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(ptr), dims,
+                        strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? FA_OK : FA_ERR_CUDA;
+}
+
+// The query rows of a decode call, [rows, d] bf16: box = 64 columns x 16
+// rows, 128-byte swizzle; rows past the end read as zero.
+int make_map_qrows(CUtensorMap *m, const void *ptr, int rows, int d) {
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(rows), 1};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2,
+                           static_cast<cuuint64_t>(rows) * static_cast<cuuint64_t>(d) * 2};
+  cuuint32_t box[3] = {64, 16, 1};
   cuuint32_t estr[3] = {1, 1, 1};
   CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(ptr), dims,
                         strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
@@ -387,6 +404,110 @@ int launch_decode(DeviceState *ds, const void *q, const void *k, const void *v, 
   fa::fa_decode_combine_kernel<D><<<cblocks, 128, 0, stream>>>(p);
   if (cudaGetLastError() != cudaSuccess) return FA_ERR_LAUNCH;
   return FA_OK;
+}
+
+// Decode on the tensor cores (up to 16 query rows per kv head): the call's
+// key tiles are shared evenly by `ctas` persistent CTAs, one per SM by
+// default, or num_splits per (batch, kv head) when given.  Each CTA leaves one
+// partial per (batch, kv head) its share touches, so there are at most
+// ctas + B * Hkv of them, 16 row slots each.
+constexpr int kDecodeTcMaxRows = 16;
+constexpr int kDecodeTcAutoCtasMax = 256;
+constexpr long long kDecodeTcCtasMax = 1024;
+
+bool decode_uses_tc(int Hq, int Hkv, int Nq) {
+  return static_cast<long long>(Hq / Hkv) * Nq <= kDecodeTcMaxRows;
+}
+
+int decode_tc_ctas(int B, int Hkv, int num_splits, int num_sms) {
+  if (num_splits > 0)
+    return static_cast<int>(
+        std::min(kDecodeTcCtasMax, static_cast<long long>(num_splits) * B * Hkv));
+  return std::max(1, std::min(num_sms, kDecodeTcAutoCtasMax));
+}
+
+size_t decode_tc_workspace_bytes(int B, int Hkv, int d, int ctas) {
+  const size_t pieces = static_cast<size_t>(ctas) + static_cast<size_t>(B) * Hkv;
+  const size_t o_bytes = pieces * kDecodeTcMaxRows * d * sizeof(float);
+  const size_t ml_bytes = pieces * kDecodeTcMaxRows * 2 * sizeof(float);
+  return ((o_bytes + 255) / 256) * 256 + ml_bytes;
+}
+
+template <int D, int NR>
+int launch_decode_tc_rows(DeviceState *ds, const CUtensorMap &tq, const CUtensorMap &tk,
+                          const CUtensorMap &tv, const fa::DecodeParams &p,
+                          cudaStream_t stream) {
+  using C = fa::DecodeTcCfg<D>;
+  auto kernel = fa::fa_decode_tc_kernel<D, NR>;
+  bool &attr = ds->dec_tc_attr[D == 128][NR == 4 ? 0 : NR == 8 ? 1 : 2];
+  if (!attr) {
+    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             C::SMEM_ALLOC) != cudaSuccess) {
+      cudaGetLastError();
+      return FA_ERR_LAUNCH;
+    }
+    attr = true;
+  }
+  kernel<<<p.ctas, C::THREADS, C::SMEM_ALLOC, stream>>>(tq, tk, tv, p);
+  if (cudaGetLastError() != cudaSuccess) return FA_ERR_LAUNCH;
+  // The merge is a programmatic dependent launch: it may start while the
+  // split kernel finishes and waits for it in the kernel before reading.
+  const long long rows = static_cast<long long>(p.B) * p.Hq * p.Nq;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>((rows + 3) / 4));
+  cfg.blockDim = dim3(128);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = stream;
+  cudaLaunchAttribute pdl[1];
+  pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  pdl[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = pdl;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, fa::fa_decode_tc_combine_kernel<D>, p) != cudaSuccess) {
+    cudaGetLastError();
+    return FA_ERR_LAUNCH;
+  }
+  return FA_OK;
+}
+
+template <int D>
+int launch_decode_tc(DeviceState *ds, const void *q, const void *k, const void *v, void *o,
+                     float *lse, int B, int Hq, int Hkv, int Nq, int Nk, float scale, int causal,
+                     const int *seqlens, int ctas, void *workspace, cudaStream_t stream,
+                     int *status) {
+  CUtensorMap tq, tk, tv;
+  if (make_map_qrows(&tq, q, B * Hq * Nq, D) != FA_OK ||
+      make_map(&tk, k, B * Hkv, Nk, D) != FA_OK || make_map(&tv, v, B * Hkv, Nk, D) != FA_OK)
+    return FA_ERR_CUDA;
+  const size_t pieces = static_cast<size_t>(ctas) + static_cast<size_t>(B) * Hkv;
+  fa::DecodeParams p;
+  p.q = static_cast<const uint16_t *>(q);
+  p.k = static_cast<const uint16_t *>(k);
+  p.v = static_cast<const uint16_t *>(v);
+  p.o = static_cast<uint16_t *>(o);
+  p.lse = lse;
+  p.seqlens = seqlens;
+  p.part_o = static_cast<float *>(workspace);
+  p.part_ml = reinterpret_cast<float *>(
+      static_cast<char *>(workspace) +
+      ((pieces * kDecodeTcMaxRows * D * sizeof(float) + 255) / 256) * 256);
+  p.status = status;
+  p.B = B;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.Nq = Nq;
+  p.Nk = Nk;
+  p.group = Hq / Hkv;
+  p.splits = 0;
+  p.keys_per_split = 0;
+  p.ctas = ctas;
+  p.causal = causal ? 1 : 0;
+  p.scale_log2 = scale * kLog2e;
+  p.wait_limit_ns = kWaitLimitNs;
+  const int rows = p.group * Nq;
+  if (rows <= 4) return launch_decode_tc_rows<D, 4>(ds, tq, tk, tv, p, stream);
+  if (rows <= 8) return launch_decode_tc_rows<D, 8>(ds, tq, tk, tv, p, stream);
+  return launch_decode_tc_rows<D, 16>(ds, tq, tk, tv, p, stream);
 }
 
 size_t bwd_workspace_bytes(int B, int Hq, int N) {
@@ -716,6 +837,9 @@ size_t fa_decode_workspace_size(int B, int Hq, int Hkv, int Nq, int Nk, int d, i
   if (B <= 0 || Hq <= 0 || Hkv <= 0 || Nq <= 0 || Nk <= 0 || (d != 64 && d != 128) ||
       Hq % Hkv != 0 || num_splits < 0)
     return 0;
+  if (decode_uses_tc(Hq, Hkv, Nq))
+    return decode_tc_workspace_bytes(B, Hkv, d,
+                                     decode_tc_ctas(B, Hkv, num_splits, kDecodeTcAutoCtasMax));
   const int groups = ((Hq / Hkv) * Nq + 3) / 4;
   const DecodeSplit sp = decode_split(B, Hkv, groups, Nk, d, num_splits);
   return decode_workspace_bytes(B, Hq, Nq, d, sp.splits);
@@ -728,16 +852,25 @@ int fa_fwd_decode(const void *q, const void *k, const void *v, void *o, float *l
   int rc = check_decode_args(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, scale);
   if (rc != FA_OK) return rc;
   if (num_splits < 0 || num_splits > 128) return FA_ERR_SHAPE;
-  const int groups = ((Hq / Hkv) * Nq + 3) / 4;
-  const DecodeSplit sp = decode_split(B, Hkv, groups, Nk, d, num_splits);
+  // The workspace must hold what fa_decode_workspace_size reports, which does
+  // not depend on the device.
   if (!workspace || !aligned16(workspace) ||
-      workspace_bytes < decode_workspace_bytes(B, Hq, Nq, d, sp.splits))
+      workspace_bytes < fa_decode_workspace_size(B, Hq, Hkv, Nq, Nk, d, num_splits))
     return FA_ERR_WORKSPACE;
   DeviceState *ds = nullptr;
   rc = current_device(&ds);
   if (rc != FA_OK) return rc;
   int *status = status_dev ? status_dev : ds->status_word;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (decode_uses_tc(Hq, Hkv, Nq)) {
+    const int ctas = decode_tc_ctas(B, Hkv, num_splits, ds->num_sms);
+    return d == 64 ? launch_decode_tc<64>(ds, q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, scale, causal,
+                                          seqlens_k, ctas, workspace, st, status)
+                   : launch_decode_tc<128>(ds, q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, scale,
+                                           causal, seqlens_k, ctas, workspace, st, status);
+  }
+  const int groups = ((Hq / Hkv) * Nq + 3) / 4;
+  const DecodeSplit sp = decode_split(B, Hkv, groups, Nk, d, num_splits);
   return d == 64 ? launch_decode<64>(ds, q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, scale, causal,
                                      seqlens_k, sp, workspace, st, status)
                  : launch_decode<128>(ds, q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, scale, causal,
@@ -796,10 +929,15 @@ extern "C" int fa_fwd_decode_noalloc(const void *q, const void *k, const void *v
   int rc = check_decode_args(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, scale);
   if (rc != FA_OK) return rc;
   if (num_splits < 0 || num_splits > 128) return FA_ERR_SHAPE;
+  const bool tc = decode_uses_tc(Hq, Hkv, Nq);
   const int groups = ((Hq / Hkv) * Nq + 3) / 4;
   const DecodeSplit sp = decode_split(B, Hkv, groups, Nk, d, num_splits);
-  if (decode_workspace_bytes(B, Hq, Nq, d, sp.splits) > kNoAllocScratchBytes)
-    return FA_ERR_WORKSPACE;
+  // the size fa_decode_workspace_size reports, so a shape is accepted or
+  // rejected whatever the device
+  const size_t need = tc ? decode_tc_workspace_bytes(
+                               B, Hkv, d, decode_tc_ctas(B, Hkv, num_splits, kDecodeTcAutoCtasMax))
+                         : decode_workspace_bytes(B, Hq, Nq, d, sp.splits);
+  if (need > kNoAllocScratchBytes) return FA_ERR_WORKSPACE;
   DeviceState *ds = nullptr;
   rc = current_device(&ds);
   if (rc != FA_OK) return rc;
@@ -813,6 +951,13 @@ extern "C" int fa_fwd_decode_noalloc(const void *q, const void *k, const void *v
   if (rc != FA_OK) return rc;
   int *status = status_dev ? status_dev : ds->status_word;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (tc) {
+    const int ctas = decode_tc_ctas(B, Hkv, num_splits, ds->num_sms);
+    return d == 64 ? launch_decode_tc<64>(ds, q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, scale, causal,
+                                          seqlens_k, ctas, scratch, st, status)
+                   : launch_decode_tc<128>(ds, q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, scale,
+                                           causal, seqlens_k, ctas, scratch, st, status);
+  }
   return d == 64 ? launch_decode<64>(ds, q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, scale, causal,
                                      seqlens_k, sp, scratch, st, status)
                  : launch_decode<128>(ds, q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, scale, causal,

@@ -1,9 +1,9 @@
-// Split-KV decode forward: a few query rows per (batch, kv head) against a
-// long key/value cache.  The wiki note "FlashAttention" (section on common
-// misconceptions) observes that generating one token is bound by reading the
-// cached K/V, not by arithmetic; at d = 128 and 4 query rows per kv head this
-// path does 4 FLOP per byte read, far below the B200 ridge, so it is written
-// for HBM bandwidth on CUDA cores rather than for the tensor cores.
+// Split-KV decode forward on CUDA cores: query rows per (batch, kv head)
+// against a long key/value cache.  The wiki note "FlashAttention" (section on
+// common misconceptions) observes that generating one token is bound by
+// reading the cached K/V, not by arithmetic.  Calls with up to 16 query rows
+// per kv head run on the tensor cores (fa_decode_tc.cuh); this kernel serves
+// the rest, 4 query rows per CTA, any number of them.
 //
 // Phase 1 (fa_decode_split_kernel): grid = (splits, B * Hkv, row groups).
 //   Each CTA streams the K and V rows of one key range of one (batch, kv head)
@@ -35,6 +35,7 @@ struct DecodeParams {
   int *status;
   int B, Hq, Hkv, Nq, Nk, group;
   int splits, keys_per_split;
+  int ctas;                   // tensor-core path: CTAs sharing the key tiles
   int causal;
   float scale_log2;
   unsigned long long wait_limit_ns;

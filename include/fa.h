@@ -214,14 +214,23 @@ FA_API int fa_fwd_varlen(const void *q, const void *k, const void *v, void *o, f
  *         valid cached keys of sequence b (keys past it are ignored).
  *  causal: 0/1; query i is position len_b - Nq + i of its sequence, so it sees
  *         keys j <= len_b - Nq + i (with Nq = 1: every valid key).
- *  num_splits: key ranges processed in parallel per (batch, kv head), 1..128,
- *         or 0 for an automatic choice (about 16 CTAs per SM of a B200 in
- *         all, at least 256 keys per range).
+ *  Two kernels serve the call, chosen by G * Nq, the query rows per kv head
+ *  (G = Hq / Hkv):
+ *   - G * Nq <= 16: tensor cores.  The call's 128-key tiles of valid keys
+ *     are divided evenly among persistent CTAs, whatever the lengths.
+ *   - G * Nq > 16: CUDA cores, per key range of each (batch, kv head).
+ *  num_splits: 0 for the automatic choice, or 1..128.
+ *   - Tensor-core kernel: 0 gives one CTA per SM; n gives
+ *     min(n * B * Hkv, 1024) CTAs, so each (batch, kv head) is processed by
+ *     about n of them.
+ *   - CUDA-core kernel: the number of key ranges per (batch, kv head); 0
+ *     aims at about 16 CTAs per SM of a B200 with at least 256 keys per
+ *     range.
  *  workspace: DEVICE buffer of at least fa_decode_workspace_size() bytes,
- *         16-byte aligned, owned by the caller; it holds each key range's
- *         partial output, row max and row sum, merged by a second kernel
- *         through their log-sum-exp.  It may be reused across calls that are
- *         ordered on one stream.
+ *         16-byte aligned, owned by the caller.  It holds each CTA's partial
+ *         output, row max and row sum, which a second kernel merges through
+ *         their log-sum-exp.  It may be reused across calls that are ordered
+ *         on one stream.
  * Reference: wiki note "FlashAttention", common misconceptions: generating a
  * single token is bound by reading the cached K/V, and needs decode-oriented
  * kernels; the merge is the same online-softmax update (section "what it

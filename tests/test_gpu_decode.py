@@ -38,8 +38,11 @@ def test_single_query_lengths(Nk, d):
     compare(o, lse, o_r, l_r, o_tol=O_TOL_BF16, lse_tol=LSE_TOL_BF16, what=f"Nk{Nk} d{d}")
 
 
+# Up to 16 query rows per kv head take the tensor-core kernel (4, 8 or 16
+# row slots); more take the CUDA-core kernel: (4, 5) and (8, 3) give 20 and 24.
 @pytest.mark.parametrize("splits", [1, 3, 7, 0])
-@pytest.mark.parametrize("group,nq", [(1, 1), (4, 1), (8, 1), (4, 3), (1, 5)])
+@pytest.mark.parametrize("group,nq", [(1, 1), (4, 1), (8, 1), (4, 3), (1, 5), (4, 4), (4, 5),
+                                      (8, 3)])
 def test_groups_rows_and_splits(group, nq, splits):
     inp = wl.draw(3, 8, 8 // group, 2000, 128, seed=700 + group * 10 + nq, nq=nq)
     inp.seqlens = np.array([2000, 1, 777], dtype=np.int32)
