@@ -9,8 +9,11 @@ causal layer, B=2, Hq=32, Hkv=8, N=8192, d=128, K scaled by 2.
 
 With N > 1 (launched by torch.distributed.run) every rank runs its own
 replica of the workload on its own GPU; there is no data exchange between
-ranks (the work units are independent), so scaling is weak.  Rank 0 prints
-one JSON line.  `--impl reference` times the CPU oracle instead (rank 0 only).
+ranks (the work units are independent), so scaling is weak.  With
+`--shard heads` the ranks instead split one problem by kv-head groups
+(strong scaling); one NCCL all-gather of O after the timed region reports
+what collecting it costs.  Rank 0 prints one JSON line.  `--impl reference`
+times the CPU oracle instead (rank 0 only).
 """
 from __future__ import annotations
 
@@ -113,6 +116,24 @@ def job_throughput(flops_per_step: float, steps: int, ms_max: float, world: int)
     """Whole-job TFLOP/s: `world` replicas each ran `steps` steps in at most
     ms_max milliseconds."""
     return world * flops_per_step * steps / (ms_max * 1e-3) / 1e12
+
+
+def head_shard(Hkv: int, group: int, world: int, rank: int):
+    """Head sharding of one problem: rank r takes the kv heads [g0, g1) and
+    the query heads [h0, h1) = [g0 * group, g1 * group) that share them, so
+    no rank needs another's K or V (work units are independent)."""
+    if Hkv % world:
+        raise ValueError(f"{Hkv} kv heads do not split over {world} ranks")
+    per = Hkv // world
+    g0, g1 = rank * per, (rank + 1) * per
+    return g0, g1, g0 * group, g1 * group
+
+
+def assemble_heads(parts):
+    """O (or LSE) of the whole problem from the ranks' head slices, given in
+    rank order: the slices are concatenated along the head axis (axis 1)."""
+    import torch
+    return torch.cat(list(parts), dim=1)
 
 
 class ClockSampler:
@@ -341,16 +362,32 @@ def run_mine(args, w: wl.Workload):
         import datetime
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=dev)
-    # Each rank: its own replica of the workload (seed offset by rank).
-    inp = wl.draw(w.B, w.Hq, w.Hkv, w.N, w.d, replica_seed(w, rank), k_scale=w.k_scale,
-                  seqlen_range=w.seqlen_range)
+    heads = args.shard == "heads"
+    if heads:
+        # One problem split by kv-head groups: every rank draws the same
+        # inputs and keeps its heads.
+        inp = wl.draw(w.B, w.Hq, w.Hkv, w.N, w.d, w.seed, k_scale=w.k_scale,
+                      seqlen_range=w.seqlen_range)
+        g0, g1, h0, h1 = head_shard(w.Hkv, w.Hq // w.Hkv, world, rank)
+        inp.q_bits = np.ascontiguousarray(inp.q_bits[:, h0:h1])
+        inp.k_bits = np.ascontiguousarray(inp.k_bits[:, g0:g1])
+        inp.v_bits = np.ascontiguousarray(inp.v_bits[:, g0:g1])
+    else:
+        # Each rank: its own replica of the workload (seed offset by rank).
+        inp = wl.draw(w.B, w.Hq, w.Hkv, w.N, w.d, replica_seed(w, rank), k_scale=w.k_scale,
+                      seqlen_range=w.seqlen_range)
     q, k, v = (torch.from_numpy(x).view(torch.bfloat16).to(dev)
                for x in (inp.q_bits, inp.k_bits, inp.v_bits))
     sl = None if inp.seqlens is None else torch.from_numpy(inp.seqlens).to(dev)
     o = torch.empty_like(q)
-    lse = torch.empty((w.B, w.Hq, w.N), dtype=torch.float32, device=dev)
+    lse = torch.empty(q.shape[:3], dtype=torch.float32, device=dev)
     status = torch.zeros(1, dtype=torch.int32, device=dev)
     flops = wl.flops(w, inp.seqlens)
+    if heads:
+        flops = flops * q.shape[1] / w.Hq  # this rank's share of the problem
+    # whole-job throughput: replicas add up; shards of one problem do not
+    job_world = 1 if heads else world
+    job_flops = flops * world if heads else flops
     in_bytes = sum(t.numel() * t.element_size() for t in (q, k, v))
     stream = torch.cuda.current_stream(dev)
 
@@ -388,7 +425,22 @@ def run_mine(args, w: wl.Workload):
         raise RuntimeError("kernel reported a time-out in the timed region")
     ms_max = reduce_max(ms_total, dev)
     ms_per_step = ms_max / args.steps
-    value = job_throughput(flops, args.steps, ms_max, world)
+    value = job_throughput(job_flops, args.steps, ms_max, job_world)
+    gather_ms = None
+    if heads and world > 1:
+        # One all-gather (NCCL) brings O to every rank in head order; timed
+        # apart from the forward, as the cost a caller pays to collect it.
+        parts = [torch.empty_like(o) for _ in range(world)]
+        g_0, g_1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        barrier()
+        g_0.record(stream)
+        dist.all_gather(parts, o)
+        full_o = assemble_heads(parts)
+        g_1.record(stream)
+        torch.cuda.synchronize(dev)
+        gather_ms = reduce_max(g_0.elapsed_time(g_1), dev)
+        assert full_o.shape[1] == w.Hq
+        del parts, full_o
     kernel_tflops = flops / (ms_total / args.steps * 1e-3) / 1e12
 
     # End to end through the C ABI on host buffers: pinned host inputs are
@@ -410,7 +462,7 @@ def run_mine(args, w: wl.Workload):
     e1.record(stream)
     torch.cuda.synchronize(dev)
     e2e_ms = reduce_max(e0.elapsed_time(e1), dev)
-    e2e_value = job_throughput(flops, e2e_steps, e2e_ms, world)
+    e2e_value = job_throughput(job_flops, e2e_steps, e2e_ms, job_world)
     h2d = in_bytes + (0 if sl is None else sl.numel() * 4)
     d2h = o.numel() * 2 + lse.numel() * 4
 
@@ -429,18 +481,21 @@ def run_mine(args, w: wl.Workload):
             tj = json.load(f)
         if tj.get("kernel_source_sha256_16") == kernel_source_hash():
             traffic = tj.get(w.name)
-    cpu, _ = time_oracle(w, inp, budget_s=args.cpu_budget) if not args.no_cpu_baseline else (
-        None, None)
+    # the oracle baseline is timed at N = 1 only, on the whole workload
+    cpu, _ = (time_oracle(w, inp, budget_s=args.cpu_budget)
+              if world == 1 and not args.no_cpu_baseline else (None, None))
     line = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "higher_is_better": True, "scaling": "strong" if heads else "weak",
+        "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded, bf16-rounded N(0,1))",
         "config": dict(workload_config(w),
                        l2=(f"no flush: inputs {in_bytes / 2**20:.0f} MiB > L2 126 MiB"
                            if in_bytes > L2_BYTES else
                            f"not flushed: inputs {in_bytes / 2**20:.1f} MiB fit in L2"),
-                       parallelism=f"replicas x{world}" if world > 1 else "single GPU"),
+                       parallelism=(f"kv-head shards x{world}" if heads and world > 1 else
+                                    f"replicas x{world}" if world > 1 else "single GPU")),
         "roofline": {"bound": "tensor", "achieved": kernel_tflops, "peak": peak,
                      "unit": "TFLOP/s", "frac": kernel_tflops / peak, "traffic": traffic,
                      "peak_source": f"{src} bf16_tflops (burst; kernel timed back to back)"},
@@ -452,6 +507,8 @@ def run_mine(args, w: wl.Workload):
         "gpu_launches": args.steps,
         "cpu_baseline": cpu,
     }
+    if gather_ms is not None:
+        line["o_allgather_ms"] = gather_ms
     print(json.dumps(line), flush=True)
     return 0
 
@@ -462,7 +519,7 @@ def report_all_workloads(args):
     import torch
     dev = torch.device("cuda", 0)
     sections = {"forward": report_forward, "varlen": report_varlen, "decode": report_decode,
-                "backward": report_backward, "fp8": report_fp8}
+                "backward": report_backward, "fp8": report_fp8, "mufu": report_mufu}
     for name, fn in sections.items():
         if args.only in (None, name):
             fn(args, dev)
@@ -628,6 +685,23 @@ def report_varlen(args, dev):
                       "peak_source": src}), flush=True)
 
 
+def report_mufu(args, dev):
+    """The exponential unit's rate, measured (fa_measure_ex2_rate), beside
+    the rate at which the tensor pipe consumes score elements: one ex2 per
+    element against 4d FLOPs of MMA at 8192 dense bf16 FLOP per clock per SM.
+    Below 1, the fraction is the share of the tensor peak the MUFU pipe
+    alone allows unless part of the exponentials run on the FMA pipe."""
+    from exact_io_aware_92_b200 import attention
+    rate = attention.measure_ex2_rate(dev)
+    out = {"probe": "mufu_ex2", "ex2_per_clk_per_sm": rate,
+           "instruction": "ex2.approx.ftz.f32"}
+    for d in (64, 128):
+        consumed = 8192.0 / (4 * d)  # score elements per clock per SM at the tensor peak
+        out[f"tensor_elems_per_clk_d{d}"] = consumed
+        out[f"mufu_cap_frac_of_tensor_peak_d{d}"] = min(1.0, rate / consumed)
+    print(json.dumps(out), flush=True)
+
+
 def report_decode(args, dev):
     """The split-KV decode path: HBM bandwidth against the measured copy rate."""
     import torch
@@ -682,7 +756,10 @@ def main():
     ap.add_argument("--ref-budget", type=float, default=8.0,
                     help="seconds of CPU work per reference-arm step")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--only", choices=["forward", "varlen", "decode", "backward", "fp8"],
+    ap.add_argument("--shard", choices=["replicas", "heads"], default="replicas",
+                    help="N > 1: one replica of the workload per rank (weak scaling), or "
+                         "one problem split by kv-head groups (strong scaling)")
+    ap.add_argument("--only", choices=["forward", "varlen", "decode", "backward", "fp8", "mufu"],
                     default=None, help="with --all-workloads: run one section")
     ap.add_argument("--all-workloads", action="store_true",
                     help="report per-workload throughput for the five workloads instead")

@@ -9,7 +9,7 @@ inputs (``workloads``).
 from . import workloads  # noqa: F401
 
 _API = ("fwd", "bwd", "fwd_fp8", "fwd_varlen", "fwd_decode", "decode_workspace_size", "bwd_workspace_size",
-        "check_status", "fwd_hostio")
+        "check_status", "fwd_hostio", "measure_ex2_rate")
 __all__ = list(_API) + ["workloads"]
 
 

@@ -49,6 +49,7 @@ SIGNATURES = {
                                    _P, _P]),
     "fa_check_status": (_I, [_P, _P]),
     "fa_selftest_bounded_wait": (_I, [_P, ctypes.c_ulonglong, _P]),
+    "fa_measure_ex2_rate": (_I, [ctypes.POINTER(ctypes.c_float), _P]),
     "fa_status_string": (ctypes.c_char_p, [_I]),
     "fa_version": (_I, []),
 }

@@ -5,6 +5,7 @@ PyTorch provides device memory and the current stream; nothing here computes.
 """
 from __future__ import annotations
 
+import ctypes
 import math
 
 import torch
@@ -222,6 +223,16 @@ def check_status(status: torch.Tensor | None = None, device: torch.device | None
     dev = status.device if status is not None else (device or torch.device("cuda"))
     return _lib.load().fa_check_status(None if status is None else status.data_ptr(),
                                        _stream_handle(dev))
+
+
+def measure_ex2_rate(device: torch.device | None = None) -> float:
+    """Calibration: exponentials (ex2.approx.ftz.f32) per SM clock on the
+    current device, the median over SMs (fa_measure_ex2_rate)."""
+    dev = device or torch.device("cuda")
+    out = ctypes.c_float(0.0)
+    _lib.check(_lib.load().fa_measure_ex2_rate(ctypes.byref(out), _stream_handle(dev)),
+               "fa_measure_ex2_rate")
+    return float(out.value)
 
 
 def fwd_hostio(q_h, k_h, v_h, o_h, lse_h, q_d, k_d, v_d, o_d, lse_d, *, causal: bool,

@@ -10,6 +10,7 @@
 #include <cmath>
 #include <cstdint>
 #include <algorithm>
+#include <vector>
 #include <cstring>
 #include <mutex>
 
@@ -587,6 +588,39 @@ __global__ void bounded_wait_selftest_kernel(int *status, unsigned long long lim
                         limit_ns, fa::kErrTimeout);
 }
 
+// Calibration of the exponential unit: every thread runs 8 independent
+// chains x <- 2^(-|x|) of ex2.approx.ftz.f32 (the instruction the softmax
+// uses; the values stay in (0, 1]) and each block records its cycle count and
+// SM.  Sized so that one block per SM keeps the unit busy: 32 warps, 8 chains.
+constexpr int kEx2Threads = 1024, kEx2Chains = 8, kEx2Iters = 2048, kEx2MaxBlocks = 1024;
+__device__ long long g_ex2_cycles[kEx2MaxBlocks];
+__device__ int g_ex2_smid[kEx2MaxBlocks];
+__device__ float g_ex2_sink[kEx2MaxBlocks];
+
+__global__ void __launch_bounds__(kEx2Threads) ex2_rate_kernel() {
+  float x[kEx2Chains];
+#pragma unroll
+  for (int c = 0; c < kEx2Chains; ++c) x[c] = -0.001f * static_cast<float>(threadIdx.x + 37 * c);
+  __syncthreads();
+  const long long t0 = clock64();
+  for (int it = 0; it < kEx2Iters; ++it) {
+#pragma unroll
+    for (int c = 0; c < kEx2Chains; ++c) x[c] = fa::ex2_approx(-fabsf(x[c]));
+  }
+  __syncthreads();
+  const long long t1 = clock64();
+  float acc = 0.f;
+#pragma unroll
+  for (int c = 0; c < kEx2Chains; ++c) acc += x[c];
+  if (acc == 12345.f) g_ex2_sink[blockIdx.x] = acc;  // keeps the chains live
+  if (threadIdx.x == 0) {
+    uint32_t smid;
+    asm volatile("mov.u32 %0, %%smid;" : "=r"(smid));
+    g_ex2_cycles[blockIdx.x] = t1 - t0;
+    g_ex2_smid[blockIdx.x] = static_cast<int>(smid);
+  }
+}
+
 }  // namespace
 
 extern "C" {
@@ -875,6 +909,46 @@ int fa_fwd_decode(const void *q, const void *k, const void *v, void *o, float *l
                                      seqlens_k, sp, workspace, st, status)
                  : launch_decode<128>(ds, q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, scale, causal,
                                       seqlens_k, sp, workspace, st, status);
+}
+
+int fa_measure_ex2_rate(float *ex2_per_clk, void *stream) {
+  if (!ex2_per_clk) return FA_ERR_NULL;
+  DeviceState *ds = nullptr;
+  int rc = current_device(&ds);
+  if (rc != FA_OK) return rc;
+  const int blocks = std::min(ds->num_sms, kEx2MaxBlocks);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  ex2_rate_kernel<<<blocks, kEx2Threads, 0, st>>>();
+  if (cudaGetLastError() != cudaSuccess) return FA_ERR_LAUNCH;
+  if (cudaStreamSynchronize(st) != cudaSuccess) {
+    cudaGetLastError();
+    return FA_ERR_CUDA;
+  }
+  std::vector<long long> cyc(blocks);
+  std::vector<int> sm(blocks);
+  if (cudaMemcpyFromSymbol(cyc.data(), g_ex2_cycles, sizeof(long long) * blocks) != cudaSuccess ||
+      cudaMemcpyFromSymbol(sm.data(), g_ex2_smid, sizeof(int) * blocks) != cudaSuccess) {
+    cudaGetLastError();
+    return FA_ERR_CUDA;
+  }
+  // Per SM: the exponentials of its blocks over the longest of their times
+  // (blocks that shared an SM ran side by side); the median over SMs.
+  std::vector<std::pair<int, long long>> per;  // (smid, cycles), sorted by smid
+  for (int i = 0; i < blocks; ++i) per.emplace_back(sm[i], cyc[i]);
+  std::sort(per.begin(), per.end());
+  std::vector<double> rates;
+  const double ops_per_block = static_cast<double>(kEx2Threads) * kEx2Chains * kEx2Iters;
+  for (size_t i = 0; i < per.size();) {
+    size_t j = i;
+    long long longest = 0;
+    while (j < per.size() && per[j].first == per[i].first) longest = std::max(longest, per[j++].second);
+    if (longest > 0) rates.push_back(ops_per_block * static_cast<double>(j - i) / longest);
+    i = j;
+  }
+  if (rates.empty()) return FA_ERR_CUDA;
+  std::sort(rates.begin(), rates.end());
+  *ex2_per_clk = static_cast<float>(rates[rates.size() / 2]);
+  return FA_OK;
 }
 
 int fa_selftest_bounded_wait(int *status_dev, unsigned long long limit_ns, void *stream) {

@@ -290,6 +290,23 @@ FA_API int fa_check_status(const int *status_dev, void *stream);
  */
 FA_API int fa_selftest_bounded_wait(int *status_dev, unsigned long long limit_ns, void *stream);
 
+/*
+ * Calibration, not part of the attention path: the throughput of the GPU's
+ * exponential unit for ex2.approx.ftz.f32, the instruction the softmax
+ * steps use.
+ *  - One block of 1024 threads per SM runs 8 independent chains of
+ *    x <- 2^(-|x|) each, for 2048 steps, and records its clock cycles and
+ *    its SM.
+ *  - The call waits for `stream` and writes to *ex2_per_clk (host) the
+ *    median over SMs of exponentials per SM clock.
+ *  - One exponential per score element is needed against 4d FLOPs of MMA,
+ *    so this rate bounds the path at ex2_per_clk * 4d FLOP per clock per SM.
+ *  - Its records live in a small static device array: calls that overlap on
+ *    the GPU race.
+ * Returns FA_OK, FA_ERR_NULL, FA_ERR_ARCH, FA_ERR_LAUNCH or FA_ERR_CUDA.
+ */
+FA_API int fa_measure_ex2_rate(float *ex2_per_clk, void *stream);
+
 /* Human-readable text for an fa_status code (static storage). */
 FA_API const char *fa_status_string(int status);
 

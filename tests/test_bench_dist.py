@@ -80,3 +80,48 @@ def test_two_gloo_ranks():
 def test_single_process_needs_no_group():
     assert bench.reduce_max(3.5, "cpu") == 3.5
     assert bench.job_throughput(2e12, 10, 1000.0, 1) == 20.0
+
+
+def _shard_worker(rank, world, port, queue):
+    import datetime
+
+    import torch
+    import torch.distributed as dist
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank),
+                      WORLD_SIZE=str(world), LOCAL_RANK=str(rank))
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=60))
+    try:
+        B, Hq, Hkv, N, d = 2, 8, 4, 5, 3
+        full = torch.arange(B * Hq * N * d, dtype=torch.float32).reshape(B, Hq, N, d)
+        g0, g1, h0, h1 = bench.head_shard(Hkv, Hq // Hkv, world, rank)
+        mine = full[:, h0:h1].contiguous()  # what this rank computes
+        parts = [torch.empty_like(mine) for _ in range(world)]
+        dist.all_gather(parts, mine)
+        queue.put((rank, (g0, g1, h0, h1), bool(torch.equal(bench.assemble_heads(parts), full))))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_head_shards_cover_the_problem_and_gather_back():
+    """--shard heads: the ranks' kv-head blocks tile [0, Hkv), each with the
+    query heads that share it, and the all-gathered slices reassemble O."""
+    world, port = 2, _free_port()
+    ctx = mp.get_context("spawn")
+    queue = ctx.Queue()
+    procs = [ctx.Process(target=_shard_worker, args=(r, world, port, queue)) for r in range(world)]
+    for p in procs:
+        p.start()
+    results = sorted(queue.get(timeout=240) for _ in range(world))
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    assert [r[1] for r in results] == [(0, 2, 0, 4), (2, 4, 4, 8)]
+    assert all(r[2] for r in results)
+
+
+def test_head_shard_rejects_uneven_splits():
+    import pytest
+    with pytest.raises(ValueError):
+        bench.head_shard(8, 4, 3, 0)
+    assert bench.head_shard(8, 4, 8, 7) == (7, 8, 28, 32)

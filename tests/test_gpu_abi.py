@@ -101,3 +101,14 @@ def test_launch_errors_are_returned_not_raised_on_device():
                     1, 2, 2, 64, 64, 0.125, 0, None)
     assert rc == _lib.FA_ERR_ALIGN
     assert lib.fa_check_status(None, None) == _lib.FA_OK
+
+
+def test_ex2_rate_calibration():
+    """fa_measure_ex2_rate measures the exponential unit on the device: a
+    rate between 4 and 64 per SM clock (the B200's MUFU pipe is documented
+    publicly at 16 per clock per SM for fp32 ex2; the test only requires a
+    plausible order of magnitude, the figure itself is reported by bench.py)."""
+    from exact_io_aware_92_b200 import attention
+    rate = attention.measure_ex2_rate()
+    print("ex2 per clock per SM:", rate)
+    assert 4.0 <= rate <= 64.0
