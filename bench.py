@@ -465,6 +465,41 @@ def run_mine(args, w: wl.Workload):
     e2e_value = job_throughput(job_flops, e2e_steps, e2e_ms, job_world)
     h2d = in_bytes + (0 if sl is None else sl.numel() * 4)
     d2h = o.numel() * 2 + lse.numel() * 4
+    # The copy rates of this host link alone (plain pinned copies of the same
+    # bytes, one direction at a time): what bounds the end-to-end step.
+    c0, c1, c2 = (torch.cuda.Event(enable_timing=True) for _ in range(3))
+    c0.record(stream)
+    for t_d, t_h in ((q, q_h), (k, k_h), (v, v_h)):
+        t_d.view(torch.int16).copy_(t_h.view(torch.int16), non_blocking=True)
+    c1.record(stream)
+    o_h.copy_(o.view(torch.int16), non_blocking=True)
+    lse_h.copy_(lse, non_blocking=True)
+    c2.record(stream)
+    torch.cuda.synchronize(dev)
+    h2d_ms, d2h_ms = c0.elapsed_time(c1), c1.elapsed_time(c2)
+    # both directions at once, on two streams (what the overlapped call needs)
+    s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    b0, b1, b2 = (torch.cuda.Event(enable_timing=True) for _ in range(3))
+    torch.cuda.synchronize(dev)
+    b0.record(stream)
+    s_in.wait_event(b0)
+    s_out.wait_event(b0)
+    with torch.cuda.stream(s_in):
+        for t_d, t_h in ((q, q_h), (k, k_h), (v, v_h)):
+            t_d.view(torch.int16).copy_(t_h.view(torch.int16), non_blocking=True)
+        b1.record(s_in)
+    with torch.cuda.stream(s_out):
+        o_h.copy_(o.view(torch.int16), non_blocking=True)
+        lse_h.copy_(lse, non_blocking=True)
+        b2.record(s_out)
+    torch.cuda.synchronize(dev)
+    both_ms = max(b0.elapsed_time(b1), b0.elapsed_time(b2))
+    link = {"h2d_gbs": in_bytes / h2d_ms / 1e6, "d2h_gbs": d2h / d2h_ms / 1e6,
+            "both_directions_ms": both_ms,
+            "copy_bound_ms_per_step": max(h2d_ms, d2h_ms, both_ms),
+            "e2e_ms_per_step": e2e_ms / e2e_steps,
+            "note": "plain pinned copies of one step's bytes: each direction alone, "
+                    "then both at once on two streams"}
 
     if world > 1:
         dist.barrier()
@@ -503,7 +538,7 @@ def run_mine(args, w: wl.Workload):
         "pct_of_nominal_peak": 100.0 * kernel_tflops / NOMINAL_BF16_TFLOPS,
         "clocks": clocks,
         "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
-                "d2h_bytes_per_step": d2h},
+                "d2h_bytes_per_step": d2h, "link": link},
         "gpu_launches": args.steps,
         "cpu_baseline": cpu,
     }

@@ -119,7 +119,7 @@ FA_API int fa_fwd_f32(const float *q, const float *k, const float *v, float *o, 
 /*
  * End-to-end call on HOST buffers: copies q, k, v (and seqlens) from host to
  * the caller's device buffers, runs the bf16 forward and copies o and lse
- * back, then waits.  The work runs in up to 16 slices so that copies overlap
+ * back, then waits.  The work runs in up to 8 slices so that copies overlap
  * the forward: runs of consecutive (batch, kv head) pairs, or of whole
  * batches when seqlens is given.  The copies go on two streams the library
  * creates once per device; the forward runs on `stream`, which first waits

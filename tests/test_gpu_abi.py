@@ -58,7 +58,7 @@ def test_hostio_matches_device_call():
 @pytest.mark.parametrize("B,Hq,Hkv,N,d", [(3, 8, 2, 300, 128), (4, 16, 8, 200, 64)])
 def test_hostio_kv_head_slices_match_device_call(B, Hq, Hkv, N, d):
     # Without key lengths the host path runs in slices of consecutive
-    # (batch, kv head) pairs (6 slices, then 32 pairs in 16 slices); each
+    # (batch, kv head) pairs (6 slices, then 32 pairs in 8 slices); each
     # work unit is computed alike in any launch, so results are identical.
     torch = _torch()
     inp = wl.draw(B, Hq, Hkv, N, d, seed=21)
