@@ -50,6 +50,13 @@ struct DeviceState {
   bool io_ready = false;
   cudaStream_t io_in = nullptr, io_out = nullptr;
   cudaEvent_t io_ev_in[16] = {}, io_ev_done[16] = {}, io_ev_end = nullptr;
+  // fa_bwd's second stream: the dQ kernel runs beside the dK/dV kernel.
+  // bwd_mu covers a call's fork and join, so concurrent callers do not
+  // interleave them.
+  std::mutex bwd_mu;
+  bool bwd_ready = false;
+  cudaStream_t bwd_side = nullptr;
+  cudaEvent_t bwd_fork = nullptr, bwd_join = nullptr;
 };
 DeviceState g_dev[kMaxDevices];
 std::mutex g_mu;
@@ -565,15 +572,41 @@ int launch_bwd(DeviceState *ds, const void *q, const void *k, const void *v, con
   const long long q_units = static_cast<long long>(p.q_tiles) * B * Hq;
   if (prep_blocks > 0x7fffffffll || kv_units > 0x7fffffffll || q_units > 0x7fffffffll)
     return FA_ERR_SHAPE;
+  // The dK/dV and dQ kernels read the same inputs and write disjoint outputs,
+  // so they run side by side: dK/dV on `stream`, dQ on a second stream,
+  // both after the prep kernel.  dK/dV is queued first; as its CTAs run out,
+  // dQ CTAs take the SMs its causal tail leaves idle (about 12 % of its SM
+  // time on the GQA layer when it runs alone).
+  std::lock_guard<std::mutex> lock(ds->bwd_mu);
+  if (!ds->bwd_ready) {
+    if (cudaStreamCreateWithFlags(&ds->bwd_side, cudaStreamNonBlocking) != cudaSuccess ||
+        cudaEventCreateWithFlags(&ds->bwd_fork, cudaEventDisableTiming) != cudaSuccess ||
+        cudaEventCreateWithFlags(&ds->bwd_join, cudaEventDisableTiming) != cudaSuccess) {
+      cudaGetLastError();
+      return FA_ERR_CUDA;
+    }
+    ds->bwd_ready = true;
+  }
   fa::fa_bwd_prep_kernel<D><<<static_cast<unsigned>(prep_blocks), 128, 0, stream>>>(p);
   if (cudaGetLastError() != cudaSuccess) return FA_ERR_LAUNCH;
+  if (cudaEventRecord(ds->bwd_fork, stream) != cudaSuccess ||
+      cudaStreamWaitEvent(ds->bwd_side, ds->bwd_fork, 0) != cudaSuccess) {
+    cudaGetLastError();
+    return FA_ERR_CUDA;
+  }
   fa::fa_bwd_dkdv_kernel<D><<<static_cast<unsigned>(kv_units), C::THREADS, C::SMEM_KV, stream>>>(
       tq, tk, tv, tdo, p);
-  if (cudaGetLastError() != cudaSuccess) return FA_ERR_LAUNCH;
-  fa::fa_bwd_dq_kernel<D><<<static_cast<unsigned>(q_units), C::THREADS, C::SMEM_Q, stream>>>(
-      tq, tk, tv, tdo, p);
-  if (cudaGetLastError() != cudaSuccess) return FA_ERR_LAUNCH;
-  return FA_OK;
+  const bool kv_ok = cudaGetLastError() == cudaSuccess;
+  fa::fa_bwd_dq_kernel<D>
+      <<<static_cast<unsigned>(q_units), C::THREADS, C::SMEM_Q, ds->bwd_side>>>(tq, tk, tv, tdo, p);
+  const bool q_ok = cudaGetLastError() == cudaSuccess;
+  // Join whatever was queued, so `stream` never runs ahead of the dQ kernel.
+  if (cudaEventRecord(ds->bwd_join, ds->bwd_side) != cudaSuccess ||
+      cudaStreamWaitEvent(stream, ds->bwd_join, 0) != cudaSuccess) {
+    cudaGetLastError();
+    return FA_ERR_CUDA;
+  }
+  return kv_ok && q_ok ? FA_OK : FA_ERR_LAUNCH;
 }
 
 // Waits on a barrier that nothing arrives at; the bounded wait must give up.

@@ -150,8 +150,11 @@ FA_API int fa_fwd_hostio(const void *q_h, const void *k_h, const void *v_h, void
  *  seqlens as in fa_fwd.  d in {64, 128}.
  *  workspace: DEVICE buffer of at least fa_bwd_workspace_size(B, Hq, N)
  *  bytes, 16-byte aligned (per-row D = rowsum(dout * o) and LSE*log2(e)).
- * Three kernels run on `stream`: the per-row preprocess, the dK/dV kernel
- * (one CTA per 128-key tile) and the dQ kernel (one CTA per 128-row tile).
+ * Three kernels: the per-row preprocess, then the dK/dV kernel (one CTA per
+ * 128-key tile) on `stream` and the dQ kernel (one CTA per 128-row tile) on
+ * a second stream the library creates once per device.  The dQ kernel
+ * waits for the preprocess, and `stream` waits for the dQ kernel, so all the
+ * work is ordered on `stream` as one call.
  */
 FA_API size_t fa_bwd_workspace_size(int B, int Hq, int N);
 FA_API int fa_bwd(const void *q, const void *k, const void *v, const void *o, const void *dout,
