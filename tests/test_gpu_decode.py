@@ -82,3 +82,33 @@ def test_decode_matches_last_row_of_full_forward():
     torch.cuda.synchronize()
     assert torch.allclose(o_dec[:, :, 0].float(), o_full[:, :, -1].float(), atol=2e-2)
     assert torch.allclose(l_dec[:, :, 0], l_full[:, :, -1], atol=1e-3)
+
+
+@pytest.mark.parametrize("splits", [0, 5, 1])
+@pytest.mark.parametrize("group,nq", [(4, 3), (8, 2)])
+def test_d64_twelve_and_sixteen_rows(group, nq, splits):
+    # d = 64 with 12 and 16 query rows per kv head: the tensor-core kernel's
+    # 16-slot instance, whose PV product stacks the two key halves (N = 32).
+    inp = wl.draw(2, 8, 8 // group, 1500, 64, seed=900 + group * 10 + nq, nq=nq)
+    inp.seqlens = np.array([1500, 613], dtype=np.int32)
+    for causal in (False, True):
+        o, lse = run_decode(inp, causal=causal, scale=0.125, num_splits=splits)
+        o_r, l_r = ref_decode(inp, causal=causal, scale=0.125)
+        compare(o, lse, o_r, l_r, o_tol=O_TOL_BF16, lse_tol=LSE_TOL_BF16,
+                what=f"d64 G{group} nq{nq} splits{splits} causal{causal}")
+
+
+@pytest.mark.parametrize("splits", [1, 2, 0])
+def test_many_short_caches_per_cta(splits):
+    # 40 sequences x 2 kv heads with short, ragged caches (some empty): a
+    # CTA's share of the tiles spans many (batch, kv head) pieces.
+    B = 40
+    inp = wl.draw(B, 8, 2, 300, 128, seed=950 + splits, nq=1)
+    rng = np.random.default_rng(951)
+    lens = rng.integers(0, 301, size=B).astype(np.int32)
+    lens[[3, 17, 29]] = 0
+    inp.seqlens = lens
+    o, lse = run_decode(inp, causal=True, scale=0.088, num_splits=splits)
+    o_r, l_r = ref_decode(inp, causal=True, scale=0.088)
+    compare(o, lse, o_r, l_r, o_tol=O_TOL_BF16, lse_tol=LSE_TOL_BF16,
+            what=f"B{B} short caches splits{splits}")
