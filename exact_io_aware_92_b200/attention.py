@@ -236,15 +236,18 @@ def measure_ex2_rate(device: torch.device | None = None) -> float:
 
 
 def fwd_hostio(q_h, k_h, v_h, o_h, lse_h, q_d, k_d, v_d, o_d, lse_d, *, causal: bool,
-               scale: float, seqlens_h=None, seqlens_d=None) -> None:
+               scale: float, seqlens_h=None, seqlens_d=None, wait: bool = True) -> None:
     """End-to-end call on host tensors (pinned for asynchronous copies):
-    host->device copies, the forward, device->host copies, then a wait."""
+    host->device copies, the forward, device->host copies, then a wait.
+    wait=False (fa_fwd_hostio_async): return once queued on the current
+    stream; consecutive such calls on the same buffers overlap (see fa.h)."""
     B, Hq, N, d = q_h.shape
     Hkv = k_h.shape[1]
-    rc = _lib.load().fa_fwd_hostio(
+    lib = _lib.load()
+    rc = (lib.fa_fwd_hostio if wait else lib.fa_fwd_hostio_async)(
         q_h.data_ptr(), k_h.data_ptr(), v_h.data_ptr(), o_h.data_ptr(), lse_h.data_ptr(),
         None if seqlens_h is None else seqlens_h.data_ptr(), q_d.data_ptr(), k_d.data_ptr(),
         v_d.data_ptr(), o_d.data_ptr(), lse_d.data_ptr(),
         None if seqlens_d is None else seqlens_d.data_ptr(), B, Hq, Hkv, N, d, float(scale),
         int(bool(causal)), _stream_handle(q_d.device))
-    _lib.check(rc, "fa_fwd_hostio")
+    _lib.check(rc, "fa_fwd_hostio" if wait else "fa_fwd_hostio_async")

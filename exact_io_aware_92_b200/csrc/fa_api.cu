@@ -50,6 +50,12 @@ struct DeviceState {
   bool io_ready = false;
   cudaStream_t io_in = nullptr, io_out = nullptr;
   cudaEvent_t io_ev_in[16] = {}, io_ev_done[16] = {}, io_ev_end = nullptr;
+  // The previous call's device buffers, shape and stream; a call with the
+  // same ones (and no key lengths) is chained to it slice by slice.
+  bool io_prev = false;
+  const void *io_prev_ptr[5] = {};
+  int io_prev_shape[5] = {};
+  cudaStream_t io_prev_stream = nullptr;
   // fa_bwd's second stream: the dQ kernel runs beside the dK/dV kernel.
   // bwd_mu covers a call's fork and join, so concurrent callers do not
   // interleave them.
@@ -743,10 +749,14 @@ int fa_check_status(const int *status_dev, void *stream) {
   return word == 0 ? FA_OK : word;
 }
 
-int fa_fwd_hostio(const void *q_h, const void *k_h, const void *v_h, void *o_h, float *lse_h,
-                  const int *seqlens_h, void *q_d, void *k_d, void *v_d, void *o_d, float *lse_d,
-                  int *seqlens_d, int B, int Hq, int Hkv, int N, int d, float scale, int causal,
-                  void *stream) {
+}  // extern "C"
+
+namespace {
+// fa_fwd_hostio and fa_fwd_hostio_async; `wait` makes the call synchronous.
+int hostio_impl(const void *q_h, const void *k_h, const void *v_h, void *o_h, float *lse_h,
+                const int *seqlens_h, void *q_d, void *k_d, void *v_d, void *o_d, float *lse_d,
+                int *seqlens_d, int B, int Hq, int Hkv, int N, int d, float scale, int causal,
+                void *stream, bool wait) {
   if (!q_h || !k_h || !v_h || !o_h || !lse_h) return FA_ERR_NULL;
   if (seqlens_h && !seqlens_d) return FA_ERR_NULL;
   int rc = check_args(q_d, k_d, v_d, o_d, lse_d, B, Hq, Hkv, N, d, scale);
@@ -789,6 +799,7 @@ int fa_fwd_hostio(const void *q_h, const void *k_h, const void *v_h, void *o_h, 
     return static_cast<const uint8_t *>(p) + off * 2;
   };
   auto fail = [&]() {
+    ds->io_prev = false;
     cudaGetLastError();
     cudaStreamSynchronize(ds->io_in);
     cudaStreamSynchronize(ds->io_out);
@@ -796,10 +807,22 @@ int fa_fwd_hostio(const void *q_h, const void *k_h, const void *v_h, void *o_h, 
     cudaGetLastError();
     return FA_ERR_CUDA;
   };
-  // the slices' inputs must not be overwritten before earlier work on the
-  // caller's stream has finished with the device buffers
-  if (cudaEventRecord(ds->io_ev_end, st) != cudaSuccess ||
-      cudaStreamWaitEvent(ds->io_in, ds->io_ev_end, 0) != cudaSuccess)
+  // The slices' inputs must not be overwritten before earlier work has
+  // finished with the device buffers.  An asynchronous call chained to the
+  // previous asynchronous one (same device buffers, shape and stream, no key
+  // lengths) waits per slice for the previous call's forward of that slice,
+  // so its copies in start while the previous call's last slices are
+  // computed and copied out; any other call waits for all earlier work on
+  // `stream`.  The forward of a slice runs on `stream`, after the previous
+  // call's copies out (joined to `stream` at the end of every call).
+  const void *ptrs[5] = {q_d, k_d, v_d, o_d, lse_d};
+  const int shape[5] = {B, Hq, Hkv, N, d};
+  const bool chained = !wait && !seqlens_h && ds->io_prev && ds->io_prev_stream == st &&
+                       std::equal(ptrs, ptrs + 5, ds->io_prev_ptr) &&
+                       std::equal(shape, shape + 5, ds->io_prev_shape);
+  ds->io_prev = false;
+  if (!chained && (cudaEventRecord(ds->io_ev_end, st) != cudaSuccess ||
+                   cudaStreamWaitEvent(ds->io_in, ds->io_ev_end, 0) != cudaSuccess))
     return fail();
   if (seqlens_h && cudaMemcpyAsync(seqlens_d, seqlens_h, sizeof(int) * B, cudaMemcpyHostToDevice,
                                    ds->io_in) != cudaSuccess)
@@ -809,6 +832,8 @@ int fa_fwd_hostio(const void *q_h, const void *k_h, const void *v_h, void *o_h, 
     const int u1 = static_cast<int>(static_cast<long long>(units) * (s + 1) / nslices);
     const int nu = u1 - u0;
     const size_t qo = q_unit * u0, ko = k_unit * u0, lo = l_unit * u0;
+    if (chained && cudaStreamWaitEvent(ds->io_in, ds->io_ev_done[s], 0) != cudaSuccess)
+      return fail();
     if (cudaMemcpyAsync(const_cast<uint8_t *>(bytes16(q_d, qo)), bytes16(q_h, qo),
                         q_unit * nu * 2, cudaMemcpyHostToDevice, ds->io_in) != cudaSuccess ||
         cudaMemcpyAsync(const_cast<uint8_t *>(bytes16(k_d, ko)), bytes16(k_h, ko),
@@ -840,7 +865,32 @@ int fa_fwd_hostio(const void *q_h, const void *k_h, const void *v_h, void *o_h, 
   if (cudaEventRecord(ds->io_ev_end, ds->io_out) != cudaSuccess ||
       cudaStreamWaitEvent(st, ds->io_ev_end, 0) != cudaSuccess)
     return fail();
-  return fa_check_status(nullptr, stream);
+  if (!wait && !seqlens_h) {
+    std::copy(ptrs, ptrs + 5, ds->io_prev_ptr);
+    std::copy(shape, shape + 5, ds->io_prev_shape);
+    ds->io_prev_stream = st;
+    ds->io_prev = true;
+  }
+  return wait ? fa_check_status(nullptr, stream) : FA_OK;
+}
+}  // namespace
+
+extern "C" {
+
+int fa_fwd_hostio(const void *q_h, const void *k_h, const void *v_h, void *o_h, float *lse_h,
+                  const int *seqlens_h, void *q_d, void *k_d, void *v_d, void *o_d, float *lse_d,
+                  int *seqlens_d, int B, int Hq, int Hkv, int N, int d, float scale, int causal,
+                  void *stream) {
+  return hostio_impl(q_h, k_h, v_h, o_h, lse_h, seqlens_h, q_d, k_d, v_d, o_d, lse_d, seqlens_d,
+                     B, Hq, Hkv, N, d, scale, causal, stream, true);
+}
+
+int fa_fwd_hostio_async(const void *q_h, const void *k_h, const void *v_h, void *o_h,
+                        float *lse_h, const int *seqlens_h, void *q_d, void *k_d, void *v_d,
+                        void *o_d, float *lse_d, int *seqlens_d, int B, int Hq, int Hkv, int N,
+                        int d, float scale, int causal, void *stream) {
+  return hostio_impl(q_h, k_h, v_h, o_h, lse_h, seqlens_h, q_d, k_d, v_d, o_d, lse_d, seqlens_d,
+                     B, Hq, Hkv, N, d, scale, causal, stream, false);
 }
 
 int fa_fwd_varlen(const void *q, const void *k, const void *v, void *o, float *lse,

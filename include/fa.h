@@ -139,6 +139,28 @@ FA_API int fa_fwd_hostio(const void *q_h, const void *k_h, const void *v_h, void
                   void *stream);
 
 /*
+ * fa_fwd_hostio without the final wait, for a stream of steps on host
+ * buffers.  Same arguments, same work, ordered on `stream`.  It returns FA_OK
+ * once everything is queued, or an error before anything is queued.
+ * Completion: synchronise `stream` (fa_check_status reads the status word
+ * then).  Host buffers must stay valid and unchanged until then.
+ *
+ * Chaining.  A call that follows another fa_fwd_hostio_async call with the
+ * same device buffers, the same B, Hq, Hkv, N, d and the same stream, without
+ * key lengths, is chained to it.  Its copy into the device buffers for a
+ * slice waits only for the previous call's forward of that slice, not for
+ * all of the previous call's work, so its copies in overlap the previous
+ * call's last forward and copies out.  Between two chained calls, no other
+ * work may read or write q_d, k_d or v_d; o_d and lse_d follow stream order.
+ * Any other call waits for all earlier work on `stream` before it overwrites
+ * the device buffers.
+ */
+FA_API int fa_fwd_hostio_async(const void *q_h, const void *k_h, const void *v_h, void *o_h,
+                               float *lse_h, const int *seqlens_h, void *q_d, void *k_d, void *v_d,
+                               void *o_d, float *lse_d, int *seqlens_d, int B, int Hq, int Hkv,
+                               int N, int d, float scale, int causal, void *stream);
+
+/*
  * Attention backward by recomputation: the gradients of sum(dout * O) for
  * O = fa_fwd(q, k, v, ...), rebuilt from q, k, v, o, dout and the forward's
  * LSE without any stored probability matrix (interview notes "Why is

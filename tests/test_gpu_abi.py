@@ -78,6 +78,38 @@ def test_hostio_kv_head_slices_match_device_call(B, Hq, Hkv, N, d):
         assert np.array_equal(lse_h.numpy(), lse_ref.astype(np.float32))
 
 
+def test_hostio_async_chained_steps():
+    """Three fa_fwd_hostio_async calls in a row with different host inputs
+    and outputs through the same device buffers: the second and third are
+    chained (each slice's copy in waits only for the previous call's forward
+    of that slice).  Every call's host output must equal the device call on
+    its own inputs."""
+    torch = _torch()
+    from exact_io_aware_92_b200 import attention
+    B, Hq, Hkv, N, d = 2, 8, 2, 520, 128
+    scale = 1.0 / np.sqrt(d)
+    pin = lambda a: torch.from_numpy(a).pin_memory()  # noqa: E731
+    steps = []
+    for i in range(3):
+        inp = wl.draw(B, Hq, Hkv, N, d, seed=31 + i)
+        ref = run_bf16(inp, causal=True, scale=scale)
+        host = [pin(x) for x in (inp.q_bits, inp.k_bits, inp.v_bits)]
+        o_h = torch.empty(host[0].shape, dtype=torch.int16).pin_memory()
+        lse_h = torch.empty((B, Hq, N), dtype=torch.float32).pin_memory()
+        steps.append((host, o_h, lse_h, ref))
+    q_d, k_d, v_d = (torch.empty(x.shape, dtype=torch.int16, device="cuda")
+                     for x in steps[0][0])
+    o_d = torch.empty_like(q_d)
+    lse_d = torch.empty((B, Hq, N), dtype=torch.float32, device="cuda")
+    for (q_h, k_h, v_h), o_h, lse_h, _ in steps:
+        attention.fwd_hostio(q_h, k_h, v_h, o_h, lse_h, q_d, k_d, v_d, o_d, lse_d, causal=True,
+                             scale=scale, wait=False)
+    assert attention.check_status() == 0  # waits for the stream
+    for _, o_h, lse_h, (o_ref, lse_ref) in steps:
+        assert np.array_equal(o_h.view(torch.bfloat16).float().numpy(), o_ref.astype(np.float32))
+        assert np.array_equal(lse_h.numpy(), lse_ref.astype(np.float32))
+
+
 def test_bounded_wait_gives_up_and_context_survives():
     torch = _torch()
     lib = _lib.load()
