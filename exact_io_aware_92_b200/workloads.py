@@ -61,8 +61,9 @@ LLAMA_GQA = Workload("llama_gqa_causal_b2_hq32_hkv8_n8192_d128", 2, 32, 8, 8192,
 LONG = Workload("long_causal_b1_h16_n32768_d128", 1, 16, 16, 32768, 128, True, seed=5,
                 sample_rows=256)
 
-# Decode against a KV cache (SURVEY "next" row): one new token per sequence,
-# the Llama-style GQA heads, caches of 16K-32K tokens.
+# Decode against a KV cache (wiki note "FlashAttention", common misconceptions:
+# one generated token is bound by reading the cache): one new token per
+# sequence, the Llama-style GQA heads, caches of 16K-32K tokens.
 DECODE = Workload("llama_gqa_decode_b8_hq32_hkv8_nq1_nk32768_d128", 8, 32, 8, 32768, 128, True,
                   seed=6, seqlen_range=(16384, 32768), nq=1)
 
