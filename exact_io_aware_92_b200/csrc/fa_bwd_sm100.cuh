@@ -347,23 +347,34 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
         tmem_ld32(tS, sv);
         tmem_ld32(tS + 64, dp);
         tmem_wait_ld();
+        // Only a block on the diagonal tile has queries above some key
+        // (query tile == key tile): elsewhere every (i, j) of the block is
+        // visible and the per-element test is skipped (warp-uniform).
+        const bool diag = p.causal && q0 + c0 < key0 + 127;
         uint32_t pk[16], dk[16];
 #pragma unroll
-        for (int x = 0; x < 16; ++x) {
-          float pv[2], dv[2];
+        for (int x4 = 0; x4 < 8; ++x4) {
+          // this block's LSE2 and D values, four columns per shared load
+          const float4 l4 = *reinterpret_cast<const float4 *>(lse2 + c0 + 4 * x4);
+          const float4 d4 = *reinterpret_cast<const float4 *>(delta + c0 + 4 * x4);
+          const float lv[4] = {l4.x, l4.y, l4.z, l4.w}, dl[4] = {d4.x, d4.y, d4.z, d4.w};
+          float pv[4], dv[4];
 #pragma unroll
-          for (int u = 0; u < 2; ++u) {
-            const int c = c0 + 2 * x + u;  // query column within the tile
-            const int i = q0 + c;
-            const bool vis = key_ok && (!p.causal || i >= j);
-            const float pp = vis ? ex2_approx(fmaf(__uint_as_float(sv[2 * x + u]), p.scale_log2,
-                                                   -lse2[c]))
-                                 : 0.f;
+          for (int u = 0; u < 4; ++u) {
+            float pp = ex2_approx(fmaf(__uint_as_float(sv[4 * x4 + u]), p.scale_log2, -lv[u]));
+            if (diag && q0 + c0 + 4 * x4 + u < j) pp = 0.f;
             pv[u] = pp;
-            dv[u] = pp * (__uint_as_float(dp[2 * x + u]) - delta[c]);
+            dv[u] = pp * (__uint_as_float(dp[4 * x4 + u]) - dl[u]);
           }
-          pk[x] = pack_bf16x2(pv[0], pv[1]);
-          dk[x] = pack_bf16x2(dv[0], dv[1]);
+          pk[2 * x4] = pack_bf16x2(pv[0], pv[1]);
+          pk[2 * x4 + 1] = pack_bf16x2(pv[2], pv[3]);
+          dk[2 * x4] = pack_bf16x2(dv[0], dv[1]);
+          dk[2 * x4 + 1] = pack_bf16x2(dv[2], dv[3]);
+        }
+        // keys past the length get no gradient
+        if (!key_ok) {
+#pragma unroll
+          for (int x = 0; x < 16; ++x) pk[x] = dk[x] = 0u;
         }
         // P^T over the first 16 of this block's 32 S^T columns, dS^T over dP^T's.
         tmem_st16(tS, pk);
@@ -622,15 +633,17 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
         tmem_ld32(tS + 64, dp);
         tmem_wait_ld();
         uint32_t dk[16];
+        // When every row of the warp sees all 32 keys of the block (most
+        // blocks), the per-element limit test is skipped (warp-uniform).
+        const int key_first = jt * 128 + 64 * hk + 32 * e;
+        const bool masked = !__all_sync(0xffffffffu, key_first + 31 < limit);
 #pragma unroll
         for (int x = 0; x < 16; ++x) {
           float dv[2];
 #pragma unroll
           for (int u = 0; u < 2; ++u) {
-            const int key = jt * 128 + 64 * hk + 32 * e + 2 * x + u;
-            const float pp = key < limit ? ex2_approx(fmaf(__uint_as_float(sv[2 * x + u]),
-                                                           p.scale_log2, -lse2))
-                                         : 0.f;
+            float pp = ex2_approx(fmaf(__uint_as_float(sv[2 * x + u]), p.scale_log2, -lse2));
+            if (masked && key_first + 2 * x + u >= limit) pp = 0.f;
             dv[u] = pp * (__uint_as_float(dp[2 * x + u]) - delta);
           }
           dk[x] = pack_bf16x2(dv[0], dv[1]);
