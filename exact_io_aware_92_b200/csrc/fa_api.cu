@@ -559,8 +559,8 @@ int launch_bwd(DeviceState *ds, const void *q, const void *k, const void *v, con
   p.dv = static_cast<uint16_t *>(dv);
   p.Npad = (N + 127) / 128 * 128;
   const size_t vec = static_cast<size_t>(B) * Hq * p.Npad;
-  p.ws_lse2 = static_cast<float *>(workspace);
-  p.ws_delta = p.ws_lse2 + vec;
+  p.ws_nlse2 = static_cast<float *>(workspace);
+  p.ws_delta = p.ws_nlse2 + vec;
   p.seqlens = seqlens;
   p.status = status;
   p.B = B;

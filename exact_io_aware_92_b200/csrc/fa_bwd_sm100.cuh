@@ -6,8 +6,8 @@
 // P = exp(scale Q K^T - LSE), dP = dO V^T, D_i = sum_c dO_ic O_ic and
 // dS = P * (dP - D):  dV = P^T dO,  dK = scale dS^T Q,  dQ = scale dS K.
 //
-// fa_bwd_prep_kernel   D and LSE*log2(e) per query row, in a workspace padded
-//                      to whole 128-row tiles (padding: D = 0, LSE = +inf).
+// fa_bwd_prep_kernel   D and -LSE*log2(e) per query row, in a workspace padded
+//                      to whole 128-row tiles (padding: D = 0, -LSE*log2(e) = -inf).
 // fa_bwd_dkdv_kernel   one CTA per 128-key tile of one (batch, kv head); it
 //                      walks the query tiles of every query head of the
 //                      group, each as two halves of 64 queries.  Per half:
@@ -40,7 +40,7 @@ struct BwdParams {
   const uint16_t *o, *dout;   // bf16 [B,Hq,N,d]
   const float *lse;           // fp32 [B,Hq,N]
   uint16_t *dq, *dk, *dv;     // bf16 [B,Hq,N,d], [B,Hkv,N,d] x2
-  float *ws_lse2;             // [B*Hq][Npad]: LSE * log2(e); +inf on padding rows
+  float *ws_nlse2;            // [B*Hq][Npad]: -LSE * log2(e); -inf on padding rows
   float *ws_delta;            // [B*Hq][Npad]: D; 0 on padding rows
   const int *seqlens;
   int *status;
@@ -71,7 +71,8 @@ struct BwdCfg {
 };
 
 // ---------------------------------------------------------------------------
-// Preprocess: D_i = sum_c dO_ic O_ic, LSE2_i = LSE_i * log2(e)
+// Preprocess: D_i = sum_c dO_ic O_ic, NLSE2_i = -LSE_i * log2(e) (stored
+// negated, so the elementwise steps add it in one fused multiply-add)
 // ---------------------------------------------------------------------------
 template <int D>
 __global__ void __launch_bounds__(128) fa_bwd_prep_kernel(const BwdParams p) {
@@ -79,7 +80,7 @@ __global__ void __launch_bounds__(128) fa_bwd_prep_kernel(const BwdParams p) {
   if (row >= static_cast<long long>(p.B) * p.Hq * p.Npad) return;
   const int bh = static_cast<int>(row / p.Npad), i = static_cast<int>(row % p.Npad);
   if (i >= p.N) {
-    p.ws_lse2[row] = INFINITY;
+    p.ws_nlse2[row] = -INFINITY;
     p.ws_delta[row] = 0.f;
     return;
   }
@@ -99,8 +100,8 @@ __global__ void __launch_bounds__(128) fa_bwd_prep_kernel(const BwdParams p) {
   }
   p.ws_delta[row] = acc;
   const float l = p.lse[static_cast<size_t>(bh) * p.N + i];
-  // A row that saw no key keeps no gradient: +inf makes its probabilities 0.
-  p.ws_lse2[row] = (l == -INFINITY) ? INFINITY : l * 1.4426950408889634f;
+  // A row that saw no key keeps no gradient: -inf makes its probabilities 0.
+  p.ws_nlse2[row] = (l == -INFINITY) ? -INFINITY : -l * 1.4426950408889634f;
 }
 
 // Bulk copy of `bytes` (multiple of 16) global -> shared, completing on `bar`.
@@ -111,6 +112,18 @@ __device__ __forceinline__ void bwd_bulk(uint32_t dst, const void *src, uint32_t
           "r"(dst),
       "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(bar)
       : "memory");
+}
+
+// Packed fp32 pair arithmetic beyond fma/add (sm100_ptx.cuh).
+__device__ __forceinline__ uint64_t sub_f32x2(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ uint64_t mul_f32x2_bwd(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
 }
 
 // Load one 128-row x D bf16 tile (two 64-column boxes) with TMA.
@@ -209,7 +222,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
         load_tile<D>(dst, &tm_q, bar_full + 8 * st, qt * 128, bh);
         load_tile<D>(dst + C::TILE_BYTES, &tm_do, bar_full + 8 * st, qt * 128, bh);
         const size_t vrow = static_cast<size_t>(bh) * p.Npad + qt * 128;
-        bwd_bulk(dst + 2 * C::TILE_BYTES, p.ws_lse2 + vrow, 512, bar_full + 8 * st);
+        bwd_bulk(dst + 2 * C::TILE_BYTES, p.ws_nlse2 + vrow, 512, bar_full + 8 * st);
         bwd_bulk(dst + 2 * C::TILE_BYTES + 512, p.ws_delta + vrow, 512, bar_full + 8 * st);
       }
       volatile int never = 0;
@@ -338,9 +351,9 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
       tc_fence_after();
       const int c0 = 64 * hq + 32 * e;  // first query column of this thread's block
       const int q0 = step_qt(s) * 128;
-      const float *lse2 =
+      const float *nlse2 =
           reinterpret_cast<const float *>(smem + C::OFF_RING + st * C::STAGE_BYTES + 2 * C::TILE_BYTES);
-      const float *delta = lse2 + 128;
+      const float *delta = nlse2 + 128;
       const uint32_t tS = tmem + lane_base + hq * 128 + 32 * e;
       {
         uint32_t sv[32], dp[32];
@@ -351,25 +364,37 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
         // (query tile == key tile): elsewhere every (i, j) of the block is
         // visible and the per-element test is skipped (warp-uniform).
         const bool diag = p.causal && q0 + c0 < key0 + 127;
+        const uint64_t scl2 = f32x2(p.scale_log2, p.scale_log2);
         uint32_t pk[16], dk[16];
 #pragma unroll
         for (int x4 = 0; x4 < 8; ++x4) {
-          // this block's LSE2 and D values, four columns per shared load
-          const float4 l4 = *reinterpret_cast<const float4 *>(lse2 + c0 + 4 * x4);
+          // this block's -LSE2 and D values, four columns per shared load;
+          // the arithmetic runs on pairs (fma/sub/mul.rn.f32x2)
+          const float4 l4 = *reinterpret_cast<const float4 *>(nlse2 + c0 + 4 * x4);
           const float4 d4 = *reinterpret_cast<const float4 *>(delta + c0 + 4 * x4);
-          const float lv[4] = {l4.x, l4.y, l4.z, l4.w}, dl[4] = {d4.x, d4.y, d4.z, d4.w};
-          float pv[4], dv[4];
 #pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            float pp = ex2_approx(fmaf(__uint_as_float(sv[4 * x4 + u]), p.scale_log2, -lv[u]));
-            if (diag && q0 + c0 + 4 * x4 + u < j) pp = 0.f;
-            pv[u] = pp;
-            dv[u] = pp * (__uint_as_float(dp[4 * x4 + u]) - dl[u]);
+          for (int h2 = 0; h2 < 2; ++h2) {
+            const int u = 4 * x4 + 2 * h2;  // first of the pair's two columns
+            const uint64_t t = fma_f32x2(
+                f32x2(__uint_as_float(sv[u]), __uint_as_float(sv[u + 1])), scl2,
+                h2 ? f32x2(l4.z, l4.w) : f32x2(l4.x, l4.y));
+            float t0, t1;
+            f32x2_split(t, t0, t1);
+            float p0 = ex2_approx(t0), p1 = ex2_approx(t1);
+            if (diag) {
+              const int i0 = q0 + c0 + u;
+              if (i0 < j) p0 = 0.f;
+              if (i0 + 1 < j) p1 = 0.f;
+            }
+            const uint64_t pp = f32x2(p0, p1);
+            const uint64_t dd = sub_f32x2(
+                f32x2(__uint_as_float(dp[u]), __uint_as_float(dp[u + 1])),
+                h2 ? f32x2(d4.z, d4.w) : f32x2(d4.x, d4.y));
+            float s0, s1;
+            f32x2_split(mul_f32x2_bwd(pp, dd), s0, s1);
+            pk[u >> 1] = pack_bf16x2(p0, p1);
+            dk[u >> 1] = pack_bf16x2(s0, s1);
           }
-          pk[2 * x4] = pack_bf16x2(pv[0], pv[1]);
-          pk[2 * x4 + 1] = pack_bf16x2(pv[2], pv[3]);
-          dk[2 * x4] = pack_bf16x2(dv[0], dv[1]);
-          dk[2 * x4 + 1] = pack_bf16x2(dv[2], dv[3]);
         }
         // keys past the length get no gradient
         if (!key_ok) {
@@ -613,7 +638,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
     const int i = row0 + (threadIdx.x & 127);
     const uint32_t lane_base = static_cast<uint32_t>(warp & 3) * 32u << 16;
     const size_t vrow = static_cast<size_t>(bh) * p.Npad + i;
-    const float lse2 = p.ws_lse2[vrow];
+    const float nlse2 = p.ws_nlse2[vrow];
     const float delta = p.ws_delta[vrow];
     const int limit = p.causal ? min(L, i + 1) : L;
     bool ok = true;
@@ -642,7 +667,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
           float dv[2];
 #pragma unroll
           for (int u = 0; u < 2; ++u) {
-            float pp = ex2_approx(fmaf(__uint_as_float(sv[2 * x + u]), p.scale_log2, -lse2));
+            float pp = ex2_approx(fmaf(__uint_as_float(sv[2 * x + u]), p.scale_log2, nlse2));
             if (masked && key_first + 2 * x + u >= limit) pp = 0.f;
             dv[u] = pp * (__uint_as_float(dp[2 * x + u]) - delta);
           }
