@@ -77,6 +77,26 @@ def test_hostio_requires_device_seqlens_with_host_seqlens(lib):
     assert rc == _lib.FA_ERR_NULL
 
 
+def test_hostio_async_rejects_bad_arguments_before_any_device_call(lib):
+    # the asynchronous form validates exactly like the synchronous one
+    rc = lib.fa_fwd_hostio_async(A, A, A, A, A, A, A, A, A, A, A, None, 1, 2, 1, 128, 64, 0.125, 0,
+                                 None)
+    assert rc == _lib.FA_ERR_NULL
+    rc = lib.fa_fwd_hostio_async(None, A, A, A, A, None, A, A, A, A, A, None, 1, 2, 1, 128, 64,
+                                 0.125, 0, None)
+    assert rc == _lib.FA_ERR_NULL
+    rc = lib.fa_fwd_hostio_async(A, A, A, A, A, None, A, A, A, A, A, None, 1, 3, 2, 128, 64, 0.125,
+                                 0, None)
+    assert rc == _lib.FA_ERR_HEADS
+    rc = lib.fa_fwd_hostio_async(A, A, A, A, A, None, A, A, A, A, A, None, 1, 2, 1, 128, 96, 0.125,
+                                 0, None)
+    assert rc == _lib.FA_ERR_HEADDIM
+
+
+def test_ex2_calibration_needs_an_output(lib):
+    assert lib.fa_measure_ex2_rate(None, None) == _lib.FA_ERR_NULL
+
+
 def test_decode_workspace_size_and_errors(lib):
     n = lib.fa_decode_workspace_size(8, 32, 8, 1, 32768, 128, 0)
     assert n > 0 and n % 4 == 0

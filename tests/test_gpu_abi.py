@@ -110,6 +110,39 @@ def test_hostio_async_chained_steps():
         assert np.array_equal(lse_h.numpy(), lse_ref.astype(np.float32))
 
 
+def test_hostio_async_with_key_lengths_is_not_chained():
+    """Asynchronous calls with key lengths copy seqlens into one device
+    buffer that every slice reads, so they are never chained: each waits for
+    all earlier work.  Two such calls in a row with different inputs and
+    lengths must each equal the device call on their own inputs."""
+    torch = _torch()
+    from exact_io_aware_92_b200 import attention
+    B, Hq, Hkv, N, d = 3, 4, 2, 300, 64
+    scale = 0.125
+    pin = lambda a: torch.from_numpy(a).pin_memory()  # noqa: E731
+    q_d, k_d, v_d = (torch.empty((B, h, N, d), dtype=torch.int16, device="cuda")
+                     for h in (Hq, Hkv, Hkv))
+    o_d = torch.empty_like(q_d)
+    lse_d = torch.empty((B, Hq, N), dtype=torch.float32, device="cuda")
+    sl_d = torch.empty(B, dtype=torch.int32, device="cuda")
+    steps = []
+    for i, lens in enumerate(([300, 17, 0], [1, 299, 150])):
+        inp = wl.draw(B, Hq, Hkv, N, d, seed=41 + i)
+        inp.seqlens = np.array(lens, dtype=np.int32)
+        ref = run_bf16(inp, causal=False, scale=scale)
+        host = [pin(x) for x in (inp.q_bits, inp.k_bits, inp.v_bits)]
+        o_h = torch.empty(host[0].shape, dtype=torch.int16).pin_memory()
+        lse_h = torch.empty((B, Hq, N), dtype=torch.float32).pin_memory()
+        steps.append((host, pin(inp.seqlens), o_h, lse_h, ref))
+    for (q_h, k_h, v_h), sl_h, o_h, lse_h, _ in steps:
+        attention.fwd_hostio(q_h, k_h, v_h, o_h, lse_h, q_d, k_d, v_d, o_d, lse_d, causal=False,
+                             scale=scale, seqlens_h=sl_h, seqlens_d=sl_d, wait=False)
+    assert attention.check_status() == 0
+    for _, _, o_h, lse_h, (o_ref, lse_ref) in steps:
+        assert np.array_equal(o_h.view(torch.bfloat16).float().numpy(), o_ref.astype(np.float32))
+        assert np.array_equal(lse_h.numpy(), lse_ref.astype(np.float32))
+
+
 def test_bounded_wait_gives_up_and_context_survives():
     torch = _torch()
     lib = _lib.load()
