@@ -114,6 +114,28 @@ def test_decode_workspace_size_and_errors(lib):
                              None, None) == _lib.FA_ERR_HEADS
 
 
+def test_decode_workspace_sizes_of_both_kernels(lib):
+    """Up to 16 query rows per kv head (G * Nq) take the tensor-core kernel:
+    partials for at most ctas + B * Hkv pieces, 16 row slots of d + 2 floats,
+    with ctas = 256 by default (one CTA per SM, at most 256) or
+    min(num_splits * B * Hkv, 1024).  Beyond 16 rows the CUDA-core kernel's
+    per-key-range partials apply, so the size jumps at 17 rows."""
+    def tc_bytes(B, Hkv, d, ctas):
+        pieces = ctas + B * Hkv
+        o_bytes = pieces * 16 * d * 4
+        return (o_bytes + 255) // 256 * 256 + pieces * 16 * 2 * 4
+
+    assert lib.fa_decode_workspace_size(8, 32, 8, 1, 32768, 128, 0) == tc_bytes(8, 8, 128, 256)
+    assert lib.fa_decode_workspace_size(8, 32, 8, 4, 32768, 64, 0) == tc_bytes(8, 8, 64, 256)
+    assert lib.fa_decode_workspace_size(3, 8, 2, 1, 2000, 128, 7) == tc_bytes(3, 2, 128, 42)
+    assert lib.fa_decode_workspace_size(64, 64, 16, 1, 4096, 128, 2) == tc_bytes(64, 16, 128, 1024)
+    # 4 query heads per kv head x 4 rows = 16: tensor cores; x 5 = 20: CUDA cores
+    tc16 = lib.fa_decode_workspace_size(2, 8, 2, 4, 1000, 128, 3)
+    cc20 = lib.fa_decode_workspace_size(2, 8, 2, 5, 1000, 128, 3)
+    assert tc16 == tc_bytes(2, 2, 128, 12)
+    assert cc20 != tc_bytes(2, 2, 128, 12) and cc20 > 0
+
+
 def test_without_a_b200_valid_calls_report_arch():
     import torch
     if torch.cuda.is_available():
