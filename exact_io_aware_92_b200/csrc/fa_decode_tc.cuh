@@ -18,7 +18,9 @@
 // the cache lengths.  The part of a CTA's share that lies in one (b, g) is a
 // piece; it produces one partial (O, m, l) per query row in workspace slot
 // c + (b Hkv + g), which is unique per piece.  A second kernel merges each
-// row's pieces through their log-sum-exp.
+// row's pieces through their log-sum-exp; it is launched as a programmatic
+// dependent of this one (this kernel triggers it after set-up, and it waits
+// for this grid to finish before it reads a partial).
 //
 // Roles (224 threads, one CTA per SM):
 //   warps 0-3  softmax: thread t owns key t of the tile (tensor-memory lane t)
