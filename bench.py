@@ -202,7 +202,11 @@ class ClockSampler:
                 self.samples.append((t, float(sm), pw, int(rs)))
             except Exception:
                 pass
-            self.stop_evt.wait(0.01)
+            self.stop_evt.wait(self.PERIOD_S)
+
+    # Poll period.  A contract region of 20 launches lasts under 20 ms, so the
+    # sampler polls every millisecond to see the clocks inside it.
+    PERIOD_S = 0.001
 
     def start(self):
         import threading
@@ -238,7 +242,7 @@ class ClockSampler:
                 "power_w_1s_avg_median": statistics.median(pw),
                 "power_w_1s_avg_max": max(pw),
                 "power_w_instant_max": max(inst) if inst else None,
-                "source": "NVML, 10 ms, timed region only"}
+                "source": f"NVML, every {self.PERIOD_S * 1e3:g} ms, timed region only"}
 
 
 def oracle_sample_rows(w: wl.Workload, rows_per_head: int, seed: int = 1234) -> np.ndarray:
@@ -410,11 +414,13 @@ def run_mine(args, w: wl.Workload):
     torch.cuda.synchronize(dev)
     sampler.start()
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    # The region opens before the first launch is queued: the GPU starts on
+    # it at once, so samples from here on fall inside the timed launches.
+    sampler.region_start()
     start.record(stream)
     for _ in range(args.steps):
         step()
     end.record(stream)
-    sampler.region_start()  # launches are queued; the GPU runs them from here
     end.synchronize()
     sampler.region_stop()
     torch.cuda.synchronize(dev)
@@ -531,12 +537,12 @@ def run_mine(args, w: wl.Workload):
         "higher_is_better": True, "scaling": "strong" if heads else "weak",
         "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded, bf16-rounded N(0,1))",
-        "config": dict(workload_config(w),
-                       l2=(f"no flush: inputs {in_bytes / 2**20:.0f} MiB > L2 126 MiB"
-                           if in_bytes > L2_BYTES else
-                           f"not flushed: inputs {in_bytes / 2**20:.1f} MiB fit in L2"),
-                       parallelism=(f"kv-head shards x{world}" if heads and world > 1 else
-                                    f"replicas x{world}" if world > 1 else "single GPU")),
+        "config": workload_config(w),
+        "run": {"l2": (f"no flush: inputs {in_bytes / 2**20:.0f} MiB > L2 126 MiB"
+                       if in_bytes > L2_BYTES else
+                       f"not flushed: inputs {in_bytes / 2**20:.1f} MiB fit in L2"),
+                "parallelism": (f"kv-head shards x{world}" if heads and world > 1 else
+                                f"replicas x{world}" if world > 1 else "single GPU")},
         "roofline": {"bound": "tensor", "achieved": kernel_tflops, "peak": peak,
                      "unit": "TFLOP/s", "frac": kernel_tflops / peak, "traffic": traffic,
                      "peak_source": f"{src} bf16_tflops (burst; kernel timed back to back)"},

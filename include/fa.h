@@ -288,8 +288,11 @@ FA_API int fa_fwd_decode(const void *q, const void *k, const void *v, void *o, f
  * nothing is launched then.  No call allocates or frees device memory.
  *
  * The first call on a device looks up the array's device address (with that
- * device current) and remembers it; make that first call before any stream
- * capture.  The array keeps the last call's contents: every call writes all
+ * device current) and remembers it for the rest of the process; make that
+ * first call before any stream capture.  The remembered address belongs to
+ * the device's primary context: after cudaDeviceReset on that device it is
+ * no longer valid, so do not call this entry point again in that process.
+ * The array keeps the last call's contents: every call writes all
  * the partials it reads, so nothing needs clearing, but all calls share the
  * one array, so calls that overlap on the GPU (on different streams, or from
  * several host threads) race; order them on one stream.

@@ -46,6 +46,7 @@ def test_sampler_keeps_the_timed_region_and_decodes_reasons(monkeypatch):
     s.region_start()
     time.sleep(0.12)
     s.region_stop()
+    time.sleep(0.01)                 # a poll that began inside the region sees it busy
     state["busy"] = False
     time.sleep(0.06)                 # idle samples after it
     rec = s.stop()
@@ -61,3 +62,34 @@ def test_sampler_without_nvml_says_so(monkeypatch):
     monkeypatch.setitem(sys.modules, "pynvml", None)  # import fails
     rec = bench.ClockSampler(0).stop()
     assert rec["sm_mhz"] is None and rec["reasons"] == ["nvml unavailable"]
+
+
+def test_sampler_sees_a_short_region(monkeypatch):
+    # A contract region of 20 launches lasts under 20 ms; the sampler must
+    # still put samples inside it.
+    import torch
+    state = {"busy": False}
+    monkeypatch.setitem(sys.modules, "pynvml", _fake_nvml(state))
+    monkeypatch.setattr(torch.cuda, "get_device_properties",
+                        lambda i: types.SimpleNamespace(uuid="GPU-1"))
+    s = bench.ClockSampler(0)
+    s.start()
+    time.sleep(0.02)
+    state["busy"] = True
+    s.region_start()
+    time.sleep(0.018)
+    s.region_stop()
+    time.sleep(0.01)
+    state["busy"] = False
+    rec = s.stop()
+    assert rec["samples"] >= 5 and rec["sm_mhz"] == 1500.0
+
+
+def test_both_arms_report_the_same_config_keys():
+    # the reference arm and this arm describe the workload with the same
+    # keys; how a run was made (L2 handling, parallelism) sits under "run"
+    import inspect
+    src = inspect.getsource(bench.run_mine)
+    assert '"config": workload_config(w)' in src and '"run": {' in src
+    ref = inspect.getsource(bench.run_reference)
+    assert '"config": workload_config(w)' in ref
