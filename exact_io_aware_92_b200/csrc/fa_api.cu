@@ -198,6 +198,27 @@ int make_map_u8(CUtensorMap *m, const void *ptr, int planes, int rows, int cols,
   return r == CUDA_SUCCESS ? FA_OK : FA_ERR_CUDA;
 }
 
+// The forward kernels split their registers between warpgroups with
+// setmaxnreg: the softmax warpgroups' increase is served only by what the
+// control warpgroup gives up from the launch allocation.  A build whose
+// kernel was compiled with fewer registers per thread would leave that
+// increase waiting for ever, so such a kernel is never launched.
+template <typename Cfg, typename K>
+int prepare_fwd_kernel(K kernel) {
+  cudaFuncAttributes fa_attr{};
+  if (cudaFuncGetAttributes(&fa_attr, kernel) != cudaSuccess) {
+    cudaGetLastError();
+    return FA_ERR_LAUNCH;
+  }
+  if (static_cast<uint32_t>(fa_attr.numRegs) < Cfg::REGS_LAUNCH) return FA_ERR_LAUNCH;
+  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           Cfg::SMEM_ALLOC) != cudaSuccess) {
+    cudaGetLastError();
+    return FA_ERR_LAUNCH;
+  }
+  return FA_OK;
+}
+
 int launch_fp8(DeviceState *ds, const void *q, const void *k, const void *vt, void *o, float *lse,
                int B, int Hq, int Hkv, int N, int ldvt, float scale, float descale_q,
                float descale_k, float descale_v, int causal, const int *seqlens,
@@ -205,11 +226,8 @@ int launch_fp8(DeviceState *ds, const void *q, const void *k, const void *vt, vo
   using C = fa::Sm100Cfg<128, true>;
   auto kernel = fa::fa_fwd_e4m3_sm100_kernel;
   if (!ds->fp8_attr) {
-    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             C::SMEM_ALLOC) != cudaSuccess) {
-      cudaGetLastError();
-      return FA_ERR_LAUNCH;
-    }
+    const int rc = prepare_fwd_kernel<C>(kernel);
+    if (rc != FA_OK) return rc;
     ds->fp8_attr = true;
   }
   CUtensorMap tq, tk, tvt;
@@ -229,6 +247,9 @@ int launch_fp8(DeviceState *ds, const void *q, const void *k, const void *vt, vo
   p.Hkv = Hkv;
   p.N = N;
   p.group = Hq / Hkv;
+  p.div_bh = fa::make_fast_div(static_cast<uint32_t>(B * Hq));
+  p.div_hq = fa::make_fast_div(static_cast<uint32_t>(Hq));
+  p.div_group = fa::make_fast_div(static_cast<uint32_t>(Hq / Hkv));
   p.num_qpairs = (N + C::ROWS_PER_UNIT - 1) / C::ROWS_PER_UNIT;
   p.causal = causal ? 1 : 0;
   // scores of the codes times the two descales, in log2 units
@@ -254,11 +275,8 @@ int launch_bf16(DeviceState *ds, const void *q, const void *k, const void *v, vo
   auto kernel = fa::fa_fwd_bf16_sm100_kernel<D>;
   bool &attr = (D == 64) ? ds->attr64 : ds->attr128;
   if (!attr) {
-    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             C::SMEM_ALLOC) != cudaSuccess) {
-      cudaGetLastError();
-      return FA_ERR_LAUNCH;
-    }
+    const int rc = prepare_fwd_kernel<C>(kernel);
+    if (rc != FA_OK) return rc;
     attr = true;
   }
   CUtensorMap tq, tk, tv;
@@ -283,6 +301,9 @@ int launch_bf16(DeviceState *ds, const void *q, const void *k, const void *v, vo
   p.Hkv = Hkv;
   p.N = N;
   p.group = Hq / Hkv;
+  p.div_bh = fa::make_fast_div(static_cast<uint32_t>(B * Hq));
+  p.div_hq = fa::make_fast_div(static_cast<uint32_t>(Hq));
+  p.div_group = fa::make_fast_div(static_cast<uint32_t>(Hq / Hkv));
   p.num_qpairs = (N + C::ROWS_PER_UNIT - 1) / C::ROWS_PER_UNIT;
   p.causal = causal ? 1 : 0;
   p.scale_log2 = scale * kLog2e;

@@ -45,6 +45,29 @@
 
 namespace fa {
 
+// Division of non-negative 31-bit integers by a divisor fixed for the whole
+// launch, without a division instruction sequence: with l = ceil(log2 d) and
+// m = floor(2^32 (2^l - d) / d) + 1, n / d = (umulhi(n, m) + n) >> l
+// (Granlund and Montgomery, "Division by invariant integers using
+// multiplication", 1994).  The sum cannot overflow: n < 2^31 and
+// umulhi(n, m) <= n.
+struct FastDiv {
+  uint32_t d, m, l;
+  __device__ __forceinline__ int div(int n) const {
+    const uint32_t un = static_cast<uint32_t>(n);
+    return static_cast<int>((__umulhi(un, m) + un) >> l);
+  }
+};
+
+inline FastDiv make_fast_div(uint32_t d) {
+  FastDiv f;
+  f.d = d;
+  f.l = 0;
+  while ((1ull << f.l) < d) ++f.l;
+  f.m = static_cast<uint32_t>(((1ull << 32) * ((1ull << f.l) - d)) / d + 1);
+  return f;
+}
+
 struct FwdParams {
   uint16_t *o;           // bf16 [B, Hq, N, d], or [total, Hq, d] when packed
   float *lse;            // fp32 [B, Hq, N], or [Hq, total] when packed
@@ -53,6 +76,7 @@ struct FwdParams {
   int total;             // packed layout: tokens in all sequences
   int *status;           // device status word (time-outs)
   int B, Hq, Hkv, N, group;
+  FastDiv div_bh, div_hq, div_group;  // by B * Hq, Hq and group
   int num_qpairs;        // ceil(N / 256)
   int num_units;         // B * Hq * num_qpairs
   int causal;
@@ -105,6 +129,7 @@ struct Sm100Cfg {
   // Registers per thread: 168 at launch (65536 / 384, rounded down to 8);
   // the producer/MMA warpgroup gives some up to the two softmax warpgroups.
   // 128 * REGS_CONTROL + 256 * REGS_SOFTMAX = 384 * 168.
+  static constexpr uint32_t REGS_LAUNCH = 168;
   static constexpr uint32_t REGS_CONTROL = 56;
   static constexpr uint32_t REGS_SOFTMAX = 224;
   static constexpr uint32_t TMEM_COLS = 512;
@@ -155,11 +180,12 @@ __device__ __forceinline__ Unit unit_at(const FwdParams &p, int u) {
   using C = Sm100Cfg<D, F8>;
   Unit x;
   const int BH = p.B * p.Hq;
-  const int qp = p.num_qpairs - 1 - u / BH;
-  x.bh = u % BH;
-  x.b = x.bh / p.Hq;
-  x.h = x.bh % p.Hq;
-  x.hkv = x.h / p.group;
+  const int q_bh = p.div_bh.div(u);
+  const int qp = p.num_qpairs - 1 - q_bh;
+  x.bh = u - q_bh * BH;
+  x.b = p.div_hq.div(x.bh);
+  x.h = x.bh - x.b * p.Hq;
+  x.hkv = p.div_group.div(x.h);
   x.row0 = qp * C::ROWS_PER_UNIT;
   int L = p.N;
   if (p.cu_seqlens) {
