@@ -16,14 +16,21 @@
 //   warps 4-7  softmax warpgroup for Q tile 1
 //   warp  8    TMA producer: Q tiles per unit, then K_j, V_j into a ring of stages
 //   warp  9    MMA issuer: S_t = Q_t K_j^T and O_t += P_t V_j with tcgen05.mma
+//              (role_mma_split at d = 128, role_mma_triple at d = 64,
+//              role_mma for FP8)
 //   warps 10-11 idle (they complete the third warpgroup, whose registers go
 //              to the softmax warpgroups)
 // Tensor memory (512 columns, fp32): S0 [0,128) S1 [128,256) O0 [256,256+d)
-// O1 [384,384+d).  P_t (bf16, packed two per column) overwrites the first 64
-// columns of S_t and feeds the PV product straight from tensor memory; it is
-// published in two halves of 64 keys so the PV product starts on the first
-// half while the second is computed.  In a causal unit, Q tile 0 skips the last
-// key tile when it lies wholly above its rows (Q tile 1 still needs it).
+// O1 [384,384+d).  P_t (bf16, packed two per column) is published in two
+// halves of 64 keys so the PV product starts on the first half while the
+// second is computed.  The first half overwrites the first 32 columns of S_t
+// and feeds the PV product straight from tensor memory.  At d = 128 the
+// second half goes to a 16 KB shared-memory tile per Q tile (K-major,
+// 128-byte swizzled), so S_t of the next key tile is issued right after the
+// first half's PV product, while the softmax still computes the second half;
+// at d = 64 (three S buffers) and for FP8 inputs it overwrites columns 32-63.
+// In a causal unit, Q tile 0 skips the last key tile when it lies wholly above
+// its rows (Q tile 1 still needs it).
 //
 // The same body serves FP8 E4M3 inputs (F8 = true, head dim 128): 8-bit
 // tiles, kind::f8f6f4 products, V given transposed so both products read
@@ -104,7 +111,16 @@ struct Sm100Cfg {
   static constexpr int STAGES = (TILE_BYTES == 32768) ? 4 : 8;
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_KV = OFF_Q + 2 * TILE_BYTES;
-  static constexpr int OFF_BAR = OFF_KV + STAGES * TILE_BYTES;
+  // bf16, d = 128: the upper 64 keys of P go to shared memory (K-major,
+  // 128-byte swizzled: 128 rows of 128 bytes, like a Q tile of 64 columns)
+  // instead of tensor memory, so the next S product may overwrite S_t as soon
+  // as the PV product has read the lower half.  (At d = 64 the three S
+  // buffers already decouple S from P, and the extra shared-memory stores
+  // only lengthen the softmax, which bounds that head dimension.)
+  static constexpr bool P_HI_SMEM = !F8 && D == 128;
+  static constexpr int P_HI_BYTES = 128 * 128;
+  static constexpr int OFF_PHI = OFF_KV + STAGES * TILE_BYTES;  // [2 Q tiles]
+  static constexpr int OFF_BAR = OFF_PHI + (P_HI_SMEM ? 2 * P_HI_BYTES : 0);
   // barrier indices
   static constexpr int BAR_Q_FULL = 0;                  // [2 tiles]
   static constexpr int BAR_Q_EMPTY = 2;                 // [2 tiles]
@@ -120,8 +136,10 @@ struct Sm100Cfg {
   static constexpr int BAR_P_HALF = BAR_S_FULL + NSBUF; // [NSBUF][2 halves of the keys]
   static constexpr int BAR_O_FULL = BAR_P_HALF + 2 * NSBUF;  // [2 tiles]
   static constexpr int BAR_MMA_DONE = BAR_O_FULL + 2;   // 1
-  static constexpr int BAR_PV_DONE = BAR_MMA_DONE + 1;  // [2 tiles] (TRIPLE): a PV product landed
-  static constexpr int NUM_BARS = BAR_PV_DONE + (TRIPLE ? 2 : 0);
+  // [2 tiles] (TRIPLE or P_HI_SMEM): a Q tile's whole PV product landed
+  static constexpr int BAR_PV_DONE = BAR_MMA_DONE + 1;
+  static constexpr bool HAS_PV_DONE = TRIPLE || P_HI_SMEM;
+  static constexpr int NUM_BARS = BAR_PV_DONE + (HAS_PV_DONE ? 2 : 0);
   static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;  // tmem base, abort flag
   static constexpr int SMEM_BYTES = OFF_MISC + 16;
   static constexpr int SMEM_ALLOC = SMEM_BYTES + 1024;     // room to align the base to 1 KB
@@ -238,6 +256,7 @@ struct Sm100Ctx {
   __device__ uint32_t bar(int i) const { return smem + C::OFF_BAR + 8 * i; }
   __device__ uint32_t q_tile(int t) const { return smem + C::OFF_Q + t * C::TILE_BYTES; }
   __device__ uint32_t kv_tile(int slot) const { return smem + C::OFF_KV + slot * C::TILE_BYTES; }
+  __device__ uint32_t p_hi(int t) const { return smem + C::OFF_PHI + t * C::P_HI_BYTES; }
 };
 
 // Ring position of K tile g (V tile g is the next one) in a CTA's stream.
@@ -481,6 +500,171 @@ __device__ void role_mma(const Sm100Ctx<D, F8> &x, const FwdParams &p) {
       commit(C::BAR_O_FULL + 0);
     }
     if (!pv(1, vs, static_cast<uint32_t>((gs[1] + n1 - 1) & 1), n1 > 1)) {
+      ok = false;
+      break;
+    }
+    commit(C::BAR_O_FULL + 1);
+    commit(C::BAR_KV_EMPTY + vs);
+    g += n1;
+    gs[0] += n0;
+    gs[1] += n1;
+    ++qi;
+  }
+  // Every MMA issued above must finish before tensor memory is released.
+  commit(C::BAR_MMA_DONE);
+  volatile int never = 0;
+  mbar_wait_bounded(x.bar(C::BAR_MMA_DONE), 0, &never, p.status, p.wait_limit_ns, kErrTimeout);
+}
+
+// --------------------------------------------------------------------------
+// MMA issuer for two S buffers with P's upper half in shared memory (bf16,
+// D = 128).  Per key tile j and Q tile t: PV_t(j-1) over the lower 64 keys
+// (P from tensor memory), then S_t(j) into the same columns, then PV_t(j-1)
+// over the upper 64 keys (P from shared memory).  S_t(j) thus waits only for
+// the first half of the previous tile's probabilities.
+// --------------------------------------------------------------------------
+template <int D, bool F8>
+__device__ void role_mma_split(const Sm100Ctx<D, F8> &x, const FwdParams &p) {
+  using C = Sm100Cfg<D, F8>;
+  static_assert(C::P_HI_SMEM && !C::TRIPLE, "two S buffers, P's upper half in shared memory");
+  constexpr uint32_t IDESC_S = idesc_bf16_f32(128, C::BN, 0, 0);  // Q, K both K-major
+  constexpr uint32_t IDESC_O = idesc_bf16_f32(128, D, 0, 1);      // P K-major, V MN-major
+  const bool leader = elect_one();
+  const uint32_t tS[2] = {x.tmem + C::COL_S0, x.tmem + C::COL_S0 + 128};
+  const uint32_t tO[2] = {x.tmem + C::COL_O0, x.tmem + C::COL_O0 + C::O_STRIDE};
+  const uint64_t desc_q[2] = {smem_desc_sw128(x.q_tile(0), 16, 1024),
+                              smem_desc_sw128(x.q_tile(1), 16, 1024)};
+  const uint64_t desc_p[2] = {smem_desc_sw128(x.p_hi(0), 16, 1024),
+                              smem_desc_sw128(x.p_hi(1), 16, 1024)};
+  const uint64_t desc_kv_k = smem_desc_sw128(x.kv_tile(0), 16, 1024);
+  const uint64_t desc_kv_v = smem_desc_sw128(x.kv_tile(0), C::BOX_BYTES, 1024);
+  auto wait = [&](int bar, uint32_t parity) {
+    const bool ok = mbar_wait_bounded(x.bar(bar), parity, x.abort_flag, p.status,
+                                      p.wait_limit_ns, kErrTimeout);
+    return __all_sync(0xffffffffu, ok);
+  };
+  auto commit = [&](int bar) {
+    if (leader) tc_commit(x.bar(bar));
+    __syncwarp();
+  };
+  auto issue_s = [&](int t, int ks) {
+    const uint64_t kd = desc_kv_k + ((ks * C::TILE_BYTES) >> 4);
+#pragma unroll
+    for (int kk = 0; kk < C::KSTEPS; ++kk) {
+      const uint32_t off = ((kk / 4) * C::BOX_BYTES + (kk % 4) * 32) >> 4;
+      if (leader) tc_mma_ss(tS[t], desc_q[t] + off, kd + off, IDESC_S, kk > 0 ? 1u : 0u);
+    }
+    __syncwarp();
+  };
+  // O_t += P_t V over keys 0-63: P from tensor memory (8 columns per 16
+  // keys), V steps 16 key rows = 2048 bytes.
+  auto pv_lo = [&](int t, int vs, uint32_t parity, bool accumulate) {
+    if (!wait(C::BAR_P_HALF + 2 * t, parity)) return false;
+    tc_fence_after();
+    const uint64_t vd = desc_kv_v + ((vs * C::TILE_BYTES) >> 4);
+#pragma unroll
+    for (int k4 = 0; k4 < 4; ++k4)
+      if (leader)
+        tc_mma_ts(tO[t], tS[t] + k4 * 8, vd + ((k4 * 2048) >> 4), IDESC_O,
+                  (accumulate || k4 > 0) ? 1u : 0u);
+    __syncwarp();
+    return true;
+  };
+  // O_t += P_t V over keys 64-127: P from shared memory (32 bytes per 16
+  // keys inside its 128-byte rows); then the whole product is marked done.
+  auto pv_hi = [&](int t, int vs, uint32_t parity) {
+    if (!wait(C::BAR_P_HALF + 2 * t + 1, parity)) return false;
+    tc_fence_after();
+    const uint64_t vd = desc_kv_v + ((vs * C::TILE_BYTES) >> 4);
+#pragma unroll
+    for (int k4 = 0; k4 < 4; ++k4)
+      if (leader)
+        tc_mma_ss(tO[t], desc_p[t] + ((k4 * 32) >> 4), vd + (((4 + k4) * 2048) >> 4), IDESC_O,
+                  1u);
+    __syncwarp();
+    commit(C::BAR_PV_DONE + t);
+    return true;
+  };
+
+  int g = 0;             // K/V tiles consumed by this CTA so far (ring position)
+  int gs[2] = {0, 0};    // key tiles each Q tile has processed (its S/P phases)
+  int qi = 0;            // units with keys processed so far
+  bool ok = true;
+  for (int k = 0; ok; ++k) {
+    const int u = snake_unit(k, p.num_units);
+    if (u == -2) break;
+    if (u < 0) continue;
+    const Unit w = unit_at<D, F8>(p, u);
+    const int n1 = w.nkv, n0 = w.nkv0;  // n0 is n1 or n1 - 1
+    if (n1 == 0) continue;
+    const uint32_t qpar = static_cast<uint32_t>(qi & 1);
+    if (!wait(C::BAR_Q_FULL + 0, qpar) || !wait(C::BAR_Q_FULL + 1, qpar) ||
+        !wait(C::BAR_KV_FULL + ring_slot<D, F8>(2 * g), ring_parity<D, F8>(2 * g))) {
+      ok = false;
+      break;
+    }
+    tc_fence_after();
+    issue_s(0, ring_slot<D, F8>(2 * g));
+    commit(C::BAR_S_FULL + 0);
+    if (n0 == 1) commit(C::BAR_Q_EMPTY + 0);
+    issue_s(1, ring_slot<D, F8>(2 * g));
+    commit(C::BAR_S_FULL + 1);
+    commit(C::BAR_KV_EMPTY + ring_slot<D, F8>(2 * g));
+    if (n1 == 1) commit(C::BAR_Q_EMPTY + 1);
+    for (int j = 1; j < n1; ++j) {
+      const int gp = g + j - 1, gc = g + j;
+      const int vs = ring_slot<D, F8>(2 * gp + 1), ks = ring_slot<D, F8>(2 * gc);
+      const uint32_t par0 = static_cast<uint32_t>((gs[0] + j - 1) & 1);
+      const uint32_t par1 = static_cast<uint32_t>((gs[1] + j - 1) & 1);
+      if (!wait(C::BAR_KV_FULL + vs, ring_parity<D, F8>(2 * gp + 1)) ||
+          !pv_lo(0, vs, par0, j - 1 > 0) ||
+          !wait(C::BAR_KV_FULL + ks, ring_parity<D, F8>(2 * gc))) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      if (j < n0) {
+        issue_s(0, ks);
+        commit(C::BAR_S_FULL + 0);
+        if (j == n0 - 1) commit(C::BAR_Q_EMPTY + 0);
+      }
+      if (!pv_hi(0, vs, par0)) {
+        ok = false;
+        break;
+      }
+      if (j >= n0) commit(C::BAR_O_FULL + 0);  // Q tile 0's last PV was issued just above
+      if (!pv_lo(1, vs, par1, j - 1 > 0)) {
+        ok = false;
+        break;
+      }
+      issue_s(1, ks);
+      commit(C::BAR_S_FULL + 1);
+      commit(C::BAR_KV_EMPTY + ks);
+      if (j == n1 - 1) commit(C::BAR_Q_EMPTY + 1);
+      if (!pv_hi(1, vs, par1)) {
+        ok = false;
+        break;
+      }
+      commit(C::BAR_KV_EMPTY + vs);
+    }
+    if (!ok) break;
+    // Last tile's PV products, then the unit's output is complete.
+    const int gl = g + n1 - 1;
+    const int vs = ring_slot<D, F8>(2 * gl + 1);
+    if (!wait(C::BAR_KV_FULL + vs, ring_parity<D, F8>(2 * gl + 1))) {
+      ok = false;
+      break;
+    }
+    if (n0 == n1) {
+      const uint32_t par0 = static_cast<uint32_t>((gs[0] + n1 - 1) & 1);
+      if (!pv_lo(0, vs, par0, n1 > 1) || !pv_hi(0, vs, par0)) {
+        ok = false;
+        break;
+      }
+      commit(C::BAR_O_FULL + 0);
+    }
+    const uint32_t par1 = static_cast<uint32_t>((gs[1] + n1 - 1) & 1);
+    if (!pv_lo(1, vs, par1, n1 > 1) || !pv_hi(1, vs, par1)) {
       ok = false;
       break;
     }
@@ -765,12 +949,14 @@ __device__ void role_softmax(const Sm100Ctx<D, F8> &x, const FwdParams &p, int t
       const float m_use = (m_ref == -INFINITY) ? 0.0f : m_ref;
       store_p(0);
       // O holds earlier tiles' sum only for j > 0; nothing writes it until
-      // this warpgroup publishes P.  With two S buffers the PV product of
-      // tile j-1 finished before S_j did; with three it may still be running,
-      // so its completion is awaited first.  O is rescaled before the first
-      // half goes out.
+      // this warpgroup publishes P.  When S_j is issued after the whole PV
+      // product of tile j-1 (two S buffers in tensor memory, P entirely
+      // there), that product finished before S_j did; otherwise (three S
+      // buffers, or P's upper half in shared memory) it may still be
+      // running, so its completion is awaited first.  O is rescaled before
+      // the first half goes out.
       if (j > 0 && __any_sync(0xffffffffu, need)) {
-        if constexpr (C::TRIPLE) {
+        if constexpr (C::HAS_PV_DONE) {
           if (!wait_all(C::BAR_PV_DONE + t, static_cast<uint32_t>((g + j - 1) & 1))) return;
           tc_fence_after();
         }
@@ -788,9 +974,26 @@ __device__ void role_softmax(const Sm100Ctx<D, F8> &x, const FwdParams &p, int t
       tc_fence_before();
       mbar_arrive(x.bar(C::BAR_P_HALF + 2 * sb));
       // Second half of the keys.
-      exp_half(1, m_use, pk, sum2);
-      store_p(1);
-      tmem_wait_st();
+      if constexpr (C::P_HI_SMEM) {
+        // Row r of the K-major, 128-byte swizzled upper half of P: 16-byte
+        // chunk c of the row's 128 bytes sits at chunk c ^ (r % 8).  The
+        // buffer is free once this Q tile's previous PV product is done.
+        const int gt = g + j;  // key tiles this Q tile processed before this one
+        if (gt > 0 && !wait_all(C::BAR_PV_DONE + t, static_cast<uint32_t>((gt - 1) & 1))) return;
+        exp_half(1, m_use, pk, sum2);
+        // (Storing each chunk as soon as it is packed, interleaved with the
+        // exponentials, measured 3 % slower on the GQA layer.)
+        const uint32_t row = x.p_hi(t) + static_cast<uint32_t>(r) * 128u;
+#pragma unroll
+        for (int c = 0; c < 8; ++c)
+          st_shared_v4(row + (static_cast<uint32_t>(c ^ (r & 7)) << 4), pk[4 * c], pk[4 * c + 1],
+                       pk[4 * c + 2], pk[4 * c + 3]);
+        fence_proxy_async_shared();
+      } else {
+        exp_half(1, m_use, pk, sum2);
+        store_p(1);
+        tmem_wait_st();
+      }
       tc_fence_before();
       mbar_arrive(x.bar(C::BAR_P_HALF + 2 * sb + 1));
       float a0, a1;
@@ -852,7 +1055,7 @@ __device__ __forceinline__ void fwd_kernel_body(const CUtensorMap *tm_q, const C
       mbar_init(x.bar(C::BAR_Q_FULL + t), 1);
       mbar_init(x.bar(C::BAR_Q_EMPTY + t), 1);
       mbar_init(x.bar(C::BAR_O_FULL + t), 1);
-      if (C::TRIPLE) mbar_init(x.bar(C::BAR_PV_DONE + t), 1);
+      if (C::HAS_PV_DONE) mbar_init(x.bar(C::BAR_PV_DONE + t), 1);
     }
     for (int b = 0; b < C::NSBUF; ++b) {
       mbar_init(x.bar(C::BAR_S_FULL + b), 1);
@@ -890,6 +1093,8 @@ __device__ __forceinline__ void fwd_kernel_body(const CUtensorMap *tm_q, const C
     } else if (warp == 9) {
       if constexpr (C::TRIPLE)
         role_mma_triple<D, F8>(x, p);
+      else if constexpr (C::P_HI_SMEM)
+        role_mma_split<D, F8>(x, p);
       else
         role_mma<D, F8>(x, p);
     }
