@@ -38,7 +38,7 @@ struct DeviceState {
   bool ok = false;
   int num_sms = 0;
   int *status_word = nullptr;  // device address of g_status_word
-  bool attr64 = false, attr128 = false;
+  bool attr64 = false, attr64_causal = false, attr128 = false;
   bool dec_attr64 = false, dec_attr128 = false;
   bool dec_tc_attr[2][3] = {};  // [d = 64, 128][4, 8, 16 row slots]
   bool bwd_attr64 = false, bwd_attr128 = false;
@@ -272,8 +272,15 @@ int launch_bf16(DeviceState *ds, const void *q, const void *k, const void *v, vo
                 const int *seqlens, cudaStream_t stream, int *status,
                 const int *cu_seqlens = nullptr, int total = 0) {
   using C = fa::Sm100Cfg<D>;
-  auto kernel = fa::fa_fwd_bf16_sm100_kernel<D>;
-  bool &attr = (D == 64) ? ds->attr64 : ds->attr128;
+  // Causal launches at d = 64 use the instance in which Q tile 0 skips a
+  // unit's last key tile (wholly above its rows) inside the three-buffer
+  // sequence.
+  const bool sk = D == 64 && causal;
+  auto kernel = fa::fa_fwd_bf16_sm100_kernel<D, false>;
+  if constexpr (D == 64) {
+    if (sk) kernel = fa::fa_fwd_bf16_sm100_kernel<64, true>;
+  }
+  bool &attr = sk ? ds->attr64_causal : (D == 64) ? ds->attr64 : ds->attr128;
   if (!attr) {
     const int rc = prepare_fwd_kernel<C>(kernel);
     if (rc != FA_OK) return rc;

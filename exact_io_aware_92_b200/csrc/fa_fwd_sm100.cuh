@@ -95,7 +95,9 @@ struct FwdParams {
 // F8: Q, K and V are FP8 E4M3 codes (head dim 128 only) and V arrives
 // transposed ([d, keys], keys contiguous), so both products read K-major
 // operands; otherwise bf16.
-template <int D, bool F8 = false>
+// SK: causal launches at d = 64, where Q tile 0 skips a unit's last key tile
+// inside the three-buffer sequence; every other launch compiles without it.
+template <int D, bool F8 = false, bool SK = false>
 struct Sm100Cfg {
   static_assert(D == 64 || D == 128, "head dim 64 or 128");
   static_assert(!F8 || D == 128, "FP8 inputs: head dim 128");
@@ -131,6 +133,7 @@ struct Sm100Cfg {
   // interleaved), so a Q tile's next S is computed while it still works on
   // the current one.
   static constexpr bool TRIPLE = (D == 64) && !F8;
+  static constexpr bool SKIP0 = TRIPLE && SK;
   static constexpr int NSBUF = TRIPLE ? 3 : 2;
   static constexpr int BAR_S_FULL = 4 + 2 * STAGES;     // [NSBUF]
   static constexpr int BAR_P_HALF = BAR_S_FULL + NSBUF; // [NSBUF][2 halves of the keys]
@@ -193,9 +196,9 @@ struct Unit {
   size_t lse_base; // offset of row 0 in LSE
 };
 
-template <int D, bool F8>
+template <int D, bool F8, bool SK>
 __device__ __forceinline__ Unit unit_at(const FwdParams &p, int u) {
-  using C = Sm100Cfg<D, F8>;
+  using C = Sm100Cfg<D, F8, SK>;
   Unit x;
   const int BH = p.B * p.Hq;
   const int q_bh = p.div_bh.div(u);
@@ -229,7 +232,8 @@ __device__ __forceinline__ Unit unit_at(const FwdParams &p, int u) {
   const int kv_end = p.causal ? min(L, x.row0 + C::ROWS_PER_UNIT) : L;
   // A unit past the end of its sequence (packed layout) has no rows at all.
   x.nkv = x.row0 < x.q_rows ? (kv_end + C::BN - 1) / C::BN : 0;
-  x.nkv0 = (!C::TRIPLE && p.causal && x.nkv > 1 && (x.nkv - 1) * C::BN >= x.row0 + C::BM)
+  x.nkv0 = ((!C::TRIPLE || C::SKIP0) && p.causal && x.nkv > 1 &&
+             (x.nkv - 1) * C::BN >= x.row0 + C::BM)
                ? x.nkv - 1
                : x.nkv;
   return x;
@@ -246,9 +250,9 @@ __device__ __forceinline__ int snake_unit(int k, int num_units) {
   return u < num_units ? u : -1;
 }
 
-template <int D, bool F8>
+template <int D, bool F8, bool SK>
 struct Sm100Ctx {
-  using C = Sm100Cfg<D, F8>;
+  using C = Sm100Cfg<D, F8, SK>;
   uint32_t smem;      // 1 KB aligned shared base (shared-window address)
   uint32_t tmem;      // tensor-memory base address
   volatile int *abort_flag;
@@ -260,20 +264,20 @@ struct Sm100Ctx {
 };
 
 // Ring position of K tile g (V tile g is the next one) in a CTA's stream.
-template <int D, bool F8>
-__device__ __forceinline__ int ring_slot(int seq) { return seq % Sm100Cfg<D, F8>::STAGES; }
-template <int D, bool F8>
+template <int D, bool F8, bool SK>
+__device__ __forceinline__ int ring_slot(int seq) { return seq % Sm100Cfg<D, F8, SK>::STAGES; }
+template <int D, bool F8, bool SK>
 __device__ __forceinline__ uint32_t ring_parity(int seq) {
-  return static_cast<uint32_t>((seq / Sm100Cfg<D, F8>::STAGES) & 1);
+  return static_cast<uint32_t>((seq / Sm100Cfg<D, F8, SK>::STAGES) & 1);
 }
 
 // --------------------------------------------------------------------------
 // TMA producer (one thread)
 // --------------------------------------------------------------------------
-template <int D, bool F8>
-__device__ void role_producer(const Sm100Ctx<D, F8> &x, const FwdParams &p, const CUtensorMap *tm_q,
+template <int D, bool F8, bool SK>
+__device__ void role_producer(const Sm100Ctx<D, F8, SK> &x, const FwdParams &p, const CUtensorMap *tm_q,
                               const CUtensorMap *tm_k, const CUtensorMap *tm_v) {
-  using C = Sm100Cfg<D, F8>;
+  using C = Sm100Cfg<D, F8, SK>;
   int seq = 0;  // K/V tiles put into the ring so far (K and V counted apart)
   int qi = 0;   // units with keys loaded so far
   const bool packed = p.cu_seqlens != nullptr;
@@ -282,7 +286,7 @@ __device__ void role_producer(const Sm100Ctx<D, F8> &x, const FwdParams &p, cons
     const int u = snake_unit(k, p.num_units);
     if (u == -2) break;
     if (u < 0) continue;
-    const Unit w = unit_at<D, F8>(p, u);
+    const Unit w = unit_at<D, F8, SK>(p, u);
     if (w.nkv == 0) continue;
     // Q tile t of this unit replaces the previous unit's once its last
     // S product has read it.
@@ -305,8 +309,8 @@ __device__ void role_producer(const Sm100Ctx<D, F8> &x, const FwdParams &p, cons
     const int kv_plane = w.kv_plane;
     for (int j = 0; j < w.nkv && ok; ++j) {
       for (int kv = 0; kv < 2; ++kv, ++seq) {
-        const int slot = ring_slot<D, F8>(seq);
-        if (!mbar_wait_bounded(x.bar(C::BAR_KV_EMPTY + slot), ring_parity<D, F8>(seq) ^ 1,
+        const int slot = ring_slot<D, F8, SK>(seq);
+        if (!mbar_wait_bounded(x.bar(C::BAR_KV_EMPTY + slot), ring_parity<D, F8, SK>(seq) ^ 1,
                                x.abort_flag, p.status, p.wait_limit_ns, kErrTimeout)) {
           ok = false;
           break;
@@ -334,7 +338,7 @@ __device__ void role_producer(const Sm100Ctx<D, F8> &x, const FwdParams &p, cons
                         p.wait_limit_ns, kErrTimeout);
   for (int s = 0; s < C::STAGES && s < seq; ++s) {
     const int last = s + C::STAGES * ((seq - 1 - s) / C::STAGES);
-    mbar_wait_bounded(x.bar(C::BAR_KV_FULL + s), ring_parity<D, F8>(last), &never, p.status,
+    mbar_wait_bounded(x.bar(C::BAR_KV_FULL + s), ring_parity<D, F8, SK>(last), &never, p.status,
                       p.wait_limit_ns, kErrTimeout);
   }
 }
@@ -344,9 +348,9 @@ __device__ void role_producer(const Sm100Ctx<D, F8> &x, const FwdParams &p, cons
 // descriptor arithmetic stays warp-uniform; one elected lane issues the
 // tcgen05 instructions and their commits)
 // --------------------------------------------------------------------------
-template <int D, bool F8>
-__device__ void role_mma(const Sm100Ctx<D, F8> &x, const FwdParams &p) {
-  using C = Sm100Cfg<D, F8>;
+template <int D, bool F8, bool SK>
+__device__ void role_mma(const Sm100Ctx<D, F8, SK> &x, const FwdParams &p) {
+  using C = Sm100Cfg<D, F8, SK>;
   // S: Q and K both K-major.  O: P from TMEM; V MN-major (bf16) or V^T
   // K-major (FP8).
   constexpr uint32_t IDESC_S = F8 ? idesc_e4m3_f32(128, C::BN) : idesc_bf16_f32(128, C::BN, 0, 0);
@@ -436,33 +440,33 @@ __device__ void role_mma(const Sm100Ctx<D, F8> &x, const FwdParams &p) {
     const int u = snake_unit(k, p.num_units);
     if (u == -2) break;
     if (u < 0) continue;
-    const Unit w = unit_at<D, F8>(p, u);
+    const Unit w = unit_at<D, F8, SK>(p, u);
     const int n1 = w.nkv, n0 = w.nkv0;  // n0 is n1 or n1 - 1
     if (n1 == 0) continue;
     const uint32_t qpar = static_cast<uint32_t>(qi & 1);
     if (!wait(C::BAR_Q_FULL + 0, qpar) || !wait(C::BAR_Q_FULL + 1, qpar) ||
-        !wait(C::BAR_KV_FULL + ring_slot<D, F8>(2 * g), ring_parity<D, F8>(2 * g))) {
+        !wait(C::BAR_KV_FULL + ring_slot<D, F8, SK>(2 * g), ring_parity<D, F8, SK>(2 * g))) {
       ok = false;
       break;
     }
     tc_fence_after();
     // Tile 0: S for both Q tiles.
-    issue_s(0, ring_slot<D, F8>(2 * g));
+    issue_s(0, ring_slot<D, F8, SK>(2 * g));
     commit(C::BAR_S_FULL + 0);
     if (n0 == 1) commit(C::BAR_Q_EMPTY + 0);
-    issue_s(1, ring_slot<D, F8>(2 * g));
+    issue_s(1, ring_slot<D, F8, SK>(2 * g));
     commit(C::BAR_S_FULL + 1);
-    commit(C::BAR_KV_EMPTY + ring_slot<D, F8>(2 * g));
+    commit(C::BAR_KV_EMPTY + ring_slot<D, F8, SK>(2 * g));
     if (n1 == 1) commit(C::BAR_Q_EMPTY + 1);
     // Steady state: PV of tile j-1, then S of tile j into the same columns
     // (the tensor pipe runs them in order, so P is read before S lands).
     // Q tile 0 stops after its n0 tiles.
     for (int j = 1; j < n1; ++j) {
       const int gp = g + j - 1, gc = g + j;
-      const int vs = ring_slot<D, F8>(2 * gp + 1), ks = ring_slot<D, F8>(2 * gc);
-      if (!wait(C::BAR_KV_FULL + vs, ring_parity<D, F8>(2 * gp + 1)) ||
+      const int vs = ring_slot<D, F8, SK>(2 * gp + 1), ks = ring_slot<D, F8, SK>(2 * gc);
+      if (!wait(C::BAR_KV_FULL + vs, ring_parity<D, F8, SK>(2 * gp + 1)) ||
           !pv(0, vs, static_cast<uint32_t>((gs[0] + j - 1) & 1), j - 1 > 0) ||
-          !wait(C::BAR_KV_FULL + ks, ring_parity<D, F8>(2 * gc))) {
+          !wait(C::BAR_KV_FULL + ks, ring_parity<D, F8, SK>(2 * gc))) {
         ok = false;
         break;
       }
@@ -487,8 +491,8 @@ __device__ void role_mma(const Sm100Ctx<D, F8> &x, const FwdParams &p) {
     if (!ok) break;
     // Last tile's PV products, then the unit's output is complete.
     const int gl = g + n1 - 1;
-    const int vs = ring_slot<D, F8>(2 * gl + 1);
-    if (!wait(C::BAR_KV_FULL + vs, ring_parity<D, F8>(2 * gl + 1))) {
+    const int vs = ring_slot<D, F8, SK>(2 * gl + 1);
+    if (!wait(C::BAR_KV_FULL + vs, ring_parity<D, F8, SK>(2 * gl + 1))) {
       ok = false;
       break;
     }
@@ -523,9 +527,9 @@ __device__ void role_mma(const Sm100Ctx<D, F8> &x, const FwdParams &p) {
 // over the upper 64 keys (P from shared memory).  S_t(j) thus waits only for
 // the first half of the previous tile's probabilities.
 // --------------------------------------------------------------------------
-template <int D, bool F8>
-__device__ void role_mma_split(const Sm100Ctx<D, F8> &x, const FwdParams &p) {
-  using C = Sm100Cfg<D, F8>;
+template <int D, bool F8, bool SK>
+__device__ void role_mma_split(const Sm100Ctx<D, F8, SK> &x, const FwdParams &p) {
+  using C = Sm100Cfg<D, F8, SK>;
   static_assert(C::P_HI_SMEM && !C::TRIPLE, "two S buffers, P's upper half in shared memory");
   constexpr uint32_t IDESC_S = idesc_bf16_f32(128, C::BN, 0, 0);  // Q, K both K-major
   constexpr uint32_t IDESC_O = idesc_bf16_f32(128, D, 0, 1);      // P K-major, V MN-major
@@ -594,31 +598,31 @@ __device__ void role_mma_split(const Sm100Ctx<D, F8> &x, const FwdParams &p) {
     const int u = snake_unit(k, p.num_units);
     if (u == -2) break;
     if (u < 0) continue;
-    const Unit w = unit_at<D, F8>(p, u);
+    const Unit w = unit_at<D, F8, SK>(p, u);
     const int n1 = w.nkv, n0 = w.nkv0;  // n0 is n1 or n1 - 1
     if (n1 == 0) continue;
     const uint32_t qpar = static_cast<uint32_t>(qi & 1);
     if (!wait(C::BAR_Q_FULL + 0, qpar) || !wait(C::BAR_Q_FULL + 1, qpar) ||
-        !wait(C::BAR_KV_FULL + ring_slot<D, F8>(2 * g), ring_parity<D, F8>(2 * g))) {
+        !wait(C::BAR_KV_FULL + ring_slot<D, F8, SK>(2 * g), ring_parity<D, F8, SK>(2 * g))) {
       ok = false;
       break;
     }
     tc_fence_after();
-    issue_s(0, ring_slot<D, F8>(2 * g));
+    issue_s(0, ring_slot<D, F8, SK>(2 * g));
     commit(C::BAR_S_FULL + 0);
     if (n0 == 1) commit(C::BAR_Q_EMPTY + 0);
-    issue_s(1, ring_slot<D, F8>(2 * g));
+    issue_s(1, ring_slot<D, F8, SK>(2 * g));
     commit(C::BAR_S_FULL + 1);
-    commit(C::BAR_KV_EMPTY + ring_slot<D, F8>(2 * g));
+    commit(C::BAR_KV_EMPTY + ring_slot<D, F8, SK>(2 * g));
     if (n1 == 1) commit(C::BAR_Q_EMPTY + 1);
     for (int j = 1; j < n1; ++j) {
       const int gp = g + j - 1, gc = g + j;
-      const int vs = ring_slot<D, F8>(2 * gp + 1), ks = ring_slot<D, F8>(2 * gc);
+      const int vs = ring_slot<D, F8, SK>(2 * gp + 1), ks = ring_slot<D, F8, SK>(2 * gc);
       const uint32_t par0 = static_cast<uint32_t>((gs[0] + j - 1) & 1);
       const uint32_t par1 = static_cast<uint32_t>((gs[1] + j - 1) & 1);
-      if (!wait(C::BAR_KV_FULL + vs, ring_parity<D, F8>(2 * gp + 1)) ||
+      if (!wait(C::BAR_KV_FULL + vs, ring_parity<D, F8, SK>(2 * gp + 1)) ||
           !pv_lo(0, vs, par0, j - 1 > 0) ||
-          !wait(C::BAR_KV_FULL + ks, ring_parity<D, F8>(2 * gc))) {
+          !wait(C::BAR_KV_FULL + ks, ring_parity<D, F8, SK>(2 * gc))) {
         ok = false;
         break;
       }
@@ -650,8 +654,8 @@ __device__ void role_mma_split(const Sm100Ctx<D, F8> &x, const FwdParams &p) {
     if (!ok) break;
     // Last tile's PV products, then the unit's output is complete.
     const int gl = g + n1 - 1;
-    const int vs = ring_slot<D, F8>(2 * gl + 1);
-    if (!wait(C::BAR_KV_FULL + vs, ring_parity<D, F8>(2 * gl + 1))) {
+    const int vs = ring_slot<D, F8, SK>(2 * gl + 1);
+    if (!wait(C::BAR_KV_FULL + vs, ring_parity<D, F8, SK>(2 * gl + 1))) {
       ok = false;
       break;
     }
@@ -690,9 +694,9 @@ __device__ void role_mma_split(const Sm100Ctx<D, F8> &x, const FwdParams &p) {
 // buffer (phase T / 3), PV done per Q tile (one phase per tile), O full per
 // Q tile and unit.
 // --------------------------------------------------------------------------
-template <int D, bool F8>
-__device__ void role_mma_triple(const Sm100Ctx<D, F8> &x, const FwdParams &p) {
-  using C = Sm100Cfg<D, F8>;
+template <int D, bool F8, bool SK>
+__device__ void role_mma_triple(const Sm100Ctx<D, F8, SK> &x, const FwdParams &p) {
+  using C = Sm100Cfg<D, F8, SK>;
   static_assert(C::TRIPLE, "three S buffers: bf16, head dim 64");
   constexpr uint32_t IDESC_S = idesc_bf16_f32(128, C::BN, 0, 0);  // Q, K both K-major
   constexpr uint32_t IDESC_O = idesc_bf16_f32(128, D, 0, 1);      // P from TMEM, V MN-major
@@ -720,39 +724,47 @@ __device__ void role_mma_triple(const Sm100Ctx<D, F8> &x, const FwdParams &p) {
     const int u = snake_unit(k, p.num_units);
     if (u == -2) break;
     if (u < 0) continue;
-    const Unit w = unit_at<D, F8>(p, u);
+    const Unit w = unit_at<D, F8, SK>(p, u);
     const int n = w.nkv;
     if (n == 0) continue;
+    // In a causal unit Q tile 0 may skip the last key tile (it lies wholly
+    // above tile 0's rows): that slot of the sequence issues no products, but
+    // its barriers still complete, so every buffer keeps its phase count.
+    const int n0 = w.nkv0;
     const uint32_t qpar = static_cast<uint32_t>(qi & 1);
     if (!wait(C::BAR_Q_FULL + 0, qpar) || !wait(C::BAR_Q_FULL + 1, qpar)) break;
     const int t0 = T, tend = T + 2 * n;
+    const int t_skip = (C::SKIP0 && n0 < n) ? t0 + 2 * (n - 1) : -1;  // the skipped slot
     // S of sequence index tt (key tile j, Q tile q); K tile j is waited for
     // by Q tile 0's product and released after Q tile 1's.
     auto issue_s = [&](int tt) {
       const int j = (tt - t0) >> 1, q = (tt - t0) & 1;
-      const int ks = ring_slot<D, F8>(2 * (g + j));
+      const int ks = ring_slot<D, F8, SK>(2 * (g + j));
       if (q == 0) {
-        if (!wait(C::BAR_KV_FULL + ks, ring_parity<D, F8>(2 * (g + j)))) return false;
+        if (!wait(C::BAR_KV_FULL + ks, ring_parity<D, F8, SK>(2 * (g + j)))) return false;
         tc_fence_after();
       }
       const uint64_t kd = desc_kv_k + ((ks * C::TILE_BYTES) >> 4);
+      if (!C::SKIP0 || tt != t_skip) {
 #pragma unroll
-      for (int kk = 0; kk < C::KSTEPS; ++kk) {
-        const uint32_t off = ((kk / 4) * C::BOX_BYTES + (kk % 4) * 32) >> 4;
-        if (leader)
-          tc_mma_ss(sbuf(tt), (q ? desc_q1 : desc_q0) + off, kd + off, IDESC_S, kk > 0 ? 1u : 0u);
+        for (int kk = 0; kk < C::KSTEPS; ++kk) {
+          const uint32_t off = ((kk / 4) * C::BOX_BYTES + (kk % 4) * 32) >> 4;
+          if (leader)
+            tc_mma_ss(sbuf(tt), (q ? desc_q1 : desc_q0) + off, kd + off, IDESC_S,
+                      kk > 0 ? 1u : 0u);
+        }
       }
       __syncwarp();
       commit(C::BAR_S_FULL + tt % 3);
       if (q == 1) commit(C::BAR_KV_EMPTY + ks);
-      if (j == n - 1) commit(C::BAR_Q_EMPTY + q);
+      if (j == n - 1 - (C::SKIP0 && q == 0 && t_skip >= 0)) commit(C::BAR_Q_EMPTY + q);
       return true;
     };
     for (int tt = t0; ok && tt < t0 + 3 && tt < tend; ++tt) ok = issue_s(tt);
     for (int tp = t0; ok && tp < tend; ++tp) {
       const int j = (tp - t0) >> 1, q = (tp - t0) & 1;
-      const int vs = ring_slot<D, F8>(2 * (g + j) + 1);
-      if (q == 0 && !wait(C::BAR_KV_FULL + vs, ring_parity<D, F8>(2 * (g + j) + 1))) {
+      const int vs = ring_slot<D, F8, SK>(2 * (g + j) + 1);
+      if (q == 0 && !wait(C::BAR_KV_FULL + vs, ring_parity<D, F8, SK>(2 * (g + j) + 1))) {
         ok = false;
         break;
       }
@@ -767,12 +779,14 @@ __device__ void role_mma_triple(const Sm100Ctx<D, F8> &x, const FwdParams &p) {
           break;
         }
         tc_fence_after();
+        if (!C::SKIP0 || tp != t_skip) {
 #pragma unroll
-        for (int k4 = 0; k4 < 4; ++k4) {
-          const int kk = 4 * half + k4;
-          if (leader)
-            tc_mma_ts(tO, sbuf(tp) + kk * 8, vd + ((kk * 2048) >> 4), IDESC_O,
-                      (j > 0 || kk > 0) ? 1u : 0u);
+          for (int k4 = 0; k4 < 4; ++k4) {
+            const int kk = 4 * half + k4;
+            if (leader)
+              tc_mma_ts(tO, sbuf(tp) + kk * 8, vd + ((kk * 2048) >> 4), IDESC_O,
+                        (j > 0 || kk > 0) ? 1u : 0u);
+          }
         }
         __syncwarp();
       }
@@ -799,9 +813,9 @@ __device__ void role_mma_triple(const Sm100Ctx<D, F8> &x, const FwdParams &p) {
 // --------------------------------------------------------------------------
 // Softmax warpgroup t (128 threads, one query row each)
 // --------------------------------------------------------------------------
-template <int D, bool F8>
-__device__ void role_softmax(const Sm100Ctx<D, F8> &x, const FwdParams &p, int t) {
-  using C = Sm100Cfg<D, F8>;
+template <int D, bool F8, bool SK>
+__device__ void role_softmax(const Sm100Ctx<D, F8, SK> &x, const FwdParams &p, int t) {
+  using C = Sm100Cfg<D, F8, SK>;
   const int r = threadIdx.x & 127;
   const uint32_t lane_base = static_cast<uint32_t>((threadIdx.x >> 5) & 3) * 32u << 16;
   const uint32_t tS = x.tmem + lane_base + C::COL_S0 + 128 * t;
@@ -820,7 +834,7 @@ __device__ void role_softmax(const Sm100Ctx<D, F8> &x, const FwdParams &p, int t
     const int u = snake_unit(k, p.num_units);
     if (u == -2) break;
     if (u < 0) continue;
-    const Unit w = unit_at<D, F8>(p, u);
+    const Unit w = unit_at<D, F8, SK>(p, u);
     const int tile_row0 = w.row0 + t * C::BM;
     const int i = tile_row0 + r;  // this thread's query row
     const bool valid = i < w.q_rows;
@@ -1001,6 +1015,15 @@ __device__ void role_softmax(const Sm100Ctx<D, F8> &x, const FwdParams &p, int t
       l += a0 + a1;
     }
 
+    if (C::SKIP0 && nkv_t < w.nkv) {
+      // Q tile 0's skipped last key tile (three S buffers): the slot's S is
+      // committed without products; once it has, both P halves are released
+      // without any probabilities, which keeps the buffer's phases.
+      const int tt = 2 * (g + w.nkv - 1) + t;
+      if (!wait_all(C::BAR_S_FULL + tt % 3, static_cast<uint32_t>((tt / 3) & 1))) return;
+      mbar_arrive(x.bar(C::BAR_P_HALF + 2 * (tt % 3)));
+      mbar_arrive(x.bar(C::BAR_P_HALF + 2 * (tt % 3) + 1));
+    }
     // Epilogue: O = O~ / l in bf16, LSE = (m_ref + log2 l) * ln 2.
     if (!wait_all(C::BAR_O_FULL + t, static_cast<uint32_t>(qi & 1))) return;
     tc_fence_after();
@@ -1030,15 +1053,17 @@ __device__ void role_softmax(const Sm100Ctx<D, F8> &x, const FwdParams &p, int t
       p.lse[w.lse_base + i] =
           l > 0.f ? (m_lse + __log2f(l)) * 0.69314718055994530942f : -INFINITY;
     }
-    g += nkv_t;
+    // three S buffers: the sequence advances by the unit's tiles for both
+    // Q tiles (a skipped slot included)
+    g += C::SKIP0 ? w.nkv : nkv_t;
     ++qi;
   }
 }
 
-template <int D, bool F8>
+template <int D, bool F8, bool SK>
 __device__ __forceinline__ void fwd_kernel_body(const CUtensorMap *tm_q, const CUtensorMap *tm_k,
                                                 const CUtensorMap *tm_v, const FwdParams &p) {
-  using C = Sm100Cfg<D, F8>;
+  using C = Sm100Cfg<D, F8, SK>;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
@@ -1046,7 +1071,7 @@ __device__ __forceinline__ void fwd_kernel_body(const CUtensorMap *tm_q, const C
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
-  Sm100Ctx<D, F8> x;
+  Sm100Ctx<D, F8, SK> x;
   x.smem = base;
   x.abort_flag = reinterpret_cast<volatile int *>(smem + C::OFF_MISC + 4);
 
@@ -1089,18 +1114,18 @@ __device__ __forceinline__ void fwd_kernel_body(const CUtensorMap *tm_q, const C
   if (warp >= 8) {
     regs_decrease<C::REGS_CONTROL>();
     if (warp == 8) {
-      if (lane == 0) role_producer<D, F8>(x, p, tm_q, tm_k, tm_v);
+      if (lane == 0) role_producer<D, F8, SK>(x, p, tm_q, tm_k, tm_v);
     } else if (warp == 9) {
       if constexpr (C::TRIPLE)
-        role_mma_triple<D, F8>(x, p);
+        role_mma_triple<D, F8, SK>(x, p);
       else if constexpr (C::P_HI_SMEM)
-        role_mma_split<D, F8>(x, p);
+        role_mma_split<D, F8, SK>(x, p);
       else
-        role_mma<D, F8>(x, p);
+        role_mma<D, F8, SK>(x, p);
     }
   } else {
     regs_increase<C::REGS_SOFTMAX>();
-    role_softmax<D, F8>(x, p, warp >> 2);
+    role_softmax<D, F8, SK>(x, p, warp >> 2);
   }
   __syncwarp();
   tc_fence_before();
@@ -1111,12 +1136,12 @@ __device__ __forceinline__ void fwd_kernel_body(const CUtensorMap *tm_q, const C
   }
 }
 
-template <int D>
+template <int D, bool SK>
 __global__ void __launch_bounds__(Sm100Cfg<D>::THREADS, 1)
     fa_fwd_bf16_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
                              const __grid_constant__ CUtensorMap tm_k,
                              const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
-  fwd_kernel_body<D, false>(&tm_q, &tm_k, &tm_v, p);
+  fwd_kernel_body<D, false, SK>(&tm_q, &tm_k, &tm_v, p);
 }
 
 // FP8 E4M3 inputs (head dim 128); tm_v maps V^T.
@@ -1124,7 +1149,7 @@ __global__ void __launch_bounds__(Sm100Cfg<128, true>::THREADS, 1)
     fa_fwd_e4m3_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
                              const __grid_constant__ CUtensorMap tm_k,
                              const __grid_constant__ CUtensorMap tm_vt, const FwdParams p) {
-  fwd_kernel_body<128, true>(&tm_q, &tm_k, &tm_vt, p);
+  fwd_kernel_body<128, true, false>(&tm_q, &tm_k, &tm_vt, p);
 }
 
 }  // namespace fa
