@@ -750,11 +750,16 @@ def report_mufu(args, dev):
 
 
 def report_decode(args, dev):
-    """The split-KV decode path: HBM bandwidth against the measured copy rate."""
+    """The split-KV decode path: HBM bandwidth against the measured copy rate,
+    with 1 and with 4 new query rows per sequence (4 and 32 rows per kv head)."""
+    for w in (wl.DECODE, wl.DECODE_NQ4):
+        report_decode_one(args, dev, w)
+
+
+def report_decode_one(args, dev, w):
     import torch
     from exact_io_aware_92_b200 import attention
     peaks, src = load_peaks()
-    w = wl.DECODE
     inp = wl.draw_workload(w)
     q, k, v = (torch.from_numpy(x).view(torch.bfloat16).to(dev)
                for x in (inp.q_bits, inp.k_bits, inp.v_bits))

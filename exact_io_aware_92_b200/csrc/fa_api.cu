@@ -21,6 +21,7 @@
 #include "fa_bwd_sm100.cuh"
 #include "fa_decode.cuh"
 #include "fa_decode_tc.cuh"
+#include "fa_decode_rows.cuh"
 #include "fa_fwd_f32.cuh"
 #include "fa_fwd_sm100.cuh"
 
@@ -41,6 +42,7 @@ struct DeviceState {
   bool attr64 = false, attr64_causal = false, attr128 = false;
   bool dec_attr64 = false, dec_attr128 = false;
   bool dec_tc_attr[2][3] = {};  // [d = 64, 128][4, 8, 16 row slots]
+  bool dec_rows_attr[2] = {};    // [d = 64, 128]: 17 to 128 rows per kv head
   bool bwd_attr64 = false, bwd_attr128 = false;
   bool fp8_attr = false;
   // fa_fwd_hostio's copy streams and per-slice events, created on first use
@@ -165,13 +167,13 @@ int make_map_packed(CUtensorMap *m, const void *ptr, int total, int H, int d) {
   return r == CUDA_SUCCESS ? FA_OK : FA_ERR_CUDA;
 }
 
-// The query rows of a decode call, [rows, d] bf16: box = 64 columns x 16
-// rows, 128-byte swizzle; rows past the end read as zero.
-int make_map_qrows(CUtensorMap *m, const void *ptr, int rows, int d) {
+// The query rows of a decode call, [rows, d] bf16: box = 64 columns x
+// box_rows rows (16 or 128), 128-byte swizzle; rows past the end read as zero.
+int make_map_qrows(CUtensorMap *m, const void *ptr, int rows, int d, int box_rows = 16) {
   cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(rows), 1};
   cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2,
                            static_cast<cuuint64_t>(rows) * static_cast<cuuint64_t>(d) * 2};
-  cuuint32_t box[3] = {64, 16, 1};
+  cuuint32_t box[3] = {64, static_cast<cuuint32_t>(box_rows), 1};
   cuuint32_t estr[3] = {1, 1, 1};
   CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(ptr), dims,
                         strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
@@ -434,6 +436,7 @@ int launch_decode(DeviceState *ds, const void *q, const void *k, const void *v, 
   p.Nk = Nk;
   p.group = Hq / Hkv;
   p.splits = sp.splits;
+  p.part_rows = 0;
   p.keys_per_split = sp.keys_per_split;
   p.causal = causal ? 1 : 0;
   p.scale_log2 = scale * kLog2e;
@@ -448,17 +451,27 @@ int launch_decode(DeviceState *ds, const void *q, const void *k, const void *v, 
   return FA_OK;
 }
 
-// Decode on the tensor cores (up to 16 query rows per kv head): the call's
+// Decode on the tensor cores (up to 128 query rows per kv head): the call's
 // key tiles are shared evenly by `ctas` persistent CTAs, one per SM by
 // default, or num_splits per (batch, kv head) when given.  Each CTA leaves one
 // partial per (batch, kv head) its share touches, so there are at most
-// ctas + B * Hkv of them, 16 row slots each.
+// ctas + B * Hkv of them.  Up to 16 rows per kv head, fa_decode_tc.cuh (keys
+// on the tensor-memory lanes, 16 row slots per partial); from 17 to 128,
+// fa_decode_rows.cuh (rows on the lanes, the row count rounded up to 16 row
+// slots per partial).
 constexpr int kDecodeTcMaxRows = 16;
+constexpr int kDecodeRowsMax = 128;
 constexpr int kDecodeTcAutoCtasMax = 256;
 constexpr long long kDecodeTcCtasMax = 1024;
 
 bool decode_uses_tc(int Hq, int Hkv, int Nq) {
-  return static_cast<long long>(Hq / Hkv) * Nq <= kDecodeTcMaxRows;
+  return static_cast<long long>(Hq / Hkv) * Nq <= kDecodeRowsMax;
+}
+
+// Row slots per partial of the tensor-core decode.
+int decode_tc_part_rows(int Hq, int Hkv, int Nq) {
+  const int rows = (Hq / Hkv) * Nq;
+  return rows <= kDecodeTcMaxRows ? kDecodeTcMaxRows : (rows + 15) / 16 * 16;
 }
 
 int decode_tc_ctas(int B, int Hkv, int num_splits, int num_sms) {
@@ -468,12 +481,18 @@ int decode_tc_ctas(int B, int Hkv, int num_splits, int num_sms) {
   return std::max(1, std::min(num_sms, kDecodeTcAutoCtasMax));
 }
 
-size_t decode_tc_workspace_bytes(int B, int Hkv, int d, int ctas) {
+size_t decode_tc_workspace_bytes(int B, int Hkv, int d, int ctas, int part_rows) {
   const size_t pieces = static_cast<size_t>(ctas) + static_cast<size_t>(B) * Hkv;
-  const size_t o_bytes = pieces * kDecodeTcMaxRows * d * sizeof(float);
-  const size_t ml_bytes = pieces * kDecodeTcMaxRows * 2 * sizeof(float);
+  const size_t o_bytes = pieces * part_rows * d * sizeof(float);
+  const size_t ml_bytes = pieces * part_rows * 2 * sizeof(float);
   return ((o_bytes + 255) / 256) * 256 + ml_bytes;
 }
+
+// The merge of a tensor-core decode call, as a programmatic dependent launch:
+// it may start while the split kernel finishes and waits for it in the kernel
+// before reading.
+template <int D>
+int launch_decode_tc_merge(const fa::DecodeParams &p, cudaStream_t stream);
 
 template <int D, int NR>
 int launch_decode_tc_rows(DeviceState *ds, const CUtensorMap &tq, const CUtensorMap &tk,
@@ -492,6 +511,31 @@ int launch_decode_tc_rows(DeviceState *ds, const CUtensorMap &tq, const CUtensor
   }
   kernel<<<p.ctas, C::THREADS, C::SMEM_ALLOC, stream>>>(tq, tk, tv, p);
   if (cudaGetLastError() != cudaSuccess) return FA_ERR_LAUNCH;
+  return launch_decode_tc_merge<D>(p, stream);
+}
+
+// 17 to 128 query rows per kv head (fa_decode_rows.cuh).
+template <int D>
+int launch_decode_rows(DeviceState *ds, const CUtensorMap &tq, const CUtensorMap &tk,
+                       const CUtensorMap &tv, const fa::DecodeParams &p, cudaStream_t stream) {
+  using C = fa::DecodeRowsCfg<D>;
+  auto kernel = fa::fa_decode_rows_kernel<D>;
+  bool &attr = ds->dec_rows_attr[D == 128];
+  if (!attr) {
+    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             C::SMEM_ALLOC) != cudaSuccess) {
+      cudaGetLastError();
+      return FA_ERR_LAUNCH;
+    }
+    attr = true;
+  }
+  kernel<<<p.ctas, C::THREADS, C::SMEM_ALLOC, stream>>>(tq, tk, tv, p);
+  if (cudaGetLastError() != cudaSuccess) return FA_ERR_LAUNCH;
+  return launch_decode_tc_merge<D>(p, stream);
+}
+
+template <int D>
+int launch_decode_tc_merge(const fa::DecodeParams &p, cudaStream_t stream) {
   // The merge is a programmatic dependent launch: it may start while the
   // split kernel finishes and waits for it in the kernel before reading.
   const long long rows = static_cast<long long>(p.B) * p.Hq * p.Nq;
@@ -517,8 +561,10 @@ int launch_decode_tc(DeviceState *ds, const void *q, const void *k, const void *
                      float *lse, int B, int Hq, int Hkv, int Nq, int Nk, float scale, int causal,
                      const int *seqlens, int ctas, void *workspace, cudaStream_t stream,
                      int *status) {
+  const int part_rows = decode_tc_part_rows(Hq, Hkv, Nq);
+  const bool wide = part_rows > kDecodeTcMaxRows;  // rows on the tensor-memory lanes
   CUtensorMap tq, tk, tv;
-  if (make_map_qrows(&tq, q, B * Hq * Nq, D) != FA_OK ||
+  if (make_map_qrows(&tq, q, B * Hq * Nq, D, wide ? 128 : 16) != FA_OK ||
       make_map(&tk, k, B * Hkv, Nk, D) != FA_OK || make_map(&tv, v, B * Hkv, Nk, D) != FA_OK)
     return FA_ERR_CUDA;
   const size_t pieces = static_cast<size_t>(ctas) + static_cast<size_t>(B) * Hkv;
@@ -532,7 +578,8 @@ int launch_decode_tc(DeviceState *ds, const void *q, const void *k, const void *
   p.part_o = static_cast<float *>(workspace);
   p.part_ml = reinterpret_cast<float *>(
       static_cast<char *>(workspace) +
-      ((pieces * kDecodeTcMaxRows * D * sizeof(float) + 255) / 256) * 256);
+      ((pieces * part_rows * D * sizeof(float) + 255) / 256) * 256);
+  p.part_rows = part_rows;
   p.status = status;
   p.B = B;
   p.Hq = Hq;
@@ -547,6 +594,7 @@ int launch_decode_tc(DeviceState *ds, const void *q, const void *k, const void *
   p.scale_log2 = scale * kLog2e;
   p.wait_limit_ns = kWaitLimitNs;
   const int rows = p.group * Nq;
+  if (wide) return launch_decode_rows<D>(ds, tq, tk, tv, p, stream);
   if (rows <= 4) return launch_decode_tc_rows<D, 4>(ds, tq, tk, tv, p, stream);
   if (rows <= 8) return launch_decode_tc_rows<D, 8>(ds, tq, tk, tv, p, stream);
   return launch_decode_tc_rows<D, 16>(ds, tq, tk, tv, p, stream);
@@ -989,7 +1037,8 @@ size_t fa_decode_workspace_size(int B, int Hq, int Hkv, int Nq, int Nk, int d, i
     return 0;
   if (decode_uses_tc(Hq, Hkv, Nq))
     return decode_tc_workspace_bytes(B, Hkv, d,
-                                     decode_tc_ctas(B, Hkv, num_splits, kDecodeTcAutoCtasMax));
+                                     decode_tc_ctas(B, Hkv, num_splits, kDecodeTcAutoCtasMax),
+                                     decode_tc_part_rows(Hq, Hkv, Nq));
   const int groups = ((Hq / Hkv) * Nq + 3) / 4;
   const DecodeSplit sp = decode_split(B, Hkv, groups, Nk, d, num_splits);
   return decode_workspace_bytes(B, Hq, Nq, d, sp.splits);
@@ -1125,7 +1174,8 @@ extern "C" int fa_fwd_decode_noalloc(const void *q, const void *k, const void *v
   // the size fa_decode_workspace_size reports, so a shape is accepted or
   // rejected whatever the device
   const size_t need = tc ? decode_tc_workspace_bytes(
-                               B, Hkv, d, decode_tc_ctas(B, Hkv, num_splits, kDecodeTcAutoCtasMax))
+                               B, Hkv, d, decode_tc_ctas(B, Hkv, num_splits, kDecodeTcAutoCtasMax),
+                               decode_tc_part_rows(Hq, Hkv, Nq))
                          : decode_workspace_bytes(B, Hq, Nq, d, sp.splits);
   if (need > kNoAllocScratchBytes) return FA_ERR_WORKSPACE;
   DeviceState *ds = nullptr;

@@ -36,6 +36,7 @@ struct DecodeParams {
   int B, Hq, Hkv, Nq, Nk, group;
   int splits, keys_per_split;
   int ctas;                   // tensor-core path: CTAs sharing the key tiles
+  int part_rows;              // tensor-core path: row slots per workspace slot
   int causal;
   float scale_log2;
   unsigned long long wait_limit_ns;

@@ -711,10 +711,12 @@ __global__ void __launch_bounds__(DecodeTcCfg<D>::THREADS, 1)
 }
 
 // Merge of the pieces, one warp per query row: the pieces of (b, g) are
-// those of the CTAs whose shares meet its tiles.
+// those of the CTAs whose shares meet its tiles.  Serves both tensor-core
+// split kernels (this file's and fa_decode_rows.cuh's): their workspace slots
+// hold p.part_rows row slots each.
 template <int D>
 __global__ void __launch_bounds__(128) fa_decode_tc_combine_kernel(const DecodeParams p) {
-  constexpr int QROWS = DecodeTcCfg<D>::QROWS;
+  const int QROWS = p.part_rows;  // row slots per workspace slot
   constexpr int PER = D / 32;
   const int lane = threadIdx.x & 31;
   const int R = p.group * p.Nq;

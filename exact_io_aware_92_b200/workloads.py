@@ -66,13 +66,17 @@ LONG = Workload("long_causal_b1_h16_n32768_d128", 1, 16, 16, 32768, 128, True, s
 # sequence, the Llama-style GQA heads, caches of 16K-32K tokens.
 DECODE = Workload("llama_gqa_decode_b8_hq32_hkv8_nq1_nk32768_d128", 8, 32, 8, 32768, 128, True,
                   seed=6, seqlen_range=(16384, 32768), nq=1)
+# The same caches with 4 new query rows per sequence (speculative or chunked
+# decode): 8 query heads per kv head x 4 rows = 32 rows per kv head.
+DECODE_NQ4 = Workload("llama_gqa_decode_b8_hq32_hkv8_nq4_nk32768_d128", 8, 32, 8, 32768, 128,
+                      True, seed=7, seqlen_range=(16384, 32768), nq=4)
 
 ALL = (TINY, GPT2, BERT, LLAMA_GQA, LONG)
 # The GQA workload with FP8 E4M3 inputs (the same draws, quantised).
 LLAMA_GQA_FP8 = Workload("llama_gqa_causal_b2_hq32_hkv8_n8192_d128_e4m3", 2, 32, 8, 8192, 128,
                          True, seed=4, k_scale=2.0, sample_rows=32)
 
-BY_NAME = {w.name: w for w in ALL + (DECODE, LLAMA_GQA_FP8)}
+BY_NAME = {w.name: w for w in ALL + (DECODE, DECODE_NQ4, LLAMA_GQA_FP8)}
 
 
 def round_to_bf16_bits(x: np.ndarray) -> np.ndarray:

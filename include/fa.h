@@ -239,11 +239,13 @@ FA_API int fa_fwd_varlen(const void *q, const void *k, const void *v, void *o, f
  *         valid cached keys of sequence b (keys past it are ignored).
  *  causal: 0/1; query i is position len_b - Nq + i of its sequence, so it sees
  *         keys j <= len_b - Nq + i (with Nq = 1: every valid key).
- *  Two kernels serve the call, chosen by G * Nq, the query rows per kv head
- *  (G = Hq / Hkv):
- *   - G * Nq <= 16: tensor cores.  The call's 128-key tiles of valid keys
- *     are divided evenly among persistent CTAs, whatever the lengths.
- *   - G * Nq > 16: CUDA cores, per key range of each (batch, kv head).
+ *  Three kernels serve the call, chosen by G * Nq, the query rows per kv
+ *  head (G = Hq / Hkv):
+ *   - G * Nq <= 16: tensor cores, keys on the tensor-memory lanes.
+ *   - 16 < G * Nq <= 128: tensor cores, query rows on the lanes.
+ *     In both, the call's 128-key tiles of valid keys are divided evenly
+ *     among persistent CTAs, whatever the lengths.
+ *   - G * Nq > 128: CUDA cores, per key range of each (batch, kv head).
  *  num_splits: 0 for the automatic choice, or 1..128.
  *   - Tensor-core kernel: 0 gives one CTA per SM; n gives
  *     min(n * B * Hkv, 1024) CTAs, so each (batch, kv head) is processed by

@@ -115,25 +115,30 @@ def test_decode_workspace_size_and_errors(lib):
 
 
 def test_decode_workspace_sizes_of_both_kernels(lib):
-    """Up to 16 query rows per kv head (G * Nq) take the tensor-core kernel:
-    partials for at most ctas + B * Hkv pieces, 16 row slots of d + 2 floats,
-    with ctas = 256 by default (one CTA per SM, at most 256) or
-    min(num_splits * B * Hkv, 1024).  Beyond 16 rows the CUDA-core kernel's
-    per-key-range partials apply, so the size jumps at 17 rows."""
-    def tc_bytes(B, Hkv, d, ctas):
+    """Up to 128 query rows per kv head (G * Nq) take the tensor cores:
+    partials for at most ctas + B * Hkv pieces, with ctas = 256 by default
+    (one CTA per SM, at most 256) or min(num_splits * B * Hkv, 1024).  Each
+    partial holds row slots of d + 2 floats: 16 up to 16 rows (keys on the
+    tensor-memory lanes), the row count rounded up to 16 from 17 to 128 (rows
+    on the lanes).  Beyond 128 rows the CUDA-core kernel's per-key-range
+    partials apply."""
+    def tc_bytes(B, Hkv, d, ctas, slots=16):
         pieces = ctas + B * Hkv
-        o_bytes = pieces * 16 * d * 4
-        return (o_bytes + 255) // 256 * 256 + pieces * 16 * 2 * 4
+        o_bytes = pieces * slots * d * 4
+        return (o_bytes + 255) // 256 * 256 + pieces * slots * 2 * 4
 
     assert lib.fa_decode_workspace_size(8, 32, 8, 1, 32768, 128, 0) == tc_bytes(8, 8, 128, 256)
     assert lib.fa_decode_workspace_size(8, 32, 8, 4, 32768, 64, 0) == tc_bytes(8, 8, 64, 256)
+    assert lib.fa_decode_workspace_size(8, 32, 8, 8, 32768, 64, 0) == tc_bytes(8, 8, 64, 256, 32)
     assert lib.fa_decode_workspace_size(3, 8, 2, 1, 2000, 128, 7) == tc_bytes(3, 2, 128, 42)
     assert lib.fa_decode_workspace_size(64, 64, 16, 1, 4096, 128, 2) == tc_bytes(64, 16, 128, 1024)
-    # 4 query heads per kv head x 4 rows = 16: tensor cores; x 5 = 20: CUDA cores
-    tc16 = lib.fa_decode_workspace_size(2, 8, 2, 4, 1000, 128, 3)
-    cc20 = lib.fa_decode_workspace_size(2, 8, 2, 5, 1000, 128, 3)
-    assert tc16 == tc_bytes(2, 2, 128, 12)
-    assert cc20 != tc_bytes(2, 2, 128, 12) and cc20 > 0
+    # 4 query heads per kv head: x 4 rows = 16 slots; x 5 = 20 rows -> 32 slots
+    assert lib.fa_decode_workspace_size(2, 8, 2, 4, 1000, 128, 3) == tc_bytes(2, 2, 128, 12)
+    assert lib.fa_decode_workspace_size(2, 8, 2, 5, 1000, 128, 3) == tc_bytes(2, 2, 128, 12, 32)
+    # 8 x 16 = 128 rows: the last tensor-core shape; 8 x 17 = 136: CUDA cores
+    assert lib.fa_decode_workspace_size(2, 8, 1, 16, 1000, 128, 3) == tc_bytes(2, 1, 128, 6, 128)
+    cc = lib.fa_decode_workspace_size(2, 8, 1, 17, 1000, 128, 3)
+    assert cc > 0 and cc != tc_bytes(2, 1, 128, 6, 144)
 
 
 def test_without_a_b200_valid_calls_report_arch():

@@ -38,8 +38,9 @@ def test_single_query_lengths(Nk, d):
     compare(o, lse, o_r, l_r, o_tol=O_TOL_BF16, lse_tol=LSE_TOL_BF16, what=f"Nk{Nk} d{d}")
 
 
-# Up to 16 query rows per kv head take the tensor-core kernel (4, 8 or 16
-# row slots); more take the CUDA-core kernel: (4, 5) and (8, 3) give 20 and 24.
+# Up to 16 query rows per kv head take the tensor-core kernel with keys on the
+# tensor-memory lanes (4, 8 or 16 row slots); 17 to 128 the one with rows on
+# the lanes: (4, 5) and (8, 3) give 20 and 24.
 @pytest.mark.parametrize("splits", [1, 3, 7, 0])
 @pytest.mark.parametrize("group,nq", [(1, 1), (4, 1), (8, 1), (4, 3), (1, 5), (4, 4), (4, 5),
                                       (8, 3)])
@@ -112,3 +113,31 @@ def test_many_short_caches_per_cta(splits):
     o_r, l_r = ref_decode(inp, causal=True, scale=0.088)
     compare(o, lse, o_r, l_r, o_tol=O_TOL_BF16, lse_tol=LSE_TOL_BF16,
             what=f"B{B} short caches splits{splits}")
+
+
+# Rows on the tensor-memory lanes (17 to 128 query rows per kv head): 24, 32,
+# 64 and 128 rows, with ragged and empty caches, both head dims, forced
+# splits (several pieces per CTA, several CTAs per piece) and the automatic
+# split; beyond 128 rows (8 x 17 = 136) the CUDA-core kernel.
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("group,nq", [(8, 3), (8, 4), (4, 16), (16, 8), (8, 17)])
+@pytest.mark.parametrize("splits", [0, 3])
+def test_rows_on_lanes(group, nq, splits, d):
+    Hkv = 2
+    inp = wl.draw(3, group * Hkv, Hkv, 1500, d, seed=1000 + group * 10 + nq + d, nq=nq)
+    inp.seqlens = np.array([1500, 0, 333], dtype=np.int32)
+    for causal in (False, True):
+        o, lse = run_decode(inp, causal=causal, scale=1 / np.sqrt(d), num_splits=splits)
+        o_r, l_r = ref_decode(inp, causal=causal, scale=1 / np.sqrt(d))
+        compare(o, lse, o_r, l_r, o_tol=O_TOL_BF16, lse_tol=LSE_TOL_BF16,
+                what=f"d{d} G{group} nq{nq} splits{splits} causal{causal}")
+
+
+def test_rows_on_lanes_gqa_decode_workload_shape():
+    # the GQA decode workload with 4 query rows per sequence (speculative or
+    # chunked decode): 8 query heads per kv head x 4 = 32 rows; every row
+    w = wl.DECODE_NQ4
+    inp = wl.draw_workload(w)
+    o, lse = run_decode(inp, causal=w.causal, scale=w.scale)
+    o_r, l_r = ref_decode(inp, causal=w.causal, scale=w.scale)
+    compare(o, lse, o_r, l_r, o_tol=O_TOL_BF16, lse_tol=LSE_TOL_BF16, what=w.name)
