@@ -16,26 +16,26 @@
 //   warps 4-7  softmax warpgroup for Q tile 1
 //   warp  8    TMA producer: Q tiles per unit, then K_j, V_j into a ring of stages
 //   warp  9    MMA issuer: S_t = Q_t K_j^T and O_t += P_t V_j with tcgen05.mma
-//              (role_mma_split at d = 128, role_mma_triple at d = 64,
-//              role_mma for FP8)
+//              (role_mma_split at d = 128, role_mma_triple at d = 64)
 //   warps 10-11 idle (they complete the third warpgroup, whose registers go
 //              to the softmax warpgroups)
 // Tensor memory (512 columns, fp32): S0 [0,128) S1 [128,256) O0 [256,256+d)
-// O1 [384,384+d).  P_t (bf16, packed two per column) is published in two
-// halves of 64 keys so the PV product starts on the first half while the
-// second is computed.  The first half overwrites the first 32 columns of S_t
-// and feeds the PV product straight from tensor memory.  At d = 128 the
+// O1 [384,384+d).  P_t (bf16, two per column; FP8: four E4M3 codes per
+// column) is published in two halves of 64 keys so the PV product starts on
+// the first half while the second is computed.  The first half overwrites the
+// first columns of S_t and feeds the PV product straight from tensor memory.  At d = 128 the
 // second half goes to a 16 KB shared-memory tile per Q tile (K-major,
 // 128-byte swizzled), so S_t of the next key tile is issued right after the
 // first half's PV product, while the softmax still computes the second half;
-// at d = 64 (three S buffers) and for FP8 inputs it overwrites columns 32-63.
+// at d = 64 (three S buffers) it overwrites columns 32-63.
 // In a causal unit, Q tile 0 skips the last key tile when it lies wholly above
 // its rows (Q tile 1 still needs it).
 //
 // The same body serves FP8 E4M3 inputs (F8 = true, head dim 128): 8-bit
 // tiles, kind::f8f6f4 products, V given transposed so both products read
-// K-major operands, and P stored as E4M3 with a factor 2^2 and a rescale
-// threshold of 6 (log2 units) so it never saturates.
+// K-major operands, and P stored as E4M3 (its second half in the first 64
+// bytes of each shared-memory row) with a factor 2^2 and a rescale threshold
+// of 6 (log2 units) so it never saturates.
 //
 // Differences from the pages' statement of the recurrence, all algebraically
 // equivalent: O is kept unnormalised (O~ = l * O) and divided by l once at the
@@ -113,13 +113,14 @@ struct Sm100Cfg {
   static constexpr int STAGES = (TILE_BYTES == 32768) ? 4 : 8;
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_KV = OFF_Q + 2 * TILE_BYTES;
-  // bf16, d = 128: the upper 64 keys of P go to shared memory (K-major,
-  // 128-byte swizzled: 128 rows of 128 bytes, like a Q tile of 64 columns)
-  // instead of tensor memory, so the next S product may overwrite S_t as soon
-  // as the PV product has read the lower half.  (At d = 64 the three S
+  // d = 128: the upper 64 keys of P go to shared memory (K-major, 128-byte
+  // swizzled: 128 rows of 128 bytes, like a Q tile of 64 bf16 columns; E4M3
+  // codes fill the first 64 bytes of each row) instead of tensor memory, so
+  // the next S product may overwrite S_t as soon as the PV product has read
+  // the lower half.  (At d = 64 the three S
   // buffers already decouple S from P, and the extra shared-memory stores
   // only lengthen the softmax, which bounds that head dimension.)
-  static constexpr bool P_HI_SMEM = !F8 && D == 128;
+  static constexpr bool P_HI_SMEM = D == 128;
   static constexpr int P_HI_BYTES = 128 * 128;
   static constexpr int OFF_PHI = OFF_KV + STAGES * TILE_BYTES;  // [2 Q tiles]
   static constexpr int OFF_BAR = OFF_PHI + (P_HI_SMEM ? 2 * P_HI_BYTES : 0);
@@ -344,29 +345,32 @@ __device__ void role_producer(const Sm100Ctx<D, F8, SK> &x, const FwdParams &p, 
 }
 
 // --------------------------------------------------------------------------
-// MMA issuer (one warp: every lane runs the loop and the waits, so the
-// descriptor arithmetic stays warp-uniform; one elected lane issues the
-// tcgen05 instructions and their commits)
+// MMA issuer for two S buffers with P's upper half in shared memory
+// (D = 128, bf16 and FP8; every lane runs the loop and the waits, so the
+// descriptor arithmetic stays warp-uniform, and one elected lane issues the
+// tcgen05 instructions and their commits).  Per key tile j and Q tile t: PV_t(j-1) over the lower 64 keys
+// (P from tensor memory), then S_t(j) into the same columns, then PV_t(j-1)
+// over the upper 64 keys (P from shared memory).  S_t(j) thus waits only for
+// the first half of the previous tile's probabilities.
 // --------------------------------------------------------------------------
 template <int D, bool F8, bool SK>
-__device__ void role_mma(const Sm100Ctx<D, F8, SK> &x, const FwdParams &p) {
+__device__ void role_mma_split(const Sm100Ctx<D, F8, SK> &x, const FwdParams &p) {
   using C = Sm100Cfg<D, F8, SK>;
-  // S: Q and K both K-major.  O: P from TMEM; V MN-major (bf16) or V^T
-  // K-major (FP8).
+  static_assert(C::P_HI_SMEM && !C::TRIPLE, "two S buffers, P's upper half in shared memory");
+  // S: Q and K both K-major.  O: P K-major (tensor memory or shared memory);
+  // V MN-major (bf16) or V^T K-major (FP8).
   constexpr uint32_t IDESC_S = F8 ? idesc_e4m3_f32(128, C::BN) : idesc_bf16_f32(128, C::BN, 0, 0);
   constexpr uint32_t IDESC_O = F8 ? idesc_e4m3_f32(128, D) : idesc_bf16_f32(128, D, 0, 1);
   const bool leader = elect_one();
   const uint32_t tS[2] = {x.tmem + C::COL_S0, x.tmem + C::COL_S0 + 128};
   const uint32_t tO[2] = {x.tmem + C::COL_O0, x.tmem + C::COL_O0 + C::O_STRIDE};
-
-  // Descriptors are linear in the start address (16-byte units in the low
-  // bits), so they are built once and offset per operand.
   const uint64_t desc_q[2] = {smem_desc_sw128(x.q_tile(0), 16, 1024),
                               smem_desc_sw128(x.q_tile(1), 16, 1024)};
+  const uint64_t desc_p[2] = {smem_desc_sw128(x.p_hi(0), 16, 1024),
+                              smem_desc_sw128(x.p_hi(1), 16, 1024)};
   const uint64_t desc_kv_k = smem_desc_sw128(x.kv_tile(0), 16, 1024);
   const uint64_t desc_kv_v = F8 ? smem_desc_sw128(x.kv_tile(0), 16, 1024)
                                 : smem_desc_sw128(x.kv_tile(0), C::BOX_BYTES, 1024);
-
   auto wait = [&](int bar, uint32_t parity) {
     const bool ok = mbar_wait_bounded(x.bar(bar), parity, x.abort_flag, p.status,
                                       p.wait_limit_ns, kErrTimeout);
@@ -378,8 +382,8 @@ __device__ void role_mma(const Sm100Ctx<D, F8, SK> &x, const FwdParams &p) {
   };
   // S_t = Q_t K^T: K = d in steps of 32 bytes (16 bf16 or 32 FP8 values)
   // inside a 128-byte swizzled row; every 4 steps move to the next box.
-  auto issue_s = [&](int t, int k_slot_idx) {
-    const uint64_t kd = desc_kv_k + ((k_slot_idx * C::TILE_BYTES) >> 4);
+  auto issue_s = [&](int t, int ks) {
+    const uint64_t kd = desc_kv_k + ((ks * C::TILE_BYTES) >> 4);
 #pragma unroll
     for (int kk = 0; kk < C::KSTEPS; ++kk) {
       const uint32_t off = ((kk / 4) * C::BOX_BYTES + (kk % 4) * 32) >> 4;
@@ -392,199 +396,49 @@ __device__ void role_mma(const Sm100Ctx<D, F8, SK> &x, const FwdParams &p) {
     }
     __syncwarp();
   };
-  // O_t += P_t V for one half of the keys (64): K in steps of 16; P_t steps
-  // 8 columns (16 bf16) in TMEM; V steps 16 key rows = 2048 bytes; its two
-  // 64-column boxes are BOX_BYTES apart (leading byte offset), 8-row groups
-  // 1024 bytes apart.
-  // FP8: K in steps of 32 keys; P_t steps 8 columns (32 codes); V^T steps 32
-  // bytes along its 128-byte rows of keys.
-  auto issue_pv_half = [&](int t, int v_slot_idx, int half, bool accumulate) {
-    const uint64_t vd = desc_kv_v + ((v_slot_idx * C::TILE_BYTES) >> 4);
-    if constexpr (F8) {
-#pragma unroll
-      for (int k2 = 0; k2 < 2; ++k2) {
-        const int kk = 2 * half + k2;
-        if (leader)
-          tc_mma_ts_f8(tO[t], tS[t] + kk * 8, vd + ((kk * 32) >> 4), IDESC_O,
-                       (accumulate || kk > 0) ? 1u : 0u);
-      }
-    } else {
-#pragma unroll
-      for (int k4 = 0; k4 < 4; ++k4) {
-        const int kk = 4 * half + k4;
-        if (leader)
-          tc_mma_ts(tO[t], tS[t] + kk * 8, vd + ((kk * 2048) >> 4), IDESC_O,
-                    (accumulate || kk > 0) ? 1u : 0u);
-      }
-    }
-    __syncwarp();
-  };
-  // The PV product of tile t starts on the first 64 keys as soon as their
-  // probabilities are in tensor memory, and takes the second 64 when the
-  // softmax publishes them.
-  auto pv = [&](int t, int v_slot_idx, uint32_t parity, bool accumulate) {
-    if (!wait(C::BAR_P_HALF + 2 * t, parity)) return false;
-    tc_fence_after();
-    issue_pv_half(t, v_slot_idx, 0, accumulate);
-    if (!wait(C::BAR_P_HALF + 2 * t + 1, parity)) return false;
-    tc_fence_after();
-    issue_pv_half(t, v_slot_idx, 1, accumulate);
-    return true;
-  };
-
-  int g = 0;             // K/V tiles consumed by this CTA so far (ring position)
-  int gs[2] = {0, 0};    // key tiles each Q tile has processed (its S/P phases)
-  int qi = 0;            // units with keys processed so far
-  bool ok = true;
-  for (int k = 0; ok; ++k) {
-    const int u = snake_unit(k, p.num_units);
-    if (u == -2) break;
-    if (u < 0) continue;
-    const Unit w = unit_at<D, F8, SK>(p, u);
-    const int n1 = w.nkv, n0 = w.nkv0;  // n0 is n1 or n1 - 1
-    if (n1 == 0) continue;
-    const uint32_t qpar = static_cast<uint32_t>(qi & 1);
-    if (!wait(C::BAR_Q_FULL + 0, qpar) || !wait(C::BAR_Q_FULL + 1, qpar) ||
-        !wait(C::BAR_KV_FULL + ring_slot<D, F8, SK>(2 * g), ring_parity<D, F8, SK>(2 * g))) {
-      ok = false;
-      break;
-    }
-    tc_fence_after();
-    // Tile 0: S for both Q tiles.
-    issue_s(0, ring_slot<D, F8, SK>(2 * g));
-    commit(C::BAR_S_FULL + 0);
-    if (n0 == 1) commit(C::BAR_Q_EMPTY + 0);
-    issue_s(1, ring_slot<D, F8, SK>(2 * g));
-    commit(C::BAR_S_FULL + 1);
-    commit(C::BAR_KV_EMPTY + ring_slot<D, F8, SK>(2 * g));
-    if (n1 == 1) commit(C::BAR_Q_EMPTY + 1);
-    // Steady state: PV of tile j-1, then S of tile j into the same columns
-    // (the tensor pipe runs them in order, so P is read before S lands).
-    // Q tile 0 stops after its n0 tiles.
-    for (int j = 1; j < n1; ++j) {
-      const int gp = g + j - 1, gc = g + j;
-      const int vs = ring_slot<D, F8, SK>(2 * gp + 1), ks = ring_slot<D, F8, SK>(2 * gc);
-      if (!wait(C::BAR_KV_FULL + vs, ring_parity<D, F8, SK>(2 * gp + 1)) ||
-          !pv(0, vs, static_cast<uint32_t>((gs[0] + j - 1) & 1), j - 1 > 0) ||
-          !wait(C::BAR_KV_FULL + ks, ring_parity<D, F8, SK>(2 * gc))) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
-      if (j < n0) {
-        issue_s(0, ks);
-        commit(C::BAR_S_FULL + 0);
-        if (j == n0 - 1) commit(C::BAR_Q_EMPTY + 0);
-      } else {
-        commit(C::BAR_O_FULL + 0);  // Q tile 0's last PV was issued just above
-      }
-      if (!pv(1, vs, static_cast<uint32_t>((gs[1] + j - 1) & 1), j - 1 > 0)) {
-        ok = false;
-        break;
-      }
-      commit(C::BAR_KV_EMPTY + vs);
-      issue_s(1, ks);
-      commit(C::BAR_S_FULL + 1);
-      commit(C::BAR_KV_EMPTY + ks);
-      if (j == n1 - 1) commit(C::BAR_Q_EMPTY + 1);
-    }
-    if (!ok) break;
-    // Last tile's PV products, then the unit's output is complete.
-    const int gl = g + n1 - 1;
-    const int vs = ring_slot<D, F8, SK>(2 * gl + 1);
-    if (!wait(C::BAR_KV_FULL + vs, ring_parity<D, F8, SK>(2 * gl + 1))) {
-      ok = false;
-      break;
-    }
-    if (n0 == n1) {
-      if (!pv(0, vs, static_cast<uint32_t>((gs[0] + n1 - 1) & 1), n1 > 1)) {
-        ok = false;
-        break;
-      }
-      commit(C::BAR_O_FULL + 0);
-    }
-    if (!pv(1, vs, static_cast<uint32_t>((gs[1] + n1 - 1) & 1), n1 > 1)) {
-      ok = false;
-      break;
-    }
-    commit(C::BAR_O_FULL + 1);
-    commit(C::BAR_KV_EMPTY + vs);
-    g += n1;
-    gs[0] += n0;
-    gs[1] += n1;
-    ++qi;
-  }
-  // Every MMA issued above must finish before tensor memory is released.
-  commit(C::BAR_MMA_DONE);
-  volatile int never = 0;
-  mbar_wait_bounded(x.bar(C::BAR_MMA_DONE), 0, &never, p.status, p.wait_limit_ns, kErrTimeout);
-}
-
-// --------------------------------------------------------------------------
-// MMA issuer for two S buffers with P's upper half in shared memory (bf16,
-// D = 128).  Per key tile j and Q tile t: PV_t(j-1) over the lower 64 keys
-// (P from tensor memory), then S_t(j) into the same columns, then PV_t(j-1)
-// over the upper 64 keys (P from shared memory).  S_t(j) thus waits only for
-// the first half of the previous tile's probabilities.
-// --------------------------------------------------------------------------
-template <int D, bool F8, bool SK>
-__device__ void role_mma_split(const Sm100Ctx<D, F8, SK> &x, const FwdParams &p) {
-  using C = Sm100Cfg<D, F8, SK>;
-  static_assert(C::P_HI_SMEM && !C::TRIPLE, "two S buffers, P's upper half in shared memory");
-  constexpr uint32_t IDESC_S = idesc_bf16_f32(128, C::BN, 0, 0);  // Q, K both K-major
-  constexpr uint32_t IDESC_O = idesc_bf16_f32(128, D, 0, 1);      // P K-major, V MN-major
-  const bool leader = elect_one();
-  const uint32_t tS[2] = {x.tmem + C::COL_S0, x.tmem + C::COL_S0 + 128};
-  const uint32_t tO[2] = {x.tmem + C::COL_O0, x.tmem + C::COL_O0 + C::O_STRIDE};
-  const uint64_t desc_q[2] = {smem_desc_sw128(x.q_tile(0), 16, 1024),
-                              smem_desc_sw128(x.q_tile(1), 16, 1024)};
-  const uint64_t desc_p[2] = {smem_desc_sw128(x.p_hi(0), 16, 1024),
-                              smem_desc_sw128(x.p_hi(1), 16, 1024)};
-  const uint64_t desc_kv_k = smem_desc_sw128(x.kv_tile(0), 16, 1024);
-  const uint64_t desc_kv_v = smem_desc_sw128(x.kv_tile(0), C::BOX_BYTES, 1024);
-  auto wait = [&](int bar, uint32_t parity) {
-    const bool ok = mbar_wait_bounded(x.bar(bar), parity, x.abort_flag, p.status,
-                                      p.wait_limit_ns, kErrTimeout);
-    return __all_sync(0xffffffffu, ok);
-  };
-  auto commit = [&](int bar) {
-    if (leader) tc_commit(x.bar(bar));
-    __syncwarp();
-  };
-  auto issue_s = [&](int t, int ks) {
-    const uint64_t kd = desc_kv_k + ((ks * C::TILE_BYTES) >> 4);
-#pragma unroll
-    for (int kk = 0; kk < C::KSTEPS; ++kk) {
-      const uint32_t off = ((kk / 4) * C::BOX_BYTES + (kk % 4) * 32) >> 4;
-      if (leader) tc_mma_ss(tS[t], desc_q[t] + off, kd + off, IDESC_S, kk > 0 ? 1u : 0u);
-    }
-    __syncwarp();
-  };
-  // O_t += P_t V over keys 0-63: P from tensor memory (8 columns per 16
-  // keys), V steps 16 key rows = 2048 bytes.
+  // O_t += P_t V over keys 0-63, P from tensor memory.  bf16: 16 keys per
+  // step, 8 columns of P, V steps 16 key rows = 2048 bytes.  FP8: 32 keys per
+  // step, 8 columns of P (four codes each), V^T steps 32 bytes of its rows.
   auto pv_lo = [&](int t, int vs, uint32_t parity, bool accumulate) {
     if (!wait(C::BAR_P_HALF + 2 * t, parity)) return false;
     tc_fence_after();
     const uint64_t vd = desc_kv_v + ((vs * C::TILE_BYTES) >> 4);
+    if constexpr (F8) {
 #pragma unroll
-    for (int k4 = 0; k4 < 4; ++k4)
-      if (leader)
-        tc_mma_ts(tO[t], tS[t] + k4 * 8, vd + ((k4 * 2048) >> 4), IDESC_O,
-                  (accumulate || k4 > 0) ? 1u : 0u);
+      for (int k2 = 0; k2 < 2; ++k2)
+        if (leader)
+          tc_mma_ts_f8(tO[t], tS[t] + k2 * 8, vd + ((k2 * 32) >> 4), IDESC_O,
+                       (accumulate || k2 > 0) ? 1u : 0u);
+    } else {
+#pragma unroll
+      for (int k4 = 0; k4 < 4; ++k4)
+        if (leader)
+          tc_mma_ts(tO[t], tS[t] + k4 * 8, vd + ((k4 * 2048) >> 4), IDESC_O,
+                    (accumulate || k4 > 0) ? 1u : 0u);
+    }
     __syncwarp();
     return true;
   };
-  // O_t += P_t V over keys 64-127: P from shared memory (32 bytes per 16
-  // keys inside its 128-byte rows); then the whole product is marked done.
+  // O_t += P_t V over keys 64-127, P from shared memory (32 bytes per step
+  // inside its 128-byte rows: 16 bf16 or 32 FP8 keys); then the whole
+  // product is marked done.
   auto pv_hi = [&](int t, int vs, uint32_t parity) {
     if (!wait(C::BAR_P_HALF + 2 * t + 1, parity)) return false;
     tc_fence_after();
     const uint64_t vd = desc_kv_v + ((vs * C::TILE_BYTES) >> 4);
+    if constexpr (F8) {
 #pragma unroll
-    for (int k4 = 0; k4 < 4; ++k4)
-      if (leader)
-        tc_mma_ss(tO[t], desc_p[t] + ((k4 * 32) >> 4), vd + (((4 + k4) * 2048) >> 4), IDESC_O,
-                  1u);
+      for (int k2 = 0; k2 < 2; ++k2)
+        if (leader)
+          tc_mma_ss_f8(tO[t], desc_p[t] + ((k2 * 32) >> 4), vd + (((2 + k2) * 32) >> 4), IDESC_O,
+                       1u);
+    } else {
+#pragma unroll
+      for (int k4 = 0; k4 < 4; ++k4)
+        if (leader)
+          tc_mma_ss(tO[t], desc_p[t] + ((k4 * 32) >> 4), vd + (((4 + k4) * 2048) >> 4), IDESC_O,
+                    1u);
+    }
     __syncwarp();
     commit(C::BAR_PV_DONE + t);
     return true;
@@ -999,7 +853,7 @@ __device__ void role_softmax(const Sm100Ctx<D, F8, SK> &x, const FwdParams &p, i
         // exponentials, measured 3 % slower on the GQA layer.)
         const uint32_t row = x.p_hi(t) + static_cast<uint32_t>(r) * 128u;
 #pragma unroll
-        for (int c = 0; c < 8; ++c)
+        for (int c = 0; c < C::PK_WORDS / 4; ++c)  // 8 chunks (bf16) or 4 (E4M3)
           st_shared_v4(row + (static_cast<uint32_t>(c ^ (r & 7)) << 4), pk[4 * c], pk[4 * c + 1],
                        pk[4 * c + 2], pk[4 * c + 3]);
         fence_proxy_async_shared();
@@ -1118,10 +972,8 @@ __device__ __forceinline__ void fwd_kernel_body(const CUtensorMap *tm_q, const C
     } else if (warp == 9) {
       if constexpr (C::TRIPLE)
         role_mma_triple<D, F8, SK>(x, p);
-      else if constexpr (C::P_HI_SMEM)
-        role_mma_split<D, F8, SK>(x, p);
       else
-        role_mma<D, F8, SK>(x, p);
+        role_mma_split<D, F8, SK>(x, p);
     }
   } else {
     regs_increase<C::REGS_SOFTMAX>();
