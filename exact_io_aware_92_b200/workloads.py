@@ -66,9 +66,10 @@ LONG = Workload("long_causal_b1_h16_n32768_d128", 1, 16, 16, 32768, 128, True, s
 # sequence, the Llama-style GQA heads, caches of 16K-32K tokens.
 DECODE = Workload("llama_gqa_decode_b8_hq32_hkv8_nq1_nk32768_d128", 8, 32, 8, 32768, 128, True,
                   seed=6, seqlen_range=(16384, 32768), nq=1)
-# The same caches with 4 new query rows per sequence (speculative or chunked
-# decode): 8 query heads per kv head x 4 rows = 32 rows per kv head.
-DECODE_NQ4 = Workload("llama_gqa_decode_b8_hq32_hkv8_nq4_nk32768_d128", 8, 32, 8, 32768, 128,
+# Group size 8 (32 query heads on 4 kv heads) with 4 new query rows per
+# sequence (speculative or chunked decode): 8 x 4 = 32 query rows per kv head,
+# caches of 16K-32K tokens.
+DECODE_NQ4 = Workload("gqa8_decode_b8_hq32_hkv4_nq4_nk32768_d128", 8, 32, 4, 32768, 128,
                       True, seed=7, seqlen_range=(16384, 32768), nq=4)
 
 ALL = (TINY, GPT2, BERT, LLAMA_GQA, LONG)

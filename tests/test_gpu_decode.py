@@ -133,9 +133,9 @@ def test_rows_on_lanes(group, nq, splits, d):
                 what=f"d{d} G{group} nq{nq} splits{splits} causal{causal}")
 
 
-def test_rows_on_lanes_gqa_decode_workload_shape():
-    # the GQA decode workload with 4 query rows per sequence (speculative or
-    # chunked decode): 8 query heads per kv head x 4 = 32 rows; every row
+def test_rows_on_lanes_gqa8_decode_workload():
+    # group size 8 with 4 query rows per sequence (speculative or chunked
+    # decode): 8 query heads per kv head x 4 = 32 rows per kv head; every row
     w = wl.DECODE_NQ4
     inp = wl.draw_workload(w)
     o, lse = run_decode(inp, causal=w.causal, scale=w.scale)
