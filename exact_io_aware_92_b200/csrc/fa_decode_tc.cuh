@@ -751,25 +751,47 @@ __global__ void __launch_bounds__(128) fa_decode_tc_combine_kernel(const DecodeP
   const long long s = static_cast<long long>(b) * p.Hkv + g;
   const long long off = before * p.Hkv + static_cast<long long>(g) * n;
   const long long c0 = cta_of(off), c1 = cta_of(off + n - 1);
+  const unsigned full = 0xffffffffu;
   // Launched as a programmatic dependent of the split kernel: everything
   // above overlapped its tail; the partials are read only after it is done.
   asm volatile("griddepcontrol.wait;" ::: "memory");
+  // The row's pieces, 32 at a time, one per lane: the row max M first, then
+  // each lane's weight 2^(m - M) and the weighted sums.  The partial rows of
+  // a batch of pieces are independent loads.
   float M = -INFINITY;
-  for (long long c = c0; c <= c1; ++c)
-    if (start(c + 1) > start(c)) M = fmaxf(M, p.part_ml[((c + s) * QROWS + r) * 2]);
+  for (long long cb = c0; cb <= c1; cb += 32) {
+    const long long c = cb + lane;
+    const bool has = c <= c1 && start(c + 1) > start(c);
+    const float m = has ? p.part_ml[((c + s) * QROWS + r) * 2] : -INFINITY;
+    M = fmaxf(M, warp_max_f32(m));
+  }
   const float mu = M == -INFINITY ? 0.f : M;
   float acc[PER];
 #pragma unroll
   for (int e = 0; e < PER; ++e) acc[e] = 0.f;
   float L = 0.f;
-  for (long long c = c0; c <= c1; ++c) {
-    if (start(c + 1) <= start(c)) continue;
-    const long long slot = (c + s) * QROWS + r;
-    const float wgt = ex2_approx(p.part_ml[slot * 2] - mu);
-    L += wgt * p.part_ml[slot * 2 + 1];
+  for (long long cb = c0; cb <= c1; cb += 32) {
+    const long long c = cb + lane;
+    const bool has = c <= c1 && start(c + 1) > start(c);
+    float wgt = 0.f;
+    if (has) {
+      const long long slot = (c + s) * QROWS + r;
+      wgt = ex2_approx(p.part_ml[slot * 2] - mu);
+      L += wgt * p.part_ml[slot * 2 + 1];
+    }
+    const int cnt = static_cast<int>(min(32ll, c1 - cb + 1));
+#pragma unroll 4
+    for (int j = 0; j < cnt; ++j) {
+      const float wj = __shfl_sync(full, wgt, j);
+      if (wj != 0.f) {
+        const float *po = p.part_o + ((cb + j + s) * QROWS + r) * D + lane * PER;
 #pragma unroll
-    for (int e = 0; e < PER; ++e) acc[e] += wgt * p.part_o[slot * D + lane * PER + e];
+        for (int e = 0; e < PER; ++e) acc[e] += wj * po[e];
+      }
+    }
   }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) L += __shfl_xor_sync(full, L, o);
   const float inv = L > 0.f ? 1.0f / L : 0.f;
 #pragma unroll
   for (int e = 0; e < PER; e += 2)
