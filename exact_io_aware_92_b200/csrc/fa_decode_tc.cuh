@@ -755,39 +755,54 @@ __global__ void __launch_bounds__(128) fa_decode_tc_combine_kernel(const DecodeP
   // Launched as a programmatic dependent of the split kernel: everything
   // above overlapped its tail; the partials are read only after it is done.
   asm volatile("griddepcontrol.wait;" ::: "memory");
-  // The row's pieces, 32 at a time, one per lane: the row max M first, then
-  // each lane's weight 2^(m - M) and the weighted sums.  The partial rows of
-  // a batch of pieces are independent loads.
-  float M = -INFINITY;
-  for (long long cb = c0; cb <= c1; cb += 32) {
+  // The row's pieces, 32 at a time, one per lane: (m, l) of each first and
+  // the row max M, then each lane's weight 2^(m - M), and the weighted O
+  // rows with 8 pieces' loads in flight at a time.  With at most 32 pieces
+  // (the usual case) every (m, l) is read once.
+  // share c holds tiles unless the call has fewer tiles than CTAs
+  auto has = [&](long long c) { return T >= grid || start(c + 1) > start(c); };
+  const float2 *ml_all = reinterpret_cast<const float2 *>(p.part_ml);
+  auto load_ml = [&](long long cb) {
     const long long c = cb + lane;
-    const bool has = c <= c1 && start(c + 1) > start(c);
-    const float m = has ? p.part_ml[((c + s) * QROWS + r) * 2] : -INFINITY;
-    M = fmaxf(M, warp_max_f32(m));
-  }
+    return c <= c1 && has(c) ? ml_all[(c + s) * QROWS + r] : make_float2(-INFINITY, 0.f);
+  };
+  const float2 ml0 = load_ml(c0);
+  float M = warp_max_f32(ml0.x);
+  for (long long cb = c0 + 32; cb <= c1; cb += 32) M = fmaxf(M, warp_max_f32(load_ml(cb).x));
   const float mu = M == -INFINITY ? 0.f : M;
   float acc[PER];
 #pragma unroll
   for (int e = 0; e < PER; ++e) acc[e] = 0.f;
   float L = 0.f;
   for (long long cb = c0; cb <= c1; cb += 32) {
-    const long long c = cb + lane;
-    const bool has = c <= c1 && start(c + 1) > start(c);
-    float wgt = 0.f;
-    if (has) {
-      const long long slot = (c + s) * QROWS + r;
-      wgt = ex2_approx(p.part_ml[slot * 2] - mu);
-      L += wgt * p.part_ml[slot * 2 + 1];
-    }
+    const float2 ml = cb == c0 ? ml0 : load_ml(cb);
+    const float wgt = ml.x == -INFINITY ? 0.f : ex2_approx(ml.x - mu);
+    L += wgt * ml.y;
     const int cnt = static_cast<int>(min(32ll, c1 - cb + 1));
-#pragma unroll 4
-    for (int j = 0; j < cnt; ++j) {
-      const float wj = __shfl_sync(full, wgt, j);
-      if (wj != 0.f) {
-        const float *po = p.part_o + ((cb + j + s) * QROWS + r) * D + lane * PER;
+    for (int j0 = 0; j0 < cnt; j0 += 8) {
+      float wj[8], v[8][PER];
 #pragma unroll
-        for (int e = 0; e < PER; ++e) acc[e] += wj * po[e];
+      for (int u = 0; u < 8; ++u) {
+        wj[u] = j0 + u < cnt ? __shfl_sync(full, wgt, (j0 + u) & 31) : 0.f;
+        const float *po = p.part_o + ((cb + j0 + u + s) * QROWS + r) * D + lane * PER;
+        if constexpr (PER == 4) {
+          const float4 x = wj[u] != 0.f ? *reinterpret_cast<const float4 *>(po)
+                                        : make_float4(0.f, 0.f, 0.f, 0.f);
+          v[u][0] = x.x;
+          v[u][1] = x.y;
+          v[u][2] = x.z;
+          v[u][3] = x.w;
+        } else {
+          const float2 x = wj[u] != 0.f ? *reinterpret_cast<const float2 *>(po)
+                                        : make_float2(0.f, 0.f);
+          v[u][0] = x.x;
+          v[u][1] = x.y;
+        }
       }
+#pragma unroll
+      for (int u = 0; u < 8; ++u)
+#pragma unroll
+        for (int e = 0; e < PER; ++e) acc[e] += wj[u] * v[u][e];
     }
   }
 #pragma unroll
