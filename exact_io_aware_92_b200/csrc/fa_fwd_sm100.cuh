@@ -178,7 +178,11 @@ struct Sm100Cfg {
 #ifndef FA_EXP2_EMU_PAIRS_D128
 #define FA_EXP2_EMU_PAIRS_D128 2
 #endif
-  static constexpr int EXP2_EMU_PAIRS = D == 64 ? FA_EXP2_EMU_PAIRS_D64 : FA_EXP2_EMU_PAIRS_D128;
+#ifndef FA_EXP2_EMU_PAIRS_F8
+#define FA_EXP2_EMU_PAIRS_F8 2
+#endif
+  static constexpr int EXP2_EMU_PAIRS =
+      F8 ? FA_EXP2_EMU_PAIRS_F8 : D == 64 ? FA_EXP2_EMU_PAIRS_D64 : FA_EXP2_EMU_PAIRS_D128;
 };
 
 // One work unit, as every role sees it.  Rows and keys are counted from the
