@@ -4,9 +4,9 @@ allocation, a latency path that cannot afford cudaMalloc's implicit device
 synchronisation).  It keeps its partials in the library's own 8 MiB device
 array instead of a caller workspace.
 
-The test queues two calls in a row through the C ABI on one stream, the
-larger layout first, so that the second call runs over the partials the
-first one left in the shared array.  Only then are the outputs read, and
+The test queues three calls in a row through the C ABI on one stream, the
+largest layout first, so that each later call runs over the partials an
+earlier one left in the shared array.  Only then are the outputs read, and
 each is checked element by element against the fp64 oracle (queries at the
 end of their sequences) within the tolerances of the parity tests, and
 against fa_fwd_decode with a caller-provided workspace on the same inputs.
@@ -25,8 +25,11 @@ pytestmark = pytest.mark.gpu
 
 SCRATCH_BYTES = 8 << 20
 
-# the larger layout first (more key tiles and pieces), then a smaller one
+# Largest layout first, so that each later call runs over partials that an
+# earlier, larger one left in the shared array: 32 rows per kv head (the
+# rows-on-lanes kernel), then 4 and 8 (keys on the lanes).
 CASES = [
+    dict(B=2, Hq=16, Hkv=2, Nq=4, Nk=6000, d=128, causal=True, seed=903, lens=[6000, 2500]),
     dict(B=4, Hq=32, Hkv=8, Nq=1, Nk=8192, d=128, causal=True, seed=901, lens=None),
     dict(B=3, Hq=16, Hkv=4, Nq=2, Nk=3000, d=64, causal=True, seed=902, lens=[3000, 1, 1500]),
 ]
@@ -60,13 +63,13 @@ def _host(o, lse):
     return o.float().cpu().numpy().astype(np.float64), lse.cpu().numpy().astype(np.float64)
 
 
-def test_noalloc_two_calls_in_a_row_match_oracle_and_workspace_entry_point():
+def test_noalloc_calls_in_a_row_match_oracle_and_workspace_entry_point():
     import torch
     lib = _lib.load()
     stream = torch.cuda.current_stream().cuda_stream
     status = torch.zeros(1, dtype=torch.int32, device="cuda")
     cases = [_prepare(c) for c in CASES]
-    # both no-allocation calls queued back to back, nothing read in between
+    # the no-allocation calls queued back to back, nothing read in between
     got = []
     for t in cases:
         assert 0 < lib.fa_decode_workspace_size(*t["shape"], 0) <= SCRATCH_BYTES
