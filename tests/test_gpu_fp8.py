@@ -113,3 +113,10 @@ def test_fp8_full_gqa_workload_sampled_rows():
     w = wl.LLAMA_GQA_FP8
     rows = wl.sample_rows(w, 16)
     print(run_case(w.B, w.Hq, w.Hkv, w.N, w.causal, w.seed, k_scale=w.k_scale, rows=rows))
+
+
+def test_fp8_kv_beyond_l2_sampled_rows():
+    # 134 MB of E4M3 K/V, more than the L2, 32 heads of 16384 keys
+    w = wl.Workload("fp8_kv_beyond_l2", 1, 32, 32, 16384, 128, True, seed=2200)
+    rows = wl.sample_rows(w, 16)
+    print(run_case(1, 32, 32, 16384, True, 2200, k_scale=2.0, rows=rows))

@@ -134,6 +134,25 @@ def test_long_d64_sampled_rows(causal, lens):
             what=f"long d64 causal={causal}")
 
 
+@pytest.mark.parametrize("B,H,N,d,causal", [(1, 16, 16384, 128, False), (4, 16, 16384, 64, True)])
+def test_kv_beyond_l2_sampled_rows(B, H, N, d, causal):
+    # 134 and 268 MB of K/V, more than the 126 MB L2: query tiles of a head
+    # read its K/V tiles again from DRAM; many units per CTA at d = 64.
+    inp = wl.draw(B, H, H, N, d, seed=2100 + d, k_scale=2.0)
+    scale = 1.0 / np.sqrt(d)
+    o, lse = run_bf16(inp, causal=causal, scale=scale)
+    assert np.all(np.isfinite(o))
+    w = wl.Workload("kv_beyond_l2", B, H, H, N, d, causal, seed=2100 + d)
+    rows = wl.sample_rows(w, 24)
+    rows[:, 0] = 0
+    rows[:, -1] = N - 1
+    rows.sort(axis=1)
+    o_ref, lse_ref = reference(inp, causal=causal, scale=scale, rows=rows)
+    og, lg = gather_rows(o, lse, rows)
+    compare(og, lg, o_ref, lse_ref, o_tol=O_TOL_BF16, lse_tol=LSE_TOL_BF16,
+            what=f"K/V beyond L2 d{d} causal={causal}")
+
+
 def test_deterministic():
     inp = wl.draw(2, 8, 2, 1000, 128, seed=55)
     a = run_bf16(inp, causal=True, scale=0.088)
