@@ -41,8 +41,14 @@ def run_case(B, Hq, Hkv, N, d, causal, seed, seqlens=None):
     o_ref, _, p = reference(inp, causal=causal, scale=scale, return_probs=True)
     bounds = derived_grad_bounds(inp, dout_bits, p, o_ref, derived_o_bound(inp, p, o_ref, s32),
                                  ref, s32)
+    return compare_grads((dq, dk, dv), ref, bounds)
+
+
+def compare_grads(grads, ref, bounds):
+    """Every element of each GPU gradient within its derived bound; returns
+    the largest error and error / bound per gradient."""
     out = {}
-    for name, g, r, bd in zip(("dq", "dk", "dv"), (dq, dk, dv), ref, bounds):
+    for name, g, r, bd in zip(("dq", "dk", "dv"), grads, ref, bounds):
         g = g.float().cpu().numpy().astype(np.float64)
         assert np.all(np.isfinite(g)), name
         err = np.abs(g - r)
@@ -73,3 +79,38 @@ def test_backward_llama_layer_shape():
     # one layer's worth of the GQA workload at N = 1024 (the oracle's fp64
     # backward of the full N = 8192 layer would take hours on the host)
     print(run_case(1, 8, 2, 1024, 128, True, seed=1500))
+
+
+def test_backward_gqa_layer_full_size_one_group():
+    # The GQA layer's backward at full size, in the shape and launch
+    # configuration the benchmark times (B2 Hq32 Hkv8 N8192 d128, K x 2).  The
+    # oracle checks every element of one (batch, kv head) group: the dQ of
+    # its four query heads and its dK and dV, which depend on nothing outside
+    # the group.  The host side (oracle backward and the per-element bounds
+    # over 8192 x 8192 probabilities) takes 2 to 9 minutes and 8 GB.
+    import torch
+    from exact_io_aware_92_b200 import attention
+    w = wl.LLAMA_GQA
+    inp = wl.draw_workload(w)
+    dout_bits = wl.round_to_bf16_bits(np.random.default_rng(w.seed + 7).standard_normal(
+        (w.B, w.Hq, w.N, w.d), dtype=np.float32))
+    q, k, v, do = (to_device_bf16(x) for x in (inp.q_bits, inp.k_bits, inp.v_bits, dout_bits))
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    o, lse = attention.fwd(q, k, v, causal=True, scale=w.scale, status=status)
+    dq, dk, dv = attention.bwd(q, k, v, o, do, lse, causal=True, scale=w.scale, status=status)
+    assert attention.check_status(status) == 0
+    b, g = 1, 5
+    G = w.Hq // w.Hkv
+    hs = slice(g * G, (g + 1) * G)
+    part = wl.Inputs(q_bits=inp.q_bits[b:b + 1, hs], k_bits=inp.k_bits[b:b + 1, g:g + 1],
+                     v_bits=inp.v_bits[b:b + 1, g:g + 1], seqlens=None)
+    dout_part = np.ascontiguousarray(dout_bits[b:b + 1, hs])
+    s32 = float(np.float32(w.scale))
+    ref = oracle.attention_backward(part.q_bits, part.k_bits, part.v_bits, dout_part, causal=True,
+                                    scale=s32)
+    o_ref, _, p = reference(part, causal=True, scale=w.scale, return_probs=True)
+    bounds = derived_grad_bounds(part, dout_part, p, o_ref, derived_o_bound(part, p, o_ref, s32),
+                                 ref, s32)
+    del p
+    print(compare_grads((dq[b:b + 1, hs], dk[b:b + 1, g:g + 1], dv[b:b + 1, g:g + 1]), ref,
+                        bounds))

@@ -153,6 +153,32 @@ def test_kv_beyond_l2_sampled_rows(B, H, N, d, causal):
             what=f"K/V beyond L2 d{d} causal={causal}")
 
 
+@pytest.mark.parametrize("B,Hq,Hkv,N,d,causal", [
+    (2, 32, 8, 8000, 128, True),     # 8000 = 31 * 256 + 64: 64 rows in Q tile 0, none in Q tile 1
+    (2, 16, 4, 6001, 128, False),    # 6001 = 23 * 256 + 113: Q tile 1 of the last unit is empty
+    (1, 8, 2, 12345, 64, True),      # d = 64 three-buffer sequence with a ragged tail
+    (3, 8, 8, 10184, 64, False),     # 10184 = 39 * 256 + 200: Q tile 1 holds 72 rows
+])
+def test_ragged_length_at_scale_sampled_rows(B, Hq, Hkv, N, d, causal):
+    # Many units per CTA, a partial last round of the unit order, and a last
+    # unit whose Q and key tiles are cut short: rows around every tail
+    # boundary are always checked, the rest sampled.
+    inp = wl.draw(B, Hq, Hkv, N, d, seed=2300 + N % 97, k_scale=2.0)
+    scale = 1.0 / np.sqrt(d)
+    o, lse = run_bf16(inp, causal=causal, scale=scale)
+    assert np.all(np.isfinite(o)) and np.all(np.isfinite(lse))
+    rng = np.random.default_rng(2300 + N)
+    tail = [N - 257, N - 256, N - 255, N - 129, N - 128, N - 127, N - 2, N - 1]
+    rows = np.empty((B * Hq, 1 + 16 + len(tail)), dtype=np.int64)
+    for bh in range(B * Hq):
+        rows[bh] = np.sort(np.concatenate(
+            [[0], rng.choice(np.arange(1, N - 300), size=16, replace=False), tail]))
+    o_ref, lse_ref = reference(inp, causal=causal, scale=scale, rows=rows)
+    og, lg = gather_rows(o, lse, rows)
+    compare(og, lg, o_ref, lse_ref, o_tol=O_TOL_BF16, lse_tol=LSE_TOL_BF16,
+            what=f"ragged N={N} d{d} causal={causal}")
+
+
 def test_deterministic():
     inp = wl.draw(2, 8, 2, 1000, 128, seed=55)
     a = run_bf16(inp, causal=True, scale=0.088)
