@@ -113,6 +113,23 @@ def test_full_workload_sampled_rows(w):
     compare(og, lg, o_ref, lse_ref, o_tol=O_TOL_BF16, lse_tol=LSE_TOL_BF16, what=w.name)
 
 
+def test_llama_gqa_every_row_of_one_group():
+    # The contract launch (B2 Hq32 Hkv8 N8192 d128, K x 2) with every output
+    # row of one (batch, kv head) group checked: its four query heads' O and
+    # LSE depend only on that group's Q, K and V.
+    w = wl.LLAMA_GQA
+    inp = wl.draw_workload(w)
+    o, lse = run_bf16(inp, causal=w.causal, scale=w.scale)
+    b, g = 0, 3
+    G = w.Hq // w.Hkv
+    hs = slice(g * G, (g + 1) * G)
+    part = wl.Inputs(q_bits=inp.q_bits[b:b + 1, hs], k_bits=inp.k_bits[b:b + 1, g:g + 1],
+                     v_bits=inp.v_bits[b:b + 1, g:g + 1], seqlens=None)
+    o_ref, lse_ref = reference(part, causal=w.causal, scale=w.scale)
+    compare(o[b:b + 1, hs], lse[b:b + 1, hs], o_ref, lse_ref, o_tol=O_TOL_BF16,
+            lse_tol=LSE_TOL_BF16, what=f"{w.name} group (b={b}, kv head {g})")
+
+
 @pytest.mark.parametrize("causal,lens", [(True, None), (False, [4096, 2500, 1, 3333])])
 def test_long_d64_sampled_rows(causal, lens):
     # d = 64 rotates three S buffers over both Q tiles' products: units of up
