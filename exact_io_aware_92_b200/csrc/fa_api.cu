@@ -39,7 +39,7 @@ struct DeviceState {
   bool ok = false;
   int num_sms = 0;
   int *status_word = nullptr;  // device address of g_status_word
-  bool attr64 = false, attr64_causal = false, attr128 = false;
+  bool fwd_attr[2][4] = {};  // [d = 64, 128][launch variant: fa::kVarSkip0 | fa::kVarPacked]
   bool dec_attr64 = false, dec_attr128 = false;
   bool dec_tc_attr[2][3] = {};  // [d = 64, 128][4, 8, 16 row slots]
   bool dec_rows_attr[2] = {};    // [d = 64, 128]: 17 to 128 rows per kv head
@@ -276,13 +276,17 @@ int launch_bf16(DeviceState *ds, const void *q, const void *k, const void *v, vo
   using C = fa::Sm100Cfg<D>;
   // Causal launches at d = 64 use the instance in which Q tile 0 skips a
   // unit's last key tile (wholly above its rows) inside the three-buffer
-  // sequence.
-  const bool sk = D == 64 && causal;
-  auto kernel = fa::fa_fwd_bf16_sm100_kernel<D, false>;
+  // sequence; packed sequences their own instance, so that dense launches
+  // decode units without the packed layout's branch.
+  const int var = (D == 64 && causal ? fa::kVarSkip0 : 0) | (cu_seqlens ? fa::kVarPacked : 0);
+  auto kernel = fa::fa_fwd_bf16_sm100_kernel<D, 0>;
+  if (var == fa::kVarPacked) kernel = fa::fa_fwd_bf16_sm100_kernel<D, fa::kVarPacked>;
   if constexpr (D == 64) {
-    if (sk) kernel = fa::fa_fwd_bf16_sm100_kernel<64, true>;
+    if (var == fa::kVarSkip0) kernel = fa::fa_fwd_bf16_sm100_kernel<64, fa::kVarSkip0>;
+    if (var == (fa::kVarSkip0 | fa::kVarPacked))
+      kernel = fa::fa_fwd_bf16_sm100_kernel<64, fa::kVarSkip0 | fa::kVarPacked>;
   }
-  bool &attr = sk ? ds->attr64_causal : (D == 64) ? ds->attr64 : ds->attr128;
+  bool &attr = ds->fwd_attr[D == 128][var];
   if (!attr) {
     const int rc = prepare_fwd_kernel<C>(kernel);
     if (rc != FA_OK) return rc;

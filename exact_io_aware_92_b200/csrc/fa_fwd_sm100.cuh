@@ -95,9 +95,15 @@ struct FwdParams {
 // F8: Q, K and V are FP8 E4M3 codes (head dim 128 only) and V arrives
 // transposed ([d, keys], keys contiguous), so both products read K-major
 // operands; otherwise bf16.
-// SK: causal launches at d = 64, where Q tile 0 skips a unit's last key tile
-// inside the three-buffer sequence; every other launch compiles without it.
-template <int D, bool F8 = false, bool SK = false>
+// V, the launch variant (bit flags):
+//  kVarSkip0: causal launches at d = 64, where Q tile 0 skips a unit's last
+//    key tile inside the three-buffer sequence;
+//  kVarPacked: the packed layout (cu_seqlens), whose unit decode and tensor
+//    map coordinates differ; dense launches compile without that branch.
+constexpr int kVarSkip0 = 1;
+constexpr int kVarPacked = 2;
+
+template <int D, bool F8 = false, int V = 0>
 struct Sm100Cfg {
   static_assert(D == 64 || D == 128, "head dim 64 or 128");
   static_assert(!F8 || D == 128, "FP8 inputs: head dim 128");
@@ -134,7 +140,8 @@ struct Sm100Cfg {
   // interleaved), so a Q tile's next S is computed while it still works on
   // the current one.
   static constexpr bool TRIPLE = (D == 64) && !F8;
-  static constexpr bool SKIP0 = TRIPLE && SK;
+  static constexpr bool SKIP0 = TRIPLE && (V & kVarSkip0) != 0;
+  static constexpr bool PACKED = (V & kVarPacked) != 0;
   static constexpr int NSBUF = TRIPLE ? 3 : 2;
   static constexpr int BAR_S_FULL = 4 + 2 * STAGES;     // [NSBUF]
   static constexpr int BAR_P_HALF = BAR_S_FULL + NSBUF; // [NSBUF][2 halves of the keys]
@@ -201,9 +208,9 @@ struct Unit {
   size_t lse_base; // offset of row 0 in LSE
 };
 
-template <int D, bool F8, bool SK>
+template <int D, bool F8, int V>
 __device__ __forceinline__ Unit unit_at(const FwdParams &p, int u) {
-  using C = Sm100Cfg<D, F8, SK>;
+  using C = Sm100Cfg<D, F8, V>;
   Unit x;
   const int BH = p.B * p.Hq;
   const int q_bh = p.div_bh.div(u);
@@ -214,7 +221,7 @@ __device__ __forceinline__ Unit unit_at(const FwdParams &p, int u) {
   x.hkv = p.div_group.div(x.h);
   x.row0 = qp * C::ROWS_PER_UNIT;
   int L = p.N;
-  if (p.cu_seqlens) {
+  if constexpr (C::PACKED) {
     x.tok0 = p.cu_seqlens[x.b];
     L = max(p.cu_seqlens[x.b + 1] - x.tok0, 0);
     x.q_rows = L;
@@ -255,9 +262,9 @@ __device__ __forceinline__ int snake_unit(int k, int num_units) {
   return u < num_units ? u : -1;
 }
 
-template <int D, bool F8, bool SK>
+template <int D, bool F8, int V>
 struct Sm100Ctx {
-  using C = Sm100Cfg<D, F8, SK>;
+  using C = Sm100Cfg<D, F8, V>;
   uint32_t smem;      // 1 KB aligned shared base (shared-window address)
   uint32_t tmem;      // tensor-memory base address
   volatile int *abort_flag;
@@ -269,23 +276,23 @@ struct Sm100Ctx {
 };
 
 // Ring position of K tile g (V tile g is the next one) in a CTA's stream.
-template <int D, bool F8, bool SK>
-__device__ __forceinline__ int ring_slot(int seq) { return seq % Sm100Cfg<D, F8, SK>::STAGES; }
-template <int D, bool F8, bool SK>
+template <int D, bool F8, int V>
+__device__ __forceinline__ int ring_slot(int seq) { return seq % Sm100Cfg<D, F8, V>::STAGES; }
+template <int D, bool F8, int V>
 __device__ __forceinline__ uint32_t ring_parity(int seq) {
-  return static_cast<uint32_t>((seq / Sm100Cfg<D, F8, SK>::STAGES) & 1);
+  return static_cast<uint32_t>((seq / Sm100Cfg<D, F8, V>::STAGES) & 1);
 }
 
 // --------------------------------------------------------------------------
 // TMA producer (one thread)
 // --------------------------------------------------------------------------
-template <int D, bool F8, bool SK>
-__device__ void role_producer(const Sm100Ctx<D, F8, SK> &x, const FwdParams &p, const CUtensorMap *tm_q,
+template <int D, bool F8, int V>
+__device__ void role_producer(const Sm100Ctx<D, F8, V> &x, const FwdParams &p, const CUtensorMap *tm_q,
                               const CUtensorMap *tm_k, const CUtensorMap *tm_v) {
-  using C = Sm100Cfg<D, F8, SK>;
+  using C = Sm100Cfg<D, F8, V>;
   int seq = 0;  // K/V tiles put into the ring so far (K and V counted apart)
   int qi = 0;   // units with keys loaded so far
-  const bool packed = p.cu_seqlens != nullptr;
+  constexpr bool packed = C::PACKED;
   // K/V tiles are read by every query tile of their head, Q tiles once: keep
   // K/V in L2 ahead of Q (and of O, written with streaming stores).  On the
   // GQA layer this cut DRAM reads from 343 to 289 MB per launch.
@@ -295,7 +302,7 @@ __device__ void role_producer(const Sm100Ctx<D, F8, SK> &x, const FwdParams &p, 
     const int u = snake_unit(k, p.num_units);
     if (u == -2) break;
     if (u < 0) continue;
-    const Unit w = unit_at<D, F8, SK>(p, u);
+    const Unit w = unit_at<D, F8, V>(p, u);
     if (w.nkv == 0) continue;
     // Q tile t of this unit replaces the previous unit's once its last
     // S product has read it.
@@ -319,8 +326,8 @@ __device__ void role_producer(const Sm100Ctx<D, F8, SK> &x, const FwdParams &p, 
     const int kv_plane = w.kv_plane;
     for (int j = 0; j < w.nkv && ok; ++j) {
       for (int kv = 0; kv < 2; ++kv, ++seq) {
-        const int slot = ring_slot<D, F8, SK>(seq);
-        if (!mbar_wait_bounded(x.bar(C::BAR_KV_EMPTY + slot), ring_parity<D, F8, SK>(seq) ^ 1,
+        const int slot = ring_slot<D, F8, V>(seq);
+        if (!mbar_wait_bounded(x.bar(C::BAR_KV_EMPTY + slot), ring_parity<D, F8, V>(seq) ^ 1,
                                x.abort_flag, p.status, p.wait_limit_ns, kErrTimeout)) {
           ok = false;
           break;
@@ -348,7 +355,7 @@ __device__ void role_producer(const Sm100Ctx<D, F8, SK> &x, const FwdParams &p, 
                         p.wait_limit_ns, kErrTimeout);
   for (int s = 0; s < C::STAGES && s < seq; ++s) {
     const int last = s + C::STAGES * ((seq - 1 - s) / C::STAGES);
-    mbar_wait_bounded(x.bar(C::BAR_KV_FULL + s), ring_parity<D, F8, SK>(last), &never, p.status,
+    mbar_wait_bounded(x.bar(C::BAR_KV_FULL + s), ring_parity<D, F8, V>(last), &never, p.status,
                       p.wait_limit_ns, kErrTimeout);
   }
 }
@@ -362,9 +369,9 @@ __device__ void role_producer(const Sm100Ctx<D, F8, SK> &x, const FwdParams &p, 
 // over the upper 64 keys (P from shared memory).  S_t(j) thus waits only for
 // the first half of the previous tile's probabilities.
 // --------------------------------------------------------------------------
-template <int D, bool F8, bool SK>
-__device__ void role_mma_split(const Sm100Ctx<D, F8, SK> &x, const FwdParams &p) {
-  using C = Sm100Cfg<D, F8, SK>;
+template <int D, bool F8, int V>
+__device__ void role_mma_split(const Sm100Ctx<D, F8, V> &x, const FwdParams &p) {
+  using C = Sm100Cfg<D, F8, V>;
   static_assert(C::P_HI_SMEM && !C::TRIPLE, "two S buffers, P's upper half in shared memory");
   // S: Q and K both K-major.  O: P K-major (tensor memory or shared memory);
   // V MN-major (bf16) or V^T K-major (FP8).
@@ -461,31 +468,31 @@ __device__ void role_mma_split(const Sm100Ctx<D, F8, SK> &x, const FwdParams &p)
     const int u = snake_unit(k, p.num_units);
     if (u == -2) break;
     if (u < 0) continue;
-    const Unit w = unit_at<D, F8, SK>(p, u);
+    const Unit w = unit_at<D, F8, V>(p, u);
     const int n1 = w.nkv, n0 = w.nkv0;  // n0 is n1 or n1 - 1
     if (n1 == 0) continue;
     const uint32_t qpar = static_cast<uint32_t>(qi & 1);
     if (!wait(C::BAR_Q_FULL + 0, qpar) || !wait(C::BAR_Q_FULL + 1, qpar) ||
-        !wait(C::BAR_KV_FULL + ring_slot<D, F8, SK>(2 * g), ring_parity<D, F8, SK>(2 * g))) {
+        !wait(C::BAR_KV_FULL + ring_slot<D, F8, V>(2 * g), ring_parity<D, F8, V>(2 * g))) {
       ok = false;
       break;
     }
     tc_fence_after();
-    issue_s(0, ring_slot<D, F8, SK>(2 * g));
+    issue_s(0, ring_slot<D, F8, V>(2 * g));
     commit(C::BAR_S_FULL + 0);
     if (n0 == 1) commit(C::BAR_Q_EMPTY + 0);
-    issue_s(1, ring_slot<D, F8, SK>(2 * g));
+    issue_s(1, ring_slot<D, F8, V>(2 * g));
     commit(C::BAR_S_FULL + 1);
-    commit(C::BAR_KV_EMPTY + ring_slot<D, F8, SK>(2 * g));
+    commit(C::BAR_KV_EMPTY + ring_slot<D, F8, V>(2 * g));
     if (n1 == 1) commit(C::BAR_Q_EMPTY + 1);
     for (int j = 1; j < n1; ++j) {
       const int gp = g + j - 1, gc = g + j;
-      const int vs = ring_slot<D, F8, SK>(2 * gp + 1), ks = ring_slot<D, F8, SK>(2 * gc);
+      const int vs = ring_slot<D, F8, V>(2 * gp + 1), ks = ring_slot<D, F8, V>(2 * gc);
       const uint32_t par0 = static_cast<uint32_t>((gs[0] + j - 1) & 1);
       const uint32_t par1 = static_cast<uint32_t>((gs[1] + j - 1) & 1);
-      if (!wait(C::BAR_KV_FULL + vs, ring_parity<D, F8, SK>(2 * gp + 1)) ||
+      if (!wait(C::BAR_KV_FULL + vs, ring_parity<D, F8, V>(2 * gp + 1)) ||
           !pv_lo(0, vs, par0, j - 1 > 0) ||
-          !wait(C::BAR_KV_FULL + ks, ring_parity<D, F8, SK>(2 * gc))) {
+          !wait(C::BAR_KV_FULL + ks, ring_parity<D, F8, V>(2 * gc))) {
         ok = false;
         break;
       }
@@ -517,8 +524,8 @@ __device__ void role_mma_split(const Sm100Ctx<D, F8, SK> &x, const FwdParams &p)
     if (!ok) break;
     // Last tile's PV products, then the unit's output is complete.
     const int gl = g + n1 - 1;
-    const int vs = ring_slot<D, F8, SK>(2 * gl + 1);
-    if (!wait(C::BAR_KV_FULL + vs, ring_parity<D, F8, SK>(2 * gl + 1))) {
+    const int vs = ring_slot<D, F8, V>(2 * gl + 1);
+    if (!wait(C::BAR_KV_FULL + vs, ring_parity<D, F8, V>(2 * gl + 1))) {
       ok = false;
       break;
     }
@@ -557,9 +564,9 @@ __device__ void role_mma_split(const Sm100Ctx<D, F8, SK> &x, const FwdParams &p)
 // buffer (phase T / 3), PV done per Q tile (one phase per tile), O full per
 // Q tile and unit.
 // --------------------------------------------------------------------------
-template <int D, bool F8, bool SK>
-__device__ void role_mma_triple(const Sm100Ctx<D, F8, SK> &x, const FwdParams &p) {
-  using C = Sm100Cfg<D, F8, SK>;
+template <int D, bool F8, int V>
+__device__ void role_mma_triple(const Sm100Ctx<D, F8, V> &x, const FwdParams &p) {
+  using C = Sm100Cfg<D, F8, V>;
   static_assert(C::TRIPLE, "three S buffers: bf16, head dim 64");
   constexpr uint32_t IDESC_S = idesc_bf16_f32(128, C::BN, 0, 0);  // Q, K both K-major
   constexpr uint32_t IDESC_O = idesc_bf16_f32(128, D, 0, 1);      // P from TMEM, V MN-major
@@ -587,7 +594,7 @@ __device__ void role_mma_triple(const Sm100Ctx<D, F8, SK> &x, const FwdParams &p
     const int u = snake_unit(k, p.num_units);
     if (u == -2) break;
     if (u < 0) continue;
-    const Unit w = unit_at<D, F8, SK>(p, u);
+    const Unit w = unit_at<D, F8, V>(p, u);
     const int n = w.nkv;
     if (n == 0) continue;
     // In a causal unit Q tile 0 may skip the last key tile (it lies wholly
@@ -602,9 +609,9 @@ __device__ void role_mma_triple(const Sm100Ctx<D, F8, SK> &x, const FwdParams &p
     // by Q tile 0's product and released after Q tile 1's.
     auto issue_s = [&](int tt) {
       const int j = (tt - t0) >> 1, q = (tt - t0) & 1;
-      const int ks = ring_slot<D, F8, SK>(2 * (g + j));
+      const int ks = ring_slot<D, F8, V>(2 * (g + j));
       if (q == 0) {
-        if (!wait(C::BAR_KV_FULL + ks, ring_parity<D, F8, SK>(2 * (g + j)))) return false;
+        if (!wait(C::BAR_KV_FULL + ks, ring_parity<D, F8, V>(2 * (g + j)))) return false;
         tc_fence_after();
       }
       const uint64_t kd = desc_kv_k + ((ks * C::TILE_BYTES) >> 4);
@@ -626,8 +633,8 @@ __device__ void role_mma_triple(const Sm100Ctx<D, F8, SK> &x, const FwdParams &p
     for (int tt = t0; ok && tt < t0 + 3 && tt < tend; ++tt) ok = issue_s(tt);
     for (int tp = t0; ok && tp < tend; ++tp) {
       const int j = (tp - t0) >> 1, q = (tp - t0) & 1;
-      const int vs = ring_slot<D, F8, SK>(2 * (g + j) + 1);
-      if (q == 0 && !wait(C::BAR_KV_FULL + vs, ring_parity<D, F8, SK>(2 * (g + j) + 1))) {
+      const int vs = ring_slot<D, F8, V>(2 * (g + j) + 1);
+      if (q == 0 && !wait(C::BAR_KV_FULL + vs, ring_parity<D, F8, V>(2 * (g + j) + 1))) {
         ok = false;
         break;
       }
@@ -676,9 +683,9 @@ __device__ void role_mma_triple(const Sm100Ctx<D, F8, SK> &x, const FwdParams &p
 // --------------------------------------------------------------------------
 // Softmax warpgroup t (128 threads, one query row each)
 // --------------------------------------------------------------------------
-template <int D, bool F8, bool SK>
-__device__ void role_softmax(const Sm100Ctx<D, F8, SK> &x, const FwdParams &p, int t) {
-  using C = Sm100Cfg<D, F8, SK>;
+template <int D, bool F8, int V>
+__device__ void role_softmax(const Sm100Ctx<D, F8, V> &x, const FwdParams &p, int t) {
+  using C = Sm100Cfg<D, F8, V>;
   const int r = threadIdx.x & 127;
   const uint32_t lane_base = static_cast<uint32_t>((threadIdx.x >> 5) & 3) * 32u << 16;
   const uint32_t tS = x.tmem + lane_base + C::COL_S0 + 128 * t;
@@ -697,7 +704,7 @@ __device__ void role_softmax(const Sm100Ctx<D, F8, SK> &x, const FwdParams &p, i
     const int u = snake_unit(k, p.num_units);
     if (u == -2) break;
     if (u < 0) continue;
-    const Unit w = unit_at<D, F8, SK>(p, u);
+    const Unit w = unit_at<D, F8, V>(p, u);
     const int tile_row0 = w.row0 + t * C::BM;
     const int i = tile_row0 + r;  // this thread's query row
     const bool valid = i < w.q_rows;
@@ -923,10 +930,10 @@ __device__ void role_softmax(const Sm100Ctx<D, F8, SK> &x, const FwdParams &p, i
   }
 }
 
-template <int D, bool F8, bool SK>
+template <int D, bool F8, int V>
 __device__ __forceinline__ void fwd_kernel_body(const CUtensorMap *tm_q, const CUtensorMap *tm_k,
                                                 const CUtensorMap *tm_v, const FwdParams &p) {
-  using C = Sm100Cfg<D, F8, SK>;
+  using C = Sm100Cfg<D, F8, V>;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
@@ -934,7 +941,7 @@ __device__ __forceinline__ void fwd_kernel_body(const CUtensorMap *tm_q, const C
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
-  Sm100Ctx<D, F8, SK> x;
+  Sm100Ctx<D, F8, V> x;
   x.smem = base;
   x.abort_flag = reinterpret_cast<volatile int *>(smem + C::OFF_MISC + 4);
 
@@ -977,16 +984,16 @@ __device__ __forceinline__ void fwd_kernel_body(const CUtensorMap *tm_q, const C
   if (warp >= 8) {
     regs_decrease<C::REGS_CONTROL>();
     if (warp == 8) {
-      if (lane == 0) role_producer<D, F8, SK>(x, p, tm_q, tm_k, tm_v);
+      if (lane == 0) role_producer<D, F8, V>(x, p, tm_q, tm_k, tm_v);
     } else if (warp == 9) {
       if constexpr (C::TRIPLE)
-        role_mma_triple<D, F8, SK>(x, p);
+        role_mma_triple<D, F8, V>(x, p);
       else
-        role_mma_split<D, F8, SK>(x, p);
+        role_mma_split<D, F8, V>(x, p);
     }
   } else {
     regs_increase<C::REGS_SOFTMAX>();
-    role_softmax<D, F8, SK>(x, p, warp >> 2);
+    role_softmax<D, F8, V>(x, p, warp >> 2);
   }
   __syncwarp();
   tc_fence_before();
@@ -997,12 +1004,12 @@ __device__ __forceinline__ void fwd_kernel_body(const CUtensorMap *tm_q, const C
   }
 }
 
-template <int D, bool SK>
+template <int D, int V>
 __global__ void __launch_bounds__(Sm100Cfg<D>::THREADS, 1)
     fa_fwd_bf16_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
                              const __grid_constant__ CUtensorMap tm_k,
                              const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
-  fwd_kernel_body<D, false, SK>(&tm_q, &tm_k, &tm_v, p);
+  fwd_kernel_body<D, false, V>(&tm_q, &tm_k, &tm_v, p);
 }
 
 // FP8 E4M3 inputs (head dim 128); tm_v maps V^T.
@@ -1010,7 +1017,7 @@ __global__ void __launch_bounds__(Sm100Cfg<128, true>::THREADS, 1)
     fa_fwd_e4m3_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
                              const __grid_constant__ CUtensorMap tm_k,
                              const __grid_constant__ CUtensorMap tm_vt, const FwdParams p) {
-  fwd_kernel_body<128, true, false>(&tm_q, &tm_k, &tm_vt, p);
+  fwd_kernel_body<128, true, 0>(&tm_q, &tm_k, &tm_vt, p);
 }
 
 }  // namespace fa
